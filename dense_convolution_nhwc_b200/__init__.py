@@ -1,0 +1,27 @@
+"""B200 (sm_100a) NHWC convolution forward.
+
+The library itself is the C-ABI shared object built from ``csrc/`` (declared in
+``include/b200conv.h``); ``binding`` marshals arguments into it with ctypes and
+nothing else.  The binding is loaded on first use of one of its names, and
+loading fails loudly if the shared object has not been built: there is no CPU
+fallback.
+"""
+_BINDING_NAMES = frozenset({
+    # C-ABI entry points (same names as include/b200conv.h)
+    "conv2d_forward", "conv3d_forward", "conv2d_plan", "conv3d_plan",
+    "conv2d_plan_for_props", "conv3d_plan_for_props",
+    "conv2d_workspace_size", "conv3d_workspace_size", "conv_check",
+    "conv_status_string", "conv_device_props", "conv_accumulate",
+    # types and helpers
+    "ConvError", "Conv2dDesc", "Conv3dDesc", "ConvPlan", "ConvOptions", "DeviceProps",
+    "ALGO", "DTYPE", "STATUS", "library_path",
+    # torch conveniences
+    "conv2d", "conv3d", "plan2d", "plan3d",
+})
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(f"module 'dense_convolution_nhwc_b200' has no attribute {name!r}")
