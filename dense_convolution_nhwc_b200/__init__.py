@@ -14,7 +14,7 @@ _BINDING_NAMES = frozenset({
     "conv_status_string", "conv_device_props", "conv_accumulate",
     # types and helpers
     "ConvError", "Conv2dDesc", "Conv3dDesc", "ConvPlan", "ConvOptions", "DeviceProps",
-    "ALGO", "DTYPE", "STATUS", "library_path",
+    "ALGO", "DTYPE", "STATUS", "ENGINE", "library_path", "make_desc2d", "make_desc3d", "make_options",
     # torch conveniences
     "conv2d", "conv3d", "plan2d", "plan3d",
 })

@@ -1,0 +1,570 @@
+// api.cu -- the C ABI: validation, the algorithm selector, and dispatch.
+//
+// Selector ("Bound winograd conv2d working set by tiling the batch", Problem
+// and Fix; maintainer review: dispatch never depends on current memory):
+//   * Winograd is considered for 3x3, stride 1, dilation 1 convs that meet
+//     the page's channel rule C % 32 == 0 && O % 32 == 0 && C + O >= 256, for
+//     fp32 inputs (16-bit inputs take the tensor-core implicit GEMM unless
+//     Winograd is forced: on B200 the unfused transforms' HBM traffic costs
+//     more than the tensor cores save).
+//   * The batch is cut into tiles of nb images, nb = floor(budget /
+//     per-image scratch), budget = min(3/4 * total device memory - (input +
+//     output + transformed filter), 8 GiB).  nb = 0, or tiles carrying fewer
+//     GEMM rows than one wave of 128-row tiles per SM, fall back to the
+//     scratch-free implicit GEMM.  A forced tile size is capped by nb.
+//   * Everything is a pure function of (shape, dtype, constant device
+//     properties, options); the environment hooks are read before selection.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+
+namespace b200conv {
+namespace {
+
+__device__ int g_error_word;
+
+constexpr long long kWinogradCap = 8LL << 30;   // 8 GiB: the GPU is shared
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  conv_device_props_t props{};
+  int* err_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+conv_status_t device_state(int dev, DeviceState** out) {
+  if (dev < 0 || dev >= kMaxDevices) return CONV_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return CONV_ERR_CUDA;
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return CONV_ERR_CUDA;
+    d.props.sm_count = p.multiProcessorCount;
+    d.props.cc_major = p.major;
+    d.props.cc_minor = p.minor;
+    d.props.total_global_mem = (unsigned long long)p.totalGlobalMem;
+    if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return CONV_ERR_CUDA;
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_error_word);
+    if (e == cudaSuccess) e = cudaMemset(addr, 0, sizeof(int));
+    if (cur != dev) cudaSetDevice(cur);
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    d.err_word = static_cast<int*>(addr);
+    d.ready = true;
+  }
+  *out = &d;
+  return CONV_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+long long out_extent(long long in, int k, int s, int p, int d) {
+  return (in + 2LL * p - (long long)d * (k - 1) - 1) / s + 1;
+}
+
+// ----------------------------- options ---------------------------------------
+
+conv_options_t effective_options(const conv_options_t* opts) {
+  if (opts) return *opts;
+  conv_options_t o{CONV_ALGO_AUTO, -1, 0};
+  if (const char* a = std::getenv("B200CONV_ALGO")) {
+    std::string s(a);
+    if (s == "implicit") o.algo = CONV_ALGO_IMPLICIT_GEMM;
+    else if (s == "winograd") o.algo = CONV_ALGO_WINOGRAD;
+    else if (s == "direct") o.algo = CONV_ALGO_DIRECT;
+  }
+  if (const char* b = std::getenv("B200CONV_WINOGRAD_WORKSPACE_BYTES")) o.winograd_budget_bytes = std::atoll(b);
+  if (const char* t = std::getenv("B200CONV_WINOGRAD_TILE_BATCH")) o.winograd_tile_batch = std::atoi(t);
+  return o;
+}
+
+// ----------------------------- validation ------------------------------------
+
+bool valid_dtype(conv_dtype_t t) { return t == CONV_F32 || t == CONV_F16 || t == CONV_BF16; }
+
+conv_status_t geom2d(const conv2d_desc_t* d, Geom* g) {
+  if (!d) return CONV_ERR_INVALID;
+  if (d->n < 0 || d->h <= 0 || d->w <= 0 || d->c <= 0 || d->o <= 0 || d->kh <= 0 || d->kw <= 0)
+    return CONV_ERR_INVALID;
+  for (int i = 0; i < 2; ++i)
+    if (d->stride[i] <= 0 || d->dilation[i] <= 0 || d->pad[i] < 0) return CONV_ERR_INVALID;
+  long long oh = out_extent(d->h, d->kh, d->stride[0], d->pad[0], d->dilation[0]);
+  long long ow = out_extent(d->w, d->kw, d->stride[1], d->pad[1], d->dilation[1]);
+  if (oh <= 0 || ow <= 0 || oh > (1 << 30) || ow > (1 << 30)) return CONV_ERR_INVALID;
+  g->n = d->n; g->h = d->h; g->w = d->w; g->c = d->c; g->o = d->o; g->kh = d->kh; g->kw = d->kw;
+  g->sh = d->stride[0]; g->sw = d->stride[1];
+  g->ph = d->pad[0]; g->pw = d->pad[1];
+  g->dh = d->dilation[0]; g->dw = d->dilation[1];
+  g->oh = (int)oh; g->ow = (int)ow;
+  g->in_img_stride = (long long)d->h * d->w * d->c;
+  g->w_row_stride = (long long)d->kh * d->kw * d->c;
+  g->out_img_stride = oh * ow * d->o;
+  return CONV_OK;
+}
+
+// ------------------------------- selector ------------------------------------
+
+struct Sel {
+  conv_algo_t algo = CONV_ALGO_IMPLICIT_GEMM;
+  conv_engine_t engine = CONV_ENGINE_SIMT;
+  int tile_m = 128, tile_n = 128;
+  int wino_m = 0, nb = 0, ntiles = 0, cpad = 0;
+  conv_dtype_t wino_store = CONV_F32;
+  size_t ws = 0;
+};
+
+bool winograd_shape(const Geom& g) {
+  return g.kh == 3 && g.kw == 3 && g.sh == 1 && g.sw == 1 && g.dh == 1 && g.dw == 1;
+}
+bool winograd_channel_rule(const Geom& g) {
+  return g.c % 32 == 0 && g.o % 32 == 0 && g.c + g.o >= 256;
+}
+int winograd_m_for(conv_dtype_t dt) { return dt == CONV_F32 ? 6 : 2; }
+
+// The tensor-core engine can express this shape (pointer alignment is checked at launch).
+bool tc_shape_ok(const Geom& g, conv_dtype_t dt, const conv_device_props_t& p) {
+  if (dt == CONV_F32 || p.cc_major != 10) return false;
+  if (g.sh > 8 || g.sw > 8) return false;
+  const int uw = g.pw - g.dw * (g.kw - 1), uh = g.ph - g.dh * (g.kh - 1);
+  if (g.pw > 128 || g.ph > 128 || uw < -128 || uw > 127 || uh < -128 || uh > 127) return false;
+  if ((long long)g.dw * (g.kw - 1) > 65535 || (long long)g.dh * (g.kh - 1) > 65535) return false;
+  return true;
+}
+
+int tc_tile_n(const Geom& g, const conv_device_props_t& p) {
+  if (g.o <= 128) return 128;
+  long long m_tiles = ((long long)g.n * g.oh * g.ow + 127) / 128;
+  long long tiles256 = m_tiles * ((g.o + 255) / 256);
+  return tiles256 < p.sm_count ? 128 : 256;
+}
+
+void winograd_sizes(const Geom& g, conv_dtype_t store, int m, size_t* u_bytes, size_t* per_img) {
+  const int a = m + 2;
+  const long long tiles = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+  const int esz = dtype_size(store);
+  *u_bytes = align256((size_t)a * a * g.o * g.c * esz);
+  *per_img = (size_t)a * a * tiles * ((size_t)g.c * esz + (size_t)g.o * 4);
+}
+
+conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t& p,
+                       const conv_options_t& o, Sel* s) {
+  const int esz = dtype_size(dt);
+  const bool wshape = winograd_shape(g);
+  bool want_wino = false;
+  if (o.algo == CONV_ALGO_WINOGRAD) {
+    if (!wshape) return CONV_ERR_UNSUPPORTED;
+    want_wino = true;
+  } else if (o.algo == CONV_ALGO_AUTO) {
+    want_wino = wshape && winograd_channel_rule(g) && dt == CONV_F32;
+  } else if (o.algo != CONV_ALGO_IMPLICIT_GEMM && o.algo != CONV_ALGO_DIRECT) {
+    return CONV_ERR_INVALID;
+  }
+
+  if (want_wino && g.n > 0) {
+    const int m = winograd_m_for(dt);
+    // 16-bit operands go to the tensor cores when their rows meet the
+    // 16-byte rule, else the transforms store fp32 for the FFMA engine.
+    const bool tc_gemm = dt != CONV_F32 && p.cc_major == 10 && g.c % 8 == 0;
+    const conv_dtype_t store = (dt == CONV_F32 || !tc_gemm) ? CONV_F32 : dt;
+    size_t u_bytes, per_img;
+    winograd_sizes(g, store, m, &u_bytes, &per_img);
+    const long long tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+    long long budget;
+    if (o.winograd_budget_bytes >= 0) {
+      budget = o.winograd_budget_bytes;
+    } else {
+      const long long own = (long long)g.n * g.h * g.w * g.c * esz + (long long)g.n * g.oh * g.ow * g.o * esz +
+                            (long long)u_bytes;
+      budget = std::min((long long)(p.total_global_mem / 4 * 3) - own, kWinogradCap);
+    }
+    long long nb = budget > 0 ? budget / (long long)per_img : 0;
+    nb = std::min<long long>(nb, g.n);
+    const bool forced_tile = o.winograd_tile_batch > 0;
+    if (forced_tile) nb = std::min<long long>(nb, o.winograd_tile_batch);
+    const long long r_min = (long long)p.sm_count * 128;
+    bool fallback = nb <= 0 || (!forced_tile && nb < g.n && nb * tiles_per_img < r_min);
+    if (fallback && o.algo == CONV_ALGO_WINOGRAD) return CONV_ERR_UNSUPPORTED;
+    if (!fallback) {
+      s->algo = CONV_ALGO_WINOGRAD;
+      s->engine = tc_gemm ? CONV_ENGINE_TCGEN05 : CONV_ENGINE_SIMT;
+      s->wino_m = m;
+      s->wino_store = store;
+      s->nb = (int)nb;
+      s->ntiles = (int)((g.n + nb - 1) / nb);
+      s->tile_m = 128;
+      s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : (g.o <= 64 ? 64 : g.o <= 96 ? 96 : 128);
+      const long long t_tile = nb * tiles_per_img;
+      const int a2 = (m + 2) * (m + 2);
+      s->ws = u_bytes + align256((size_t)a2 * t_tile * g.c * dtype_size(store)) +
+              align256((size_t)a2 * t_tile * g.o * 4);
+      s->cpad = 0;
+      return CONV_OK;
+    }
+  }
+
+  // Implicit GEMM (or the direct SIMT path).
+  s->algo = o.algo == CONV_ALGO_DIRECT ? CONV_ALGO_DIRECT : CONV_ALGO_IMPLICIT_GEMM;
+  s->wino_m = 0;
+  s->nb = g.n;
+  s->ntiles = 1;
+  s->cpad = 0;
+  s->ws = 0;
+  if (s->algo == CONV_ALGO_IMPLICIT_GEMM && tc_shape_ok(g, dt, p)) {
+    s->engine = CONV_ENGINE_TCGEN05;
+    s->tile_m = 128;
+    s->tile_n = tc_tile_n(g, p);
+    if (g.c % 8 != 0) {
+      const int cp = (g.c + 7) / 8 * 8;
+      s->cpad = cp;
+      s->ws = align256((size_t)g.n * g.h * g.w * cp * esz) + align256((size_t)g.o * g.kh * g.kw * cp * esz);
+    }
+  } else {
+    s->engine = CONV_ENGINE_SIMT;
+    s->tile_m = 128;
+    s->tile_n = g.o <= 64 ? 64 : (g.o <= 96 ? 96 : 128);
+  }
+  return CONV_OK;
+}
+
+void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
+  plan->algo = s.algo;
+  plan->engine = s.engine;
+  plan->tile_m = s.tile_m;
+  plan->tile_n = s.tile_n;
+  plan->winograd_m = s.wino_m;
+  plan->batch_tile = s.nb;
+  plan->num_batch_tiles = s.ntiles;
+  plan->channel_pad = s.cpad;
+  plan->taps = taps;
+  plan->workspace_bytes = ws;
+}
+
+// ------------------------------- execution -----------------------------------
+
+conv_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CONV_OK : CONV_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Run one planned 2D conv.  ws holds at least s.ws bytes.
+conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt, const Sel& s,
+                    void* ws, const DeviceState& d, cudaStream_t st) {
+  if (g.n == 0) return CONV_OK;
+  if (s.algo == CONV_ALGO_WINOGRAD) {
+    const int m = s.wino_m, a2 = (m + 2) * (m + 2);
+    const long long tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+    size_t u_bytes, per_img;
+    winograd_sizes(g, s.wino_store, m, &u_bytes, &per_img);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    void* u = base;
+    void* v = base + u_bytes;
+    float* mb = reinterpret_cast<float*>(
+        base + u_bytes + align256((size_t)a2 * s.nb * tiles_per_img * g.c * dtype_size(s.wino_store)));
+    cudaError_t e = launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    for (int n0 = 0; n0 < g.n; n0 += s.nb) {
+      const int nbi = std::min(s.nb, g.n - n0);
+      const long long t = (long long)nbi * tiles_per_img;
+      e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
+      if (e != cudaSuccess) return CONV_ERR_CUDA;
+      BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb};
+      if (s.engine == CONV_ENGINE_TCGEN05)
+        e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
+      else
+        e = launch_simt_batched_gemm(bg, st);
+      if (e != cudaSuccess) return CONV_ERR_CUDA;
+      e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, false, st);
+      if (e != cudaSuccess) return CONV_ERR_CUDA;
+    }
+    return CONV_OK;
+  }
+  if (s.engine == CONV_ENGINE_TCGEN05) {
+    if (s.cpad) {
+      uint8_t* base = static_cast<uint8_t*>(ws);
+      const int esz = dtype_size(dt);
+      void* pin = base;
+      void* pw = base + align256((size_t)g.n * g.h * g.w * s.cpad * esz);
+      cudaError_t e = launch_channel_pad(in, g.n, (long long)g.h * g.w, g.c, g.in_img_stride, pin, s.cpad, dt, st);
+      if (e == cudaSuccess)
+        e = launch_channel_pad(w, g.o, (long long)g.kh * g.kw, g.c, g.w_row_stride, pw, s.cpad, dt, st);
+      if (e != cudaSuccess) return CONV_ERR_CUDA;
+      Geom gp = g;
+      gp.c = s.cpad;
+      gp.in_img_stride = (long long)g.h * g.w * s.cpad;
+      gp.w_row_stride = (long long)g.kh * g.kw * s.cpad;
+      return cuda_status(launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, st));
+    }
+    if (tc_conv_supported(g, dt, in, w))
+      return cuda_status(launch_tc_conv(in, w, out, g, dt, s.tile_n, d.props.sm_count, d.err_word, st));
+    // Misaligned pointers: the any-alignment path below.
+  }
+  const bool vec = s.algo != CONV_ALGO_DIRECT && g.c % 4 == 0 &&
+                   (g.in_img_stride % 4 == 0) && (g.w_row_stride % 4 == 0) &&
+                   aligned16(in) && aligned16(w);
+  return cuda_status(launch_simt_conv(in, w, out, g, dt, vec, false, st));
+}
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  if (!a || !b || an == 0 || bn == 0) return false;
+  uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bn && y < x + an;
+}
+
+// ------------------------------- conv3d --------------------------------------
+
+struct Tap {
+  int kd, od_lo, od_hi, id_lo;   // output frames od_lo..od_hi read input frame id_lo + (od - od_lo) * sd
+};
+
+conv_status_t geom3d(const conv3d_desc_t* d, long long* od, Geom* g2) {
+  if (!d) return CONV_ERR_INVALID;
+  if (d->n < 0 || d->d <= 0 || d->h <= 0 || d->w <= 0 || d->c <= 0 || d->o <= 0 || d->kd <= 0 || d->kh <= 0 ||
+      d->kw <= 0)
+    return CONV_ERR_INVALID;
+  for (int i = 0; i < 3; ++i)
+    if (d->stride[i] <= 0 || d->dilation[i] <= 0 || d->pad[i] < 0) return CONV_ERR_INVALID;
+  *od = out_extent(d->d, d->kd, d->stride[0], d->pad[0], d->dilation[0]);
+  if (*od <= 0 || *od > (1 << 30)) return CONV_ERR_INVALID;
+  // The 2D problem of one depth tap: "images" are output frames.
+  conv2d_desc_t d2{};
+  d2.n = (int)*od; d2.h = d->h; d2.w = d->w; d2.c = d->c; d2.o = d->o; d2.kh = d->kh; d2.kw = d->kw;
+  d2.stride[0] = d->stride[1]; d2.stride[1] = d->stride[2];
+  d2.pad[0] = d->pad[1]; d2.pad[1] = d->pad[2];
+  d2.dilation[0] = d->dilation[1]; d2.dilation[1] = d->dilation[2];
+  conv_status_t st = geom2d(&d2, g2);
+  if (st != CONV_OK) return st;
+  g2->in_img_stride = (long long)d->stride[0] * d->h * d->w * d->c;            // frame view stride
+  g2->w_row_stride = (long long)d->kd * d->kh * d->kw * d->c;                  // weight slice rows
+  return CONV_OK;
+}
+
+int taps3d(const conv3d_desc_t* d, long long od, Tap* taps) {
+  int n = 0;
+  for (int kd = 0; kd < d->kd; ++kd) {
+    const long long off = (long long)kd * d->dilation[0] - d->pad[0];   // id = od*sd + off
+    long long lo = off >= 0 ? 0 : (-off + d->stride[0] - 1) / d->stride[0];
+    long long hi = (d->d - 1 - off) >= 0 ? (d->d - 1 - off) / d->stride[0] : -1;
+    hi = std::min(hi, od - 1);
+    if (lo > hi) continue;
+    taps[n++] = Tap{kd, (int)lo, (int)hi, (int)(lo * d->stride[0] + off)};
+  }
+  return n;
+}
+
+conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_device_props_t& p,
+                          const conv_options_t& o, Sel* s, Geom* g2, long long* od, size_t* ws_total,
+                          size_t* tap_bytes) {
+  if (!valid_dtype(dt)) return CONV_ERR_INVALID;
+  conv_status_t st = geom3d(d, od, g2);
+  if (st != CONV_OK) return st;
+  st = select2d(*g2, dt, p, o, s);
+  if (st != CONV_OK) return st;
+  // Scratch for the taps that are added (all but a first tap that covers every frame).
+  *tap_bytes = d->kd > 1 || d->pad[0] > 0 ? align256((size_t)*od * g2->oh * g2->ow * g2->o * dtype_size(dt)) : 0;
+  *ws_total = *tap_bytes + s->ws;
+  return CONV_OK;
+}
+
+}  // namespace
+}  // namespace b200conv
+
+using namespace b200conv;
+
+extern "C" {
+
+const char* conv_status_string(conv_status_t s) {
+  switch (s) {
+    case CONV_OK: return "ok";
+    case CONV_ERR_INVALID: return "invalid argument";
+    case CONV_ERR_UNSUPPORTED: return "unsupported by the requested algorithm";
+    case CONV_ERR_ALIGNMENT: return "misaligned pointer";
+    case CONV_ERR_WORKSPACE: return "workspace too small";
+    case CONV_ERR_CUDA: return "CUDA error";
+    case CONV_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+conv_status_t conv_device_props(int device, conv_device_props_t* props) {
+  if (!props) return CONV_ERR_INVALID;
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(device, &d);
+  if (st != CONV_OK) return st;
+  *props = d->props;
+  return CONV_OK;
+}
+
+conv_status_t conv2d_plan_for_props(const conv2d_desc_t* desc, conv_dtype_t dtype, const conv_device_props_t* props,
+                                    const conv_options_t* opts, conv_plan_t* plan) {
+  if (!props || !plan || !valid_dtype(dtype)) return CONV_ERR_INVALID;
+  Geom g;
+  conv_status_t st = geom2d(desc, &g);
+  if (st != CONV_OK) return st;
+  Sel s;
+  st = select2d(g, dtype, *props, effective_options(opts), &s);
+  if (st != CONV_OK) return st;
+  fill_plan(s, plan, 1, s.ws);
+  return CONV_OK;
+}
+
+conv_status_t conv2d_plan(const conv2d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts,
+                          conv_plan_t* plan) {
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(device, &d);
+  if (st != CONV_OK) return st;
+  return conv2d_plan_for_props(desc, dtype, &d->props, opts, plan);
+}
+
+size_t conv2d_workspace_size(const conv2d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts) {
+  conv_plan_t p;
+  return conv2d_plan(desc, dtype, device, opts, &p) == CONV_OK ? p.workspace_bytes : 0;
+}
+
+conv_status_t conv2d_forward(const void* in, const void* w, void* out, const conv2d_desc_t* desc, conv_dtype_t dtype,
+                             const conv_options_t* opts, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return CONV_ERR_INVALID;
+  Geom g;
+  conv_status_t st = geom2d(desc, &g);
+  if (st != CONV_OK) return st;
+  if (g.n == 0) return CONV_OK;
+  if (!in || !w || !out) return CONV_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+  DeviceState* d = nullptr;
+  st = device_state(dev, &d);
+  if (st != CONV_OK) return st;
+  Sel s;
+  st = select2d(g, dtype, d->props, effective_options(opts), &s);
+  if (st != CONV_OK) return st;
+  if (workspace_bytes < s.ws || (s.ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
+  const int esz = dtype_size(dtype);
+  const size_t out_bytes = (size_t)g.n * g.out_img_stride * esz;
+  if (overlaps(out, out_bytes, in, (size_t)g.n * g.in_img_stride * esz) ||
+      overlaps(out, out_bytes, w, (size_t)g.o * g.w_row_stride * esz) ||
+      overlaps(out, out_bytes, workspace, s.ws))
+    return CONV_ERR_INVALID;
+  return run2d(in, w, out, g, dtype, s, workspace, *d, static_cast<cudaStream_t>(stream));
+}
+
+conv_status_t conv3d_plan_for_props(const conv3d_desc_t* desc, conv_dtype_t dtype, const conv_device_props_t* props,
+                                    const conv_options_t* opts, conv_plan_t* plan) {
+  if (!props || !plan) return CONV_ERR_INVALID;
+  Sel s;
+  Geom g2;
+  long long od;
+  size_t ws, tap_bytes;
+  conv_status_t st = plan3d_impl(desc, dtype, *props, effective_options(opts), &s, &g2, &od, &ws, &tap_bytes);
+  if (st != CONV_OK) return st;
+  fill_plan(s, plan, desc->kd, ws);
+  return CONV_OK;
+}
+
+conv_status_t conv3d_plan(const conv3d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts,
+                          conv_plan_t* plan) {
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(device, &d);
+  if (st != CONV_OK) return st;
+  return conv3d_plan_for_props(desc, dtype, &d->props, opts, plan);
+}
+
+size_t conv3d_workspace_size(const conv3d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts) {
+  conv_plan_t p;
+  return conv3d_plan(desc, dtype, device, opts, &p) == CONV_OK ? p.workspace_bytes : 0;
+}
+
+conv_status_t conv3d_forward(const void* in, const void* w, void* out, const conv3d_desc_t* desc, conv_dtype_t dtype,
+                             const conv_options_t* opts, void* workspace, size_t workspace_bytes, void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(dev, &d);
+  if (st != CONV_OK) return st;
+  Sel s;
+  Geom g2;
+  long long od;
+  size_t ws, tap_bytes;
+  st = plan3d_impl(desc, dtype, d->props, effective_options(opts), &s, &g2, &od, &ws, &tap_bytes);
+  if (st != CONV_OK) return st;
+  if (desc->n == 0) return CONV_OK;
+  if (!in || !w || !out) return CONV_ERR_INVALID;
+  if (workspace_bytes < ws || (ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
+  const int esz = dtype_size(dtype);
+  const long long frame_in = (long long)desc->h * desc->w * desc->c;
+  const long long frame_out = (long long)g2.oh * g2.ow * g2.o;
+  const size_t out_bytes = (size_t)desc->n * od * frame_out * esz;
+  if (overlaps(out, out_bytes, in, (size_t)desc->n * desc->d * frame_in * esz) ||
+      overlaps(out, out_bytes, w, (size_t)desc->o * g2.w_row_stride * esz) ||
+      overlaps(out, out_bytes, workspace, ws))
+    return CONV_ERR_INVALID;
+
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  Tap taps[1024];
+  if (desc->kd > 1024) return CONV_ERR_UNSUPPORTED;
+  const int ntaps = taps3d(desc, od, taps);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  void* tap_buf = tap_bytes ? wsb : nullptr;
+  void* ws2 = tap_bytes ? wsb + tap_bytes : workspace;
+  const bool first_covers_all = ntaps > 0 && taps[0].od_lo == 0 && taps[0].od_hi == od - 1;
+
+  for (int n = 0; n < desc->n; ++n) {
+    const uint8_t* in_n = static_cast<const uint8_t*>(in) + (size_t)n * desc->d * frame_in * esz;
+    uint8_t* out_n = static_cast<uint8_t*>(out) + (size_t)n * od * frame_out * esz;
+    if (!first_covers_all) {
+      if (launch_fill_zero(out_n, (size_t)od * frame_out * esz, st_) != cudaSuccess) return CONV_ERR_CUDA;
+    }
+    for (int i = 0; i < ntaps; ++i) {
+      const Tap& t = taps[i];
+      Geom g = g2;
+      g.n = t.od_hi - t.od_lo + 1;
+      const void* in_view = in_n + (size_t)t.id_lo * frame_in * esz;
+      const void* w_slice = static_cast<const uint8_t*>(w) + (size_t)t.kd * desc->kh * desc->kw * desc->c * esz;
+      uint8_t* out_view = out_n + (size_t)t.od_lo * frame_out * esz;
+      const bool direct_write = i == 0 && first_covers_all;
+      void* dst = direct_write ? static_cast<void*>(out_view) : tap_buf;
+      st = run2d(in_view, w_slice, dst, g, dtype, s, ws2, *d, st_);
+      if (st != CONV_OK) return st;
+      if (!direct_write) {
+        if (launch_accumulate(out_view, tap_buf, (size_t)g.n * frame_out, dtype, st_) != cudaSuccess)
+          return CONV_ERR_CUDA;
+      }
+    }
+  }
+  return CONV_OK;
+}
+
+conv_status_t conv_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dtype, void* stream) {
+  if (!valid_dtype(dtype)) return CONV_ERR_INVALID;
+  if (count == 0) return CONV_OK;
+  if (!out || !tap) return CONV_ERR_INVALID;
+  const size_t bytes = count * dtype_size(dtype);
+  if (overlaps(out, bytes, tap, bytes)) return CONV_ERR_INVALID;
+  return cuda_status(launch_accumulate(out, tap, count, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+conv_status_t conv_check(void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(dev, &d);
+  if (st != CONV_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return CONV_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, d->err_word, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return CONV_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(d->err_word, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return CONV_ERR_CUDA;
+    return CONV_ERR_TIMEOUT;
+  }
+  return CONV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+// elementwise.cu -- bandwidth-bound helpers around the GEMM cores.
+//
+//  * accumulate: out[i] = round(out[i] + tap[i]), the in-place add that sums a
+//    conv3d's depth taps ("Decompose small kernel-depth 3D convs into 2D
+//    convs", Change and Open questions 1).  fp32 add, one rounding to the
+//    storage dtype; 16-byte vector accesses when both pointers allow it.
+//  * channel pad: copies NHWC (or OHWI) rows of C channels into rows of Cp
+//    channels with zeros after C, so that rows meet the tensor-memory-access
+//    16-byte stride rule (e.g. a 3-channel stem).
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace b200conv {
+namespace {
+
+template <typename T>
+__global__ void accumulate_vec_kernel(T* __restrict__ out, const T* __restrict__ tap, size_t nvec) {
+  constexpr int E = 16 / sizeof(T);
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (; i < nvec; i += stride) {
+    uint4 a = reinterpret_cast<const uint4*>(out)[i];
+    uint4 b = __ldg(reinterpret_cast<const uint4*>(tap) + i);
+    T* pa = reinterpret_cast<T*>(&a);
+    const T* pb = reinterpret_cast<const T*>(&b);
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      pa[e] = Store<T>::from_f32(Store<T>::to_f32(pa[e]) + Store<T>::to_f32(pb[e]));
+    reinterpret_cast<uint4*>(out)[i] = a;
+  }
+}
+
+template <typename T>
+__global__ void accumulate_scalar_kernel(T* __restrict__ out, const T* __restrict__ tap, size_t n) {
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (; i < n; i += stride)
+    out[i] = Store<T>::from_f32(Store<T>::to_f32(out[i]) + Store<T>::to_f32(tap[i]));
+}
+
+template <typename T>
+cudaError_t accumulate_typed(void* out, const void* tap, size_t count, cudaStream_t s) {
+  constexpr int E = 16 / sizeof(T);
+  T* o = static_cast<T*>(out);
+  const T* t = static_cast<const T*>(tap);
+  const bool aligned = ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(tap)) & 15) == 0;
+  size_t nvec = aligned ? count / E : 0;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const unsigned cap = (unsigned)sms * 8;
+  if (nvec > 0) {
+    unsigned blocks = (unsigned)((nvec + 255) / 256 < cap ? (nvec + 255) / 256 : cap);
+    accumulate_vec_kernel<T><<<blocks, 256, 0, s>>>(o, t, nvec);
+  }
+  size_t done = nvec * E;
+  if (done < count) {
+    size_t rest = count - done;
+    unsigned blocks = (unsigned)((rest + 255) / 256 < cap ? (rest + 255) / 256 : cap);
+    accumulate_scalar_kernel<T><<<blocks, 256, 0, s>>>(o + done, t + done, rest);
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+__global__ void channel_pad_kernel(const T* __restrict__ src, long long outer, long long inner, int c,
+                                   long long src_outer_stride, T* __restrict__ dst, int cp) {
+  const long long total = outer * inner * cp;
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (; i < total; i += stride) {
+    long long row = i / cp;
+    int ch = (int)(i - row * cp);
+    long long a = row / inner, b = row - a * inner;
+    dst[i] = ch < c ? src[a * src_outer_stride + b * c + ch] : Store<T>::from_f32(0.0f);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dt,
+                              cudaStream_t s) {
+  if (count == 0) return cudaSuccess;
+  switch (dt) {
+    case CONV_F32: return accumulate_typed<float>(out, tap, count, s);
+    case CONV_F16: return accumulate_typed<__half>(out, tap, count, s);
+    case CONV_BF16: return accumulate_typed<__nv_bfloat16>(out, tap, count, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fill_zero(void* out, size_t bytes, cudaStream_t s) {
+  if (bytes == 0) return cudaSuccess;
+  return cudaMemsetAsync(out, 0, bytes, s);
+}
+
+cudaError_t launch_channel_pad(const void* src, long long outer, long long inner, int c,
+                               long long src_outer_stride, void* dst, int cp, conv_dtype_t dt,
+                               cudaStream_t s) {
+  long long total = outer * inner * cp;
+  if (total == 0) return cudaSuccess;
+  unsigned blocks = (unsigned)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
+  switch (dt) {
+    case CONV_F32:
+      channel_pad_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(src), outer, inner, c,
+                                                       src_outer_stride, static_cast<float*>(dst), cp);
+      break;
+    case CONV_F16:
+      channel_pad_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(src), outer, inner, c,
+                                                        src_outer_stride, static_cast<__half*>(dst), cp);
+      break;
+    case CONV_BF16:
+      channel_pad_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+          static_cast<const __nv_bfloat16*>(src), outer, inner, c, src_outer_stride,
+          static_cast<__nv_bfloat16*>(dst), cp);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace b200conv

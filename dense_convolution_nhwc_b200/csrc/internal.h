@@ -1,0 +1,85 @@
+// internal.h -- declarations shared by the library's translation units.
+// Nothing here is part of the C ABI (include/b200conv.h is).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/b200conv.h"
+
+namespace b200conv {
+
+// Device-side error codes written to the per-device error word.
+enum DevErr : int {
+  DEVERR_NONE = 0,
+  DEVERR_TIMEOUT_PRODUCER = 0x101,   // TMA producer waited too long for a free stage
+  DEVERR_TIMEOUT_MMA_FULL = 0x102,   // MMA issuer waited too long for a loaded stage
+  DEVERR_TIMEOUT_MMA_TMEM = 0x103,   // MMA issuer waited too long for a drained accumulator
+  DEVERR_TIMEOUT_EPILOGUE = 0x104,   // epilogue waited too long for a finished accumulator
+};
+
+inline int dtype_size(conv_dtype_t t) { return t == CONV_F32 ? 4 : 2; }
+
+// One 2D convolution as the kernels see it.  The "batch" of a 2D conv is
+// n images whose starts are in_img_stride elements apart (a conv3d depth tap
+// passes frame views with stride sd*H*W*C); the weights are O rows of
+// KH*KW*C elements, w_row_stride apart (KD*KH*KW*C for a depth-tap slice).
+struct Geom {
+  int n, h, w, c, o, kh, kw;
+  int sh, sw, ph, pw, dh, dw;
+  int oh, ow;
+  long long in_img_stride;    // elements
+  long long w_row_stride;     // elements
+  long long out_img_stride;   // elements (OH*OW*O for a dense NHWC output)
+};
+
+// Batched GEMM view used by the Winograd path: for b < batches,
+//   D_b[t][o] = sum_c A_b[t][c] * B_b[o][c]   (A: [batches][T][C], B: [batches][O][C])
+struct BatchedGemm {
+  int batches, t, c, o;
+  const void* a;        // [batches][T][C] in the input dtype (fp32 for the SIMT engine)
+  const void* b;        // [batches][O][C]
+  float* d;             // [batches][T][O] fp32
+};
+
+// ---- kernel launchers (return a CUDA error; never synchronise) ----
+
+// SIMT implicit GEMM (FFMA, fp32 accumulate): any dtype, any alignment when
+// vec == false.  accumulate: out = round(out + result).
+cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geom& g,
+                             conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s);
+// SIMT batched GEMM on fp32 operands (Winograd fp32 path).
+cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s);
+
+// tcgen05 implicit GEMM for 16-bit dtypes (TMA im2col staging, TMEM accumulators).
+// Returns cudaErrorNotSupported if the shape cannot be encoded as TMA maps.
+bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w);
+cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
+                           conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
+                           cudaStream_t s);
+// tcgen05 batched GEMM for 16-bit operands with fp32 D (Winograd 16-bit path).
+cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n,
+                                   int sm_count, int* err_word, cudaStream_t s);
+
+// Winograd transforms (fp32 arithmetic; V/U stored in `store_dt`).
+cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int c, int m,
+                               conv_dtype_t in_dt, conv_dtype_t store_dt, void* u, cudaStream_t s);
+cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int m,
+                              conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_tile,
+                              cudaStream_t s);
+cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb, int m,
+                               long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
+                               cudaStream_t s);
+
+// Elementwise helpers.
+cudaError_t launch_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dt,
+                              cudaStream_t s);
+cudaError_t launch_fill_zero(void* out, size_t bytes, cudaStream_t s);
+// Channel pad: dst[a][b][c'] = c' < c ? src[a*src_outer_stride + b*c + c'] : 0 for a < outer,
+// b < inner, c' < cp; dst is dense [outer][inner][cp].  Element strides.
+cudaError_t launch_channel_pad(const void* src, long long outer, long long inner, int c,
+                               long long src_outer_stride, void* dst, int cp, conv_dtype_t dt,
+                               cudaStream_t s);
+
+}  // namespace b200conv

@@ -1,0 +1,588 @@
+// tc_conv.cu -- implicit-GEMM convolution on the sm_100a tensor cores.
+//
+// The implicit GEMM of "Use the explicit gemm for wide convs on neural
+// accelerators" (description: im2col is never materialised), B200-first:
+//
+//   rows m = (n, oh, ow), columns o, reduction k = (kh, kw, c);
+//   A tile (128 pixels x 64 channels) of tap (kh, kw) is fetched by one TMA
+//   load in im2col mode: the tensor map walks 128 consecutive output pixels
+//   (stride sh/sw, wrapping rows and images inside the padded bounding box)
+//   and the per-tap offset (kw*dw, kh*dh) selects the filter tap; out-of-image
+//   pixels read as zero, so padding costs nothing.  The gather happens on the
+//   way into shared memory, in the 128-byte-swizzled K-major layout the MMA
+//   reads directly.
+//   B tile (BN weight rows x 64 channels) is a tiled TMA load of the OHWI
+//   weights viewed as [O][taps][C] (row stride = a conv3d slice's stride).
+//   tcgen05.mma (kind::f16, M = 128, N = BN, K = 16) accumulates in fp32 in
+//   tensor memory, double-buffered so the epilogue of one tile overlaps the
+//   main loop of the next.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0     TMA producer (one thread), multi-stage mbarrier ring
+//   warp 1     TMEM allocator + MMA issuer (one thread)
+//   warps 2-5  epilogue: tcgen05.ld -> round to the out dtype -> global
+//
+// Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that runs
+// out records a code in the device error word, raises a CTA-wide abort flag,
+// drains its own in-flight copies / MMAs (again bounded), frees TMEM and
+// returns, so a fault in the pipeline can never hang the GPU.
+//
+// The same kernel runs the Winograd batched GEMM (tiled TMA for A, fp32 D).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace b200conv {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 x 16-bit = one 128-byte swizzle row
+constexpr int THREADS = 192;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+template <int BN> struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+struct TcArgs {
+  int m_tiles, n_tiles, batches;
+  int kb_per_tap, taps;
+  int kw, dh, dw;
+  int oh, ow, sh, sw, ph, pw;
+  long long m_rows;            // rows per batch
+  int ocols;                   // output columns (O)
+  void* out;
+  long long ldo;               // elements between output rows
+  long long out_batch;         // elements between batches
+  int* err;
+};
+
+// ------------------------------- PTX wrappers -------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: true when the phase completed; false after the time limit or
+// when another role raised the abort flag.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* err, int code) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort_flag) return false;
+      if (gtimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        if (code) atomicCAS(err, 0, code);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_im2col_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                   int c, int w, int h, int n, uint16_t off_w,
+                                                   uint16_t off_h) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], {%7, %8};" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c), "r"(w), "r"(h), "r"(n), "h"(off_w),
+      "h"(off_h)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (SBO), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);   // start address
+  d |= (uint64_t)1 << 16;                    // leading-dimension byte offset (unused here)
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride-dimension byte offset
+  d |= (uint64_t)1 << 46;                    // descriptor version
+  d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 D, A and B both f16 (fmt 0) or
+// both bf16 (fmt 1), K-major, N = BN, M = 128.
+template <int BN>
+__host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt) {
+  return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+
+#define TMEM_LD32(taddr, r)                                                                        \
+  asm volatile(                                                                                    \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"              \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),       \
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),   \
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),             \
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),             \
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])              \
+      : "r"(taddr))
+
+// --------------------------------- kernel -----------------------------------
+
+template <int BN, bool IM2COL, typename TIn, typename TOut>
+__global__ void __launch_bounds__(THREADS, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcArgs a) {
+  using C = Cfg<BN>;
+  constexpr uint32_t IDESC = make_idesc<BN>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto tfull_bar = [&](int i) { return bar0 + 8u * (2 * C::STAGES + i); };
+  auto tempty_bar = [&](int i) { return bar0 + 8u * (2 * C::STAGES + 2 + i); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull_bar(i), 1);
+      mbar_init(tempty_bar(i), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const long long total_tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
+  const int ksteps = a.taps * a.kb_per_tap;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (long long tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int nt = (int)(tile % a.n_tiles);
+        const long long rest = tile / a.n_tiles;
+        const int mt = (int)(rest % a.m_tiles);
+        const int b = (int)(rest / a.m_tiles);
+        int img = 0, wx = 0, hy = 0;
+        if (IM2COL) {
+          const long long m0 = (long long)mt * BM;
+          const long long ohw = (long long)a.oh * a.ow;
+          img = (int)(m0 / ohw);
+          const int rem = (int)(m0 - (long long)img * ohw);
+          const int oy = rem / a.ow, ox = rem - (rem / a.ow) * a.ow;
+          wx = ox * a.sw - a.pw;
+          hy = oy * a.sh - a.ph;
+        }
+        for (int ks = 0; ks < ksteps; ++ks) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err, DEVERR_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          const int tap = ks / a.kb_per_tap;
+          const int kb = ks - tap * a.kb_per_tap;
+          const uint32_t fb = full_bar(stage);
+          mbar_expect_tx(fb, C::STAGE_BYTES);
+          const uint32_t dA = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t dB = smem_u32(sB + stage * C::B_BYTES);
+          if (IM2COL) {
+            const int ky = tap / a.kw, kx = tap - (tap / a.kw) * a.kw;
+            tma_load_im2col_4d(dA, &tmA, fb, kb * BK, wx, hy, img, (uint16_t)(kx * a.dw),
+                               (uint16_t)(ky * a.dh));
+            tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
+          } else {
+            tma_load_3d(dA, &tmA, fb, kb * BK, mt * BM, b);
+            tma_load_3d(dB, &tmB, fb, kb * BK, nt * BN, b);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: wait (bounded) until the last loads in flight have landed.
+      const int pending = issued < C::STAGES ? (int)issued : C::STAGES;
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < pending; ++i) {
+        if (--s < 0) {
+          s = C::STAGES - 1;
+          ph ^= 1u;
+        }
+        volatile int never = 0;
+        mbar_wait(full_bar(s), ph, &never, a.err, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (long long tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.err, DEVERR_TIMEOUT_MMA_TMEM)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, a.err, DEVERR_TIMEOUT_MMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t aa = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t bb = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            tc_mma(d_tmem, sdesc(aa + 32u * k), sdesc(bb + 32u * k), IDESC, (ks | k) != 0 ? 1u : 0u);
+          tc_commit(empty_bar(stage));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(tfull_bar(acc));
+      }
+      // Drain: all MMAs this thread issued have completed once this arrives.
+      tc_commit(drain_bar);
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never, a.err, 0);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------- epilogue --------------------------------
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (long long tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err, DEVERR_TIMEOUT_EPILOGUE)) break;
+      tc_fence_after();
+      const int nt = (int)(tile % a.n_tiles);
+      const long long rest = tile / a.n_tiles;
+      const int mt = (int)(rest % a.m_tiles);
+      const int b = (int)(rest / a.m_tiles);
+      const long long m = (long long)mt * BM + row;
+      const bool row_ok = m < a.m_rows;
+      TOut* orow = static_cast<TOut*>(a.out) + (long long)b * a.out_batch + (row_ok ? m : 0) * a.ldo;
+      const int n0 = nt * BN;
+#pragma unroll 1
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cc);
+        TMEM_LD32(taddr, r);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (!row_ok) continue;
+        const int c0 = n0 + cc;
+        if (c0 >= a.ocols) continue;
+        TOut* p = orow + c0;
+        const bool full = c0 + 32 <= a.ocols;
+        if constexpr (sizeof(TOut) == 4) {
+          if (full && ((reinterpret_cast<uintptr_t>(p) & 15) == 0)) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              float4 f = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+              reinterpret_cast<float4*>(p)[v] = f;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < a.ocols) p[j] = Store<TOut>::from_f32(__uint_as_float(r[j]));
+          }
+        } else {
+          if (full && ((reinterpret_cast<uintptr_t>(p) & 15) == 0)) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 u;
+              u.x = pack2<TOut>(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              u.y = pack2<TOut>(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              u.z = pack2<TOut>(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              u.w = pack2<TOut>(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              reinterpret_cast<uint4*>(p)[v] = u;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < a.ocols) p[j] = Store<TOut>::from_f32(__uint_as_float(r[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------- host side ----------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+PFN_cuTensorMapEncodeIm2col_v12000 g_encode_im2col = nullptr;
+
+bool driver_fns() {
+  static std::once_flag once;
+  static bool ok = false;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeIm2col", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      g_encode_im2col = reinterpret_cast<PFN_cuTensorMapEncodeIm2col_v12000>(p);
+    ok = g_encode_tiled && g_encode_im2col;
+  });
+  return ok;
+}
+
+CUtensorMapDataType tmap_dtype(conv_dtype_t dt) {
+  return dt == CONV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
+bool encode_3d(CUtensorMap* m, conv_dtype_t dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode_tiled(m, tmap_dtype(dt), 3, const_cast<void*>(base), dims, strides, box, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  // Per device; cheap enough to repeat, but cache the common case.
+  static thread_local int last_dev = -1;
+  static thread_local const void* last_k = nullptr;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (last_dev == dev && last_k == reinterpret_cast<const void*>(kernel)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) {
+    last_dev = dev;
+    last_k = reinterpret_cast<const void*>(kernel);
+  }
+  return e;
+}
+
+template <int BN, bool IM2COL, typename TIn, typename TOut>
+cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int sm_count,
+                          cudaStream_t s) {
+  auto k = tc_gemm_kernel<BN, IM2COL, TIn, TOut>;
+  cudaError_t e = set_smem(k, Cfg<BN>::SMEM);
+  if (e != cudaSuccess) return e;
+  long long tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
+  if (tiles == 0) return cudaSuccess;
+  int grid = (int)(tiles < sm_count ? tiles : sm_count);
+  k<<<grid, THREADS, Cfg<BN>::SMEM, s>>>(A, B, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w) {
+  if (dt == CONV_F32) return false;
+  if (!driver_fns()) return false;
+  if (g.c % 8 != 0) return false;                               // 16-byte row strides
+  if ((reinterpret_cast<uintptr_t>(in) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return false;
+  if ((g.in_img_stride * 2) % 16 || (g.w_row_stride * 2) % 16) return false;
+  if (g.sh > 8 || g.sw > 8) return false;                       // im2col traversal stride
+  const int lw = -g.pw, lh = -g.ph;
+  const int uw = g.pw - g.dw * (g.kw - 1), uh = g.ph - g.dh * (g.kh - 1);
+  if (lw < -128 || lh < -128 || uw < -128 || uw > 127 || uh < -128 || uh > 127) return false;
+  if ((long long)g.dw * (g.kw - 1) > 65535 || (long long)g.dh * (g.kh - 1) > 65535) return false;
+  if (g.n <= 0 || g.oh <= 0 || g.ow <= 0) return false;
+  if (g.out_img_stride != (long long)g.oh * g.ow * g.o) return false;
+  return true;
+}
+
+cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt,
+                           int tile_n, int sm_count, int* err_word, cudaStream_t s) {
+  if (!tc_conv_supported(g, dt, in, w)) return cudaErrorNotSupported;
+  const long long M = (long long)g.n * g.oh * g.ow;
+  if (M == 0) return cudaSuccess;
+  // A: im2col view of the NHWC input (C, W, H, N).
+  CUtensorMap tA, tB;
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)g.c, (cuuint64_t)g.w, (cuuint64_t)g.h, (cuuint64_t)g.n};
+    cuuint64_t strides[3] = {(cuuint64_t)g.c * 2, (cuuint64_t)g.w * g.c * 2, (cuuint64_t)g.in_img_stride * 2};
+    int lower[2] = {-g.pw, -g.ph};
+    int upper[2] = {g.pw - g.dw * (g.kw - 1), g.ph - g.dh * (g.kh - 1)};
+    cuuint32_t es[4] = {1, (cuuint32_t)g.sw, (cuuint32_t)g.sh, 1};
+    CUresult r = g_encode_im2col(&tA, tmap_dtype(dt), 4, const_cast<void*>(in), dims, strides, lower, upper,
+                                 BK, BM, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  // B: weights as (C, taps, O), row stride w_row_stride.
+  const int taps = g.kh * g.kw;
+  if (!encode_3d(&tB, dt, w, g.c, taps, g.o, (uint64_t)g.c * 2, (uint64_t)g.w_row_stride * 2, BK, 1,
+                 tile_n))
+    return cudaErrorInvalidValue;
+
+  TcArgs a{};
+  a.m_tiles = (int)((M + BM - 1) / BM);
+  a.n_tiles = (g.o + tile_n - 1) / tile_n;
+  a.batches = 1;
+  a.kb_per_tap = (g.c + BK - 1) / BK;
+  a.taps = taps;
+  a.kw = g.kw; a.dh = g.dh; a.dw = g.dw;
+  a.oh = g.oh; a.ow = g.ow; a.sh = g.sh; a.sw = g.sw; a.ph = g.ph; a.pw = g.pw;
+  a.m_rows = M;
+  a.ocols = g.o;
+  a.out = out;
+  a.ldo = g.o;
+  a.out_batch = 0;
+  a.err = err_word;
+  if (dt == CONV_BF16)
+    return tile_n == 256 ? launch_kernel<256, true, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, true, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
+  return tile_n == 256 ? launch_kernel<256, true, __half, __half>(tA, tB, a, sm_count, s)
+                       : launch_kernel<128, true, __half, __half>(tA, tB, a, sm_count, s);
+}
+
+cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n, int sm_count,
+                                   int* err_word, cudaStream_t s) {
+  if (dt == CONV_F32 || !driver_fns()) return cudaErrorNotSupported;
+  if (bg.c % 8 != 0 || (reinterpret_cast<uintptr_t>(bg.a) & 15) || (reinterpret_cast<uintptr_t>(bg.b) & 15))
+    return cudaErrorNotSupported;
+  if (bg.t == 0 || bg.batches == 0) return cudaSuccess;
+  CUtensorMap tA, tB;
+  if (!encode_3d(&tA, dt, bg.a, bg.c, bg.t, bg.batches, (uint64_t)bg.c * 2, (uint64_t)bg.t * bg.c * 2, BK,
+                 BM, 1))
+    return cudaErrorInvalidValue;
+  if (!encode_3d(&tB, dt, bg.b, bg.c, bg.o, bg.batches, (uint64_t)bg.c * 2, (uint64_t)bg.o * bg.c * 2, BK,
+                 tile_n, 1))
+    return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.m_tiles = (bg.t + BM - 1) / BM;
+  a.n_tiles = (bg.o + tile_n - 1) / tile_n;
+  a.batches = bg.batches;
+  a.kb_per_tap = (bg.c + BK - 1) / BK;
+  a.taps = 1;
+  a.kw = 1; a.dh = 1; a.dw = 1;
+  a.oh = 1; a.ow = bg.t; a.sh = 1; a.sw = 1; a.ph = 0; a.pw = 0;
+  a.m_rows = bg.t;
+  a.ocols = bg.o;
+  a.out = bg.d;
+  a.ldo = bg.o;
+  a.out_batch = (long long)bg.t * bg.o;
+  a.err = err_word;
+  if (dt == CONV_BF16)
+    return tile_n == 256 ? launch_kernel<256, false, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, false, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
+  return tile_n == 256 ? launch_kernel<256, false, __half, float>(tA, tB, a, sm_count, s)
+                       : launch_kernel<128, false, __half, float>(tA, tB, a, sm_count, s);
+}
+
+}  // namespace b200conv

@@ -1,0 +1,303 @@
+// winograd.cu -- Winograd F(m x m, 3 x 3) transforms for 3x3 stride-1 convs.
+//
+// The Winograd path of "Bound winograd conv2d working set by tiling the batch"
+// (Problem, Fix): input transform, batched GEMM, output transform.  With
+// alpha = m + 2 and T = N * ceil(OH/m) * ceil(OW/m) tiles,
+//   U[xi][o][c] = (G g_oc G^T)[xi]                      filter transform
+//   V[xi][t][c] = (B^T d_tc B)[xi]                      input transform
+//   M[xi][t][o] = sum_c V[xi][t][c] * U[xi][o][c]        batched GEMM (elsewhere)
+//   y_to        = A^T M[.][t][o] A  (m x m, cropped)     output transform
+// where d_tc is the alpha x alpha input patch of tile t (origin
+// (ty*m - ph, tx*m - pw)), zero outside the image: padding is applied by
+// bounds, not by a padded copy of the input.  All transform arithmetic is
+// fp32; U and V are stored in the GEMM's operand dtype, M is fp32.
+//
+// Every thread owns one (tile, channel) pair and every tile is transformed
+// independently, so the result for an image does not depend on which batch
+// tile it was processed in (batch tiling stays bit-identical).
+#include <cuda_runtime.h>
+
+#include <type_traits>
+
+#include "common.cuh"
+#include "internal.h"
+#include "winograd_gen.cuh"
+
+namespace b200conv {
+namespace {
+
+template <int M> struct Wino;
+template <> struct Wino<2> {
+  static constexpr int A = 4;
+  static __device__ __forceinline__ void bt(const float* x, float* y) { wino2_bt(x, y); }
+  static __device__ __forceinline__ void g(const float* x, float* y) { wino2_g(x, y); }
+  static __device__ __forceinline__ void at(const float* x, float* y) { wino2_at(x, y); }
+};
+template <> struct Wino<4> {
+  static constexpr int A = 6;
+  static __device__ __forceinline__ void bt(const float* x, float* y) { wino4_bt(x, y); }
+  static __device__ __forceinline__ void g(const float* x, float* y) { wino4_g(x, y); }
+  static __device__ __forceinline__ void at(const float* x, float* y) { wino4_at(x, y); }
+};
+template <> struct Wino<6> {
+  static constexpr int A = 8;
+  static __device__ __forceinline__ void bt(const float* x, float* y) { wino6_bt(x, y); }
+  static __device__ __forceinline__ void g(const float* x, float* y) { wino6_g(x, y); }
+  static __device__ __forceinline__ void at(const float* x, float* y) { wino6_at(x, y); }
+};
+
+// ---------------------------------------------------------------------------
+// Filter transform: one thread per (o, c).
+// ---------------------------------------------------------------------------
+template <int M, typename Tin, typename Tst>
+__global__ void wino_filter_kernel(const Tin* __restrict__ w, long long w_row_stride, int O, int C,
+                                   Tst* __restrict__ u) {
+  constexpr int A = Wino<M>::A;
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)O * C) return;
+  int o = (int)(idx / C), c = (int)(idx - (long long)o * C);
+  const Tin* wp = w + (long long)o * w_row_stride + c;
+  float g[3][3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) g[i][j] = Store<Tin>::to_f32(wp[(long long)(i * 3 + j) * C]);
+  // t = G g (A x 3), then U = t G^T (A x A)
+  float t[A][3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    float col[3] = {g[0][j], g[1][j], g[2][j]}, r[A];
+    Wino<M>::g(col, r);
+#pragma unroll
+    for (int i = 0; i < A; ++i) t[i][j] = r[i];
+  }
+  const long long plane = (long long)O * C;
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    float r[A];
+    Wino<M>::g(t[i], r);
+#pragma unroll
+    for (int j = 0; j < A; ++j) u[(long long)(i * A + j) * plane + idx] = Store<Tst>::from_f32(r[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Input transform: one thread per (tile, channel); threadIdx.x runs over
+// channels so loads and stores are coalesced.
+// ---------------------------------------------------------------------------
+struct WinoInArgs {
+  int h, w, c, ph, pw, tiles_h, tiles_w;
+  long long in_img_stride;
+  int n0;                 // first image of this batch tile
+  long long t_count;      // tiles in this batch tile (nb * tiles_h * tiles_w)
+  long long t_stride;     // row count of V's planes (the workspace's tile capacity)
+};
+
+template <int M, typename Tin, typename Tst>
+__global__ void __launch_bounds__(256)
+wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restrict__ v) {
+  constexpr int A = Wino<M>::A;
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  if (c >= a.c || t >= a.t_count) return;
+  const int per_img = a.tiles_h * a.tiles_w;
+  const int nl = (int)(t / per_img);
+  const int r = (int)(t - (long long)nl * per_img);
+  const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
+  const int y0 = ty * M - a.ph, x0 = tx * M - a.pw;
+  const Tin* base = in + (long long)(a.n0 + nl) * a.in_img_stride + c;
+
+  float d[A][A];
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    const int y = y0 + i;
+    const bool yok = y >= 0 && y < a.h;
+#pragma unroll
+    for (int j = 0; j < A; ++j) {
+      const int x = x0 + j;
+      d[i][j] = (yok && x >= 0 && x < a.w)
+                    ? Store<Tin>::to_f32(base[((long long)y * a.w + x) * a.c]) : 0.0f;
+    }
+  }
+  // columns: t = B^T d, then rows: V = t B
+  float tt[A][A];
+#pragma unroll
+  for (int j = 0; j < A; ++j) {
+    float col[A], res[A];
+#pragma unroll
+    for (int i = 0; i < A; ++i) col[i] = d[i][j];
+    Wino<M>::bt(col, res);
+#pragma unroll
+    for (int i = 0; i < A; ++i) tt[i][j] = res[i];
+  }
+  const long long plane = a.t_stride * a.c;
+  Tst* vp = v + t * a.c + c;
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    float res[A];
+    Wino<M>::bt(tt[i], res);
+#pragma unroll
+    for (int j = 0; j < A; ++j) vp[(long long)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Output transform: one thread per (tile, output channel).
+// ---------------------------------------------------------------------------
+struct WinoOutArgs {
+  int oh, ow, o, tiles_h, tiles_w;
+  long long out_img_stride;
+  int n0;
+  long long t_count, t_stride;
+  int accumulate;
+};
+
+template <int M, typename Tout>
+__global__ void __launch_bounds__(256)
+wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
+  constexpr int A = Wino<M>::A;
+  const int o = blockIdx.y * blockDim.x + threadIdx.x;
+  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  if (o >= a.o || t >= a.t_count) return;
+  const int per_img = a.tiles_h * a.tiles_w;
+  const int nl = (int)(t / per_img);
+  const int r = (int)(t - (long long)nl * per_img);
+  const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
+
+  const long long plane = a.t_stride * a.o;
+  const float* mp = mb + t * a.o + o;
+  float x[A][A];
+#pragma unroll
+  for (int i = 0; i < A; ++i)
+#pragma unroll
+    for (int j = 0; j < A; ++j) x[i][j] = __ldg(mp + (long long)(i * A + j) * plane);
+  // columns: t = A^T x (M x A), then rows: y = t A (M x M)
+  float tt[M][A];
+#pragma unroll
+  for (int j = 0; j < A; ++j) {
+    float col[A], res[M];
+#pragma unroll
+    for (int i = 0; i < A; ++i) col[i] = x[i][j];
+    Wino<M>::at(col, res);
+#pragma unroll
+    for (int i = 0; i < M; ++i) tt[i][j] = res[i];
+  }
+  Tout* op = out + (long long)(a.n0 + nl) * a.out_img_stride + o;
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    float res[M];
+    Wino<M>::at(tt[i], res);
+    const int y = ty * M + i;
+    if (y >= a.oh) continue;
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      const int xo = tx * M + j;
+      if (xo < a.ow) {
+        Tout* p = op + ((long long)y * a.ow + xo) * a.o;
+        float val = res[j];
+        if (a.accumulate) val += Store<Tout>::to_f32(*p);
+        *p = Store<Tout>::from_f32(val);
+      }
+    }
+  }
+}
+
+template <typename F>
+cudaError_t by_m(int m, F&& f) {
+  switch (m) {
+    case 2: return f(std::integral_constant<int, 2>{});
+    case 4: return f(std::integral_constant<int, 4>{});
+    case 6: return f(std::integral_constant<int, 6>{});
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename F>
+cudaError_t by_dt(conv_dtype_t dt, F&& f) {
+  switch (dt) {
+    case CONV_F32: return f(float{});
+    case CONV_F16: return f(__half{});
+    case CONV_BF16: return f(__nv_bfloat16{});
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int c, int m,
+                               conv_dtype_t in_dt, conv_dtype_t store_dt, void* u, cudaStream_t s) {
+  long long n = (long long)o * c;
+  if (n == 0) return cudaSuccess;
+  unsigned blocks = (unsigned)((n + 255) / 256);
+  return by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return by_dt(in_dt, [&](auto ti) {
+      using Tin = decltype(ti);
+      return by_dt(store_dt, [&](auto ts) {
+        using Tst = decltype(ts);
+        wino_filter_kernel<M, Tin, Tst><<<blocks, 256, 0, s>>>(
+            static_cast<const Tin*>(w), w_row_stride, o, c, static_cast<Tst*>(u));
+        return cudaGetLastError();
+      });
+    });
+  });
+}
+
+cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int m,
+                              conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_tile,
+                              cudaStream_t s) {
+  WinoInArgs a{};
+  a.h = g.h; a.w = g.w; a.c = g.c; a.ph = g.ph; a.pw = g.pw;
+  a.tiles_h = (g.oh + m - 1) / m;
+  a.tiles_w = (g.ow + m - 1) / m;
+  a.in_img_stride = g.in_img_stride;
+  a.n0 = n0;
+  a.t_count = (long long)nb * a.tiles_h * a.tiles_w;
+  a.t_stride = t_tile;
+  if (a.t_count == 0) return cudaSuccess;
+  int bx = g.c >= 64 ? 64 : 32;
+  dim3 block(bx, 256 / bx);
+  dim3 grid((unsigned)((a.t_count + block.y - 1) / block.y), (g.c + bx - 1) / bx);
+  if (grid.y > 65535) return cudaErrorInvalidValue;
+  return by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return by_dt(in_dt, [&](auto ti) {
+      using Tin = decltype(ti);
+      return by_dt(store_dt, [&](auto ts) {
+        using Tst = decltype(ts);
+        wino_input_kernel<M, Tin, Tst><<<grid, block, 0, s>>>(static_cast<const Tin*>(in), a,
+                                                              static_cast<Tst*>(v));
+        return cudaGetLastError();
+      });
+    });
+  });
+}
+
+cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb, int m,
+                               long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
+                               cudaStream_t s) {
+  WinoOutArgs a{};
+  a.oh = g.oh; a.ow = g.ow; a.o = g.o;
+  a.tiles_h = (g.oh + m - 1) / m;
+  a.tiles_w = (g.ow + m - 1) / m;
+  a.out_img_stride = g.out_img_stride;
+  a.n0 = n0;
+  a.t_count = (long long)nb * a.tiles_h * a.tiles_w;
+  a.t_stride = t_tile;
+  a.accumulate = accumulate ? 1 : 0;
+  if (a.t_count == 0) return cudaSuccess;
+  int bx = g.o >= 64 ? 64 : 32;
+  dim3 block(bx, 256 / bx);
+  dim3 grid((unsigned)((a.t_count + block.y - 1) / block.y), (g.o + bx - 1) / bx);
+  if (grid.y > 65535) return cudaErrorInvalidValue;
+  return by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return by_dt(out_dt, [&](auto to) {
+      using Tout = decltype(to);
+      wino_output_kernel<M, Tout><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
+      return cudaGetLastError();
+    });
+  });
+}
+
+}  // namespace b200conv

@@ -1,0 +1,209 @@
+/*
+ * b200conv.h -- C ABI of the B200 (sm_100a) NHWC convolution forward library.
+ *
+ * The operation (all entry points): a cross-correlation with zero padding,
+ * groups = 1,
+ *
+ *   out[n,oh,ow,o] = sum_{kh,kw,c} in[n, oh*sh - ph + kh*dh, ow*sw - pw + kw*dw, c] * w[o,kh,kw,c]
+ *   OH = floor((H + 2*ph - dh*(KH-1) - 1) / sh) + 1            (same for OW)
+ *
+ * over NHWC activations and OHWI weights, accumulated in fp32 and rounded
+ * once (round-to-nearest-even) to the storage dtype.  fp32 inputs are
+ * computed in true fp32 (FFMA; never TF32).  This is the operation the MLX pull
+ * requests "Bound winograd conv2d working set by tiling the batch" (Problem,
+ * Fix), "Use the explicit gemm for wide convs on neural accelerators"
+ * (description) and "Decompose small kernel-depth 3D convs into 2D convs"
+ * (Change) dispatch to their GPU kernels.
+ *
+ * Two algorithms sit behind one deterministic selector (conv2d_plan):
+ *  - implicit GEMM: A = im2col(in) is never materialised; 16-bit inputs run on
+ *    tcgen05 tensor cores with TMEM accumulators and TMA im2col staging, fp32
+ *    inputs on an FFMA core;
+ *  - Winograd F(m x m, 3 x 3) for 3x3 stride-1 convs: filter, input and output
+ *    transforms around a batched GEMM, with the batch tiled over one reused
+ *    workspace so that the scratch working set is bounded; tiled output is
+ *    bit-identical to untiled ("Bound winograd conv2d working set by tiling
+ *    the batch", Fix and Testing).
+ * conv3d runs as KD depth-tap 2D convs over zero-copy frame views whose results
+ * are accumulated in place ("Decompose small kernel-depth 3D convs into 2D
+ * convs", Change).
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named in/w/out/workspace are DEVICE pointers owned by the caller;
+ *    the library never allocates or frees device memory in a forward call and
+ *    holds no state except a per-device cache of constant device properties.
+ *  - in, w and out share one dtype.  in is NHWC (NDHWC for 3D) contiguous,
+ *    w is OHWI (O,KD,KH,KW,I for 3D) contiguous, out is NHWC (NDHWC) contiguous.
+ *  - Work is enqueued asynchronously on `stream` (0 = the legacy default
+ *    stream).  A returned CONV_OK means the work was validated and enqueued;
+ *    device-side failures (a bounded wait that ran out) are reported by
+ *    conv_check().
+ *  - out must not overlap in, w or workspace (CONV_ERR_INVALID).
+ *  - N = 0 is a valid no-op.  An empty output (OH <= 0, ...) or a non-positive
+ *    size, stride or dilation, or a negative pad, is CONV_ERR_INVALID.
+ *  - The selector is a pure function of (shape, dtype, device properties,
+ *    options); it never looks at the device's current free memory ("Bound
+ *    winograd conv2d working set by tiling the batch", maintainer review).
+ */
+#ifndef B200CONV_H
+#define B200CONV_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define B200CONV_API __attribute__((visibility("default")))
+#else
+#define B200CONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { CONV_F32 = 0, CONV_F16 = 1, CONV_BF16 = 2 } conv_dtype_t;
+
+typedef enum {
+    CONV_OK = 0,
+    CONV_ERR_INVALID = 1,      /* bad shape, pointer, overlap or argument */
+    CONV_ERR_UNSUPPORTED = 2,  /* forced algorithm cannot run this shape */
+    CONV_ERR_ALIGNMENT = 3,    /* reserved: misaligned pointers take the direct path instead */
+    CONV_ERR_WORKSPACE = 4,    /* workspace smaller than the plan needs; nothing was launched */
+    CONV_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    CONV_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (reported by conv_check) */
+} conv_status_t;
+
+typedef enum {
+    CONV_ALGO_AUTO = 0,
+    CONV_ALGO_IMPLICIT_GEMM = 1,
+    CONV_ALGO_WINOGRAD = 2,
+    CONV_ALGO_DIRECT = 3      /* SIMT implicit GEMM with scalar loads: any alignment */
+} conv_algo_t;
+
+typedef enum {
+    CONV_ENGINE_NONE = 0,
+    CONV_ENGINE_TCGEN05 = 1,  /* tcgen05.mma, TMEM accumulators, TMA staging (16-bit) */
+    CONV_ENGINE_SIMT = 2      /* FFMA in fp32 registers */
+} conv_engine_t;
+
+/* 2D problem.  stride/pad/dilation are {H, W}. */
+typedef struct {
+    int n, h, w, c, o, kh, kw;
+    int stride[2], pad[2], dilation[2];
+} conv2d_desc_t;
+
+/* 3D problem.  stride/pad/dilation are {D, H, W}. */
+typedef struct {
+    int n, d, h, w, c, o, kd, kh, kw;
+    int stride[3], pad[3], dilation[3];
+} conv3d_desc_t;
+
+/* Constant device properties the selector may depend on. */
+typedef struct {
+    int sm_count;
+    int cc_major, cc_minor;
+    unsigned long long total_global_mem;   /* bytes; a constant, never free memory */
+} conv_device_props_t;
+
+/*
+ * Options.  Pass NULL for the defaults, which are read from the environment
+ * (test hooks, read on every call before selection):
+ *   B200CONV_ALGO=auto|implicit|winograd|direct
+ *   B200CONV_WINOGRAD_WORKSPACE_BYTES=<bytes>   replaces the Winograd scratch budget
+ *   B200CONV_WINOGRAD_TILE_BATCH=<images>       forces the batch-tile size (capped by the budget)
+ * A non-NULL options struct ignores the environment.
+ */
+typedef struct {
+    conv_algo_t algo;                     /* CONV_ALGO_AUTO: let the selector choose */
+    long long winograd_budget_bytes;      /* < 0: the device default budget */
+    int winograd_tile_batch;              /* <= 0: derived from the budget */
+} conv_options_t;
+
+typedef struct {
+    conv_algo_t algo;          /* the algorithm that will run */
+    conv_engine_t engine;      /* the GEMM engine under it */
+    int tile_m, tile_n;        /* GEMM tile (rows x output channels) */
+    int winograd_m;            /* m of F(m x m, 3 x 3); 0 unless Winograd */
+    int batch_tile;            /* images per Winograd batch tile (= n when untiled) */
+    int num_batch_tiles;       /* number of batch tiles */
+    int channel_pad;           /* padded channel count of the pre-pass, 0 if none */
+    int taps;                  /* conv3d: number of depth taps (KD); 1 for conv2d */
+    size_t workspace_bytes;    /* bytes the caller must pass to *_forward */
+} conv_plan_t;
+
+/* Fill props for CUDA device `device`.  CONV_ERR_CUDA if there is none. */
+B200CONV_API conv_status_t conv_device_props(int device, conv_device_props_t *props);
+
+/*
+ * Plan a conv2d: validate, compute the output shape, pick the algorithm, the
+ * tile configuration and the Winograd batch tile, and size the workspace.
+ * Pure: the same arguments give the same plan in any process at any time.
+ * The Winograd budget is 3/4 of the device's total memory minus the conv's own
+ * tensors (input, output, transformed filter), capped at 8 GiB because the GPU
+ * is shared ("Bound winograd conv2d working set by tiling the batch", Fix).
+ */
+B200CONV_API conv_status_t conv2d_plan(const conv2d_desc_t *desc, conv_dtype_t dtype, int device,
+                          const conv_options_t *opts, conv_plan_t *plan);
+/* Same selector for explicit device properties (usable without a GPU). */
+B200CONV_API conv_status_t conv2d_plan_for_props(const conv2d_desc_t *desc, conv_dtype_t dtype,
+                                    const conv_device_props_t *props,
+                                    const conv_options_t *opts, conv_plan_t *plan);
+/* Workspace bytes conv2d_forward needs with these options; 0 if invalid. */
+B200CONV_API size_t conv2d_workspace_size(const conv2d_desc_t *desc, conv_dtype_t dtype, int device,
+                             const conv_options_t *opts);
+
+/*
+ * Run a conv2d on `stream`.  in [N,H,W,C], w [O,KH,KW,C], out [N,OH,OW,O],
+ * all of `dtype`, on the current CUDA device.  workspace may be NULL when the
+ * plan needs 0 bytes; a workspace_bytes smaller than the plan's is
+ * CONV_ERR_WORKSPACE and launches nothing (never a partial or zeroed result).
+ */
+B200CONV_API conv_status_t conv2d_forward(const void *in, const void *w, void *out,
+                             const conv2d_desc_t *desc, conv_dtype_t dtype,
+                             const conv_options_t *opts,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * conv3d as depth taps ("Decompose small kernel-depth 3D convs into 2D
+ * convs", Change): for each kd, a 2D conv over the zero-copy view of the input
+ * frames at depth offset kd*dd (frame stride sd*H*W*C) with the weight slice
+ * w[:, kd] (row stride KD*KH*KW*C); tap 0 writes out, taps 1..KD-1 are added
+ * in ascending order.  Depth padding, depth stride/dilation, N > 1 and any KD
+ * are handled by restricting each tap to the output frames whose input frame
+ * exists.  in [N,D,H,W,C], w [O,KD,KH,KW,C], out [N,OD,OH,OW,O].
+ */
+B200CONV_API conv_status_t conv3d_plan(const conv3d_desc_t *desc, conv_dtype_t dtype, int device,
+                          const conv_options_t *opts, conv_plan_t *plan);
+B200CONV_API conv_status_t conv3d_plan_for_props(const conv3d_desc_t *desc, conv_dtype_t dtype,
+                                    const conv_device_props_t *props,
+                                    const conv_options_t *opts, conv_plan_t *plan);
+B200CONV_API size_t conv3d_workspace_size(const conv3d_desc_t *desc, conv_dtype_t dtype, int device,
+                             const conv_options_t *opts);
+B200CONV_API conv_status_t conv3d_forward(const void *in, const void *w, void *out,
+                             const conv3d_desc_t *desc, conv_dtype_t dtype,
+                             const conv_options_t *opts,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * In-place depth-tap accumulate, out[i] = round(out[i] + tap[i]) for i < count
+ * (fp32 add, one rounding to dtype): the step the depth-tap page performs with
+ * an in-place binary add ("Decompose small kernel-depth 3D convs into 2D
+ * convs", Open questions 1).  Device pointers; out and tap must not overlap.
+ */
+B200CONV_API conv_status_t conv_accumulate(void *out, const void *tap, size_t count, conv_dtype_t dtype,
+                              void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word.
+ * Returns CONV_ERR_TIMEOUT if a kernel's bounded wait ran out since the last
+ * check, CONV_ERR_CUDA if the synchronisation failed, else CONV_OK.
+ */
+B200CONV_API conv_status_t conv_check(void *stream);
+
+/* Static description of a status code. */
+B200CONV_API const char *conv_status_string(conv_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200CONV_H */

@@ -1,0 +1,190 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/b200conv.h declares, and its selector behaves as a pure function of
+(shape, dtype, constant device properties, options).
+
+The selector follows "Bound winograd conv2d working set by tiling the batch"
+(Fix): Winograd batch tiles sized from a budget of 3/4 of device memory minus
+the conv's own tensors (capped at 8 GiB here), a fallback to the scratch-free
+implicit GEMM when no image fits or tiles carry too few GEMM rows, a forced
+tile size capped by the budget, and no dependence on current free memory.
+"""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+import dense_convolution_nhwc_b200 as dc
+from dense_convolution_nhwc_b200 import binding as B
+from dense_convolution_nhwc_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "b200conv.h")
+
+B200 = B.DeviceProps(148, 10, 0, 183359 * 2 ** 20)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"B200CONV_API[^;(]*?\b(conv\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ["conv2d_forward", "conv3d_forward", "conv2d_plan", "conv3d_plan", "conv2d_workspace_size",
+                 "conv3d_workspace_size", "conv_status_string", "conv_check", "conv_accumulate",
+                 "conv2d_plan_for_props", "conv3d_plan_for_props", "conv_device_props"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(B.library_path)
+    missing = [s for s in declared_symbols() if not hasattr(lib, s)]
+    assert not missing, missing
+
+
+def test_binding_has_the_same_names():
+    for s in declared_symbols():
+        assert callable(getattr(dc, s)), s
+
+
+def test_status_strings():
+    for code in range(7):
+        assert B.conv_status_string(code)
+    assert B.conv_status_string(4) == "workspace too small"
+
+
+def plan2d(shape: synth.Conv2dShape, dtype="f32", **opt):
+    desc = B.make_desc2d(shape.n, shape.h, shape.w, shape.c, shape.o, shape.kh, shape.kw,
+                         shape.stride, shape.pad, shape.dilation)
+    p = B.ConvPlan()
+    st = B.conv2d_plan_for_props(desc, B.DTYPE[dtype], B200, B.make_options(**opt) if opt else B.make_options(), p)
+    return st, p.as_dict()
+
+
+def test_winograd_shape_plan():
+    """40 x 512 x 512, 192 -> 96, fp32: F(6x6,3x3), per-image scratch
+    64 * 86^2 * (192 + 96) * 4 bytes = 545 MB, so an 8 GiB budget gives
+    batch tiles of 15 images (15, 15, 10)."""
+    st, p = plan2d(synth.WINOGRAD_F32)
+    assert st == 0
+    assert p["algo"] == "winograd" and p["winograd_m"] == 6 and p["engine"] == "simt"
+    assert p["batch_tile"] == 15 and p["num_batch_tiles"] == 3
+    per_img = 64 * 86 * 86 * (192 + 96) * 4
+    assert p["workspace_bytes"] >= 15 * per_img
+    assert p["workspace_bytes"] < 15 * per_img + 64 * 192 * 96 * 4 + 4096
+
+
+def test_small_shape_takes_implicit_gemm():
+    st, p = plan2d(synth.SMALL_F32)       # C + O = 64 < 256
+    assert st == 0 and p["algo"] == "implicit" and p["engine"] == "simt" and p["workspace_bytes"] == 0
+
+
+@pytest.mark.parametrize("budget,expect", [
+    (2 * 2 ** 30, ("winograd", 3)),        # 3 images/tile = 22188 GEMM rows >= 148 * 128
+    (2 ** 30, ("implicit", None)),         # 1 image/tile = 7396 rows: too few, falls back
+    (2 ** 20, ("implicit", None)),         # not even one image fits
+])
+def test_budget_injection(budget, expect):
+    st, p = plan2d(synth.WINOGRAD_F32, winograd_budget_bytes=budget)
+    assert st == 0 and p["algo"] == expect[0]
+    if expect[1]:
+        assert p["batch_tile"] == expect[1]
+
+
+@pytest.mark.parametrize("forced,nb,tiles", [(1, 1, 40), (7, 7, 6), (40, 15, 3), (15, 15, 3)])
+def test_forced_tile_is_capped_by_budget(forced, nb, tiles):
+    st, p = plan2d(synth.WINOGRAD_F32, winograd_tile_batch=forced)
+    assert st == 0 and p["algo"] == "winograd"
+    assert p["batch_tile"] == nb and p["num_batch_tiles"] == tiles
+
+
+def test_tiny_spatial_shape_falls_back_with_one_image_tiles():
+    """256 x 4 x 4, 64 -> 192: cut into one-image Winograd tiles it is the
+    page's ~40x-slower case, so the selector takes the implicit GEMM."""
+    per_img = 64 * 1 * (64 + 192) * 4
+    st, p = plan2d(synth.TINY_WINOGRAD, winograd_budget_bytes=per_img)
+    assert st == 0 and p["algo"] == "implicit"
+    st, p = plan2d(synth.TINY_WINOGRAD)   # whole batch fits: untiled Winograd
+    assert st == 0 and p["algo"] == "winograd" and p["num_batch_tiles"] == 1
+
+
+def test_sixteen_bit_takes_tensor_cores():
+    for name, shape, _ in synth.resnet50_layers(8):
+        for dt in ("f16", "bf16"):
+            st, p = plan2d(shape, dt)
+            assert st == 0 and p["algo"] == "implicit" and p["engine"] == "tcgen05", name
+            if shape.c == 3:
+                assert p["channel_pad"] == 8 and p["workspace_bytes"] > 0
+            else:
+                assert p["channel_pad"] == 0 and p["workspace_bytes"] == 0
+
+
+def test_sixteen_bit_forced_winograd_uses_f2x2():
+    st, p = plan2d(synth.Conv2dShape(2, 32, 32, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1)), "bf16", algo="winograd")
+    assert st == 0 and p["algo"] == "winograd" and p["winograd_m"] == 2 and p["engine"] == "tcgen05"
+
+
+def test_forced_winograd_rejects_other_shapes():
+    st, _ = plan2d(synth.Conv2dShape(1, 16, 16, 32, 32, 5, 5, (1, 1), (2, 2), (1, 1)), algo="winograd")
+    assert st == 2   # CONV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("shape", [
+    synth.Conv2dShape(1, 2, 2, 4, 4, 5, 5),                          # OH <= 0
+    synth.Conv2dShape(1, 8, 8, 4, 4, 3, 3, (0, 1)),                  # zero stride
+    synth.Conv2dShape(1, 8, 8, 4, 4, 3, 3, (1, 1), (-1, 0)),         # negative pad
+    synth.Conv2dShape(1, 8, 8, 0, 4, 3, 3),                          # no channels
+    synth.Conv2dShape(1, 8, 8, 4, 4, 3, 3, (1, 1), (0, 0), (0, 1)),  # zero dilation
+])
+def test_invalid_descriptors(shape):
+    st, _ = plan2d(shape)
+    assert st == 1   # CONV_ERR_INVALID
+
+
+def test_plan_is_pure_across_calls_and_processes():
+    shapes = [synth.WINOGRAD_F32, synth.SMALL_F32, synth.TINY_WINOGRAD] + [s for _, s, _ in synth.resnet50_layers(1)]
+    first = [plan2d(s, dt) for s in shapes for dt in ("f32", "bf16")]
+    again = [plan2d(s, dt) for s in shapes for dt in ("f32", "bf16")]
+    assert first == again
+    code = ("import sys; sys.path.insert(0, %r); from tests import test_abi as t; from dense_convolution_nhwc_b200 import synth; "
+            "print(repr([t.plan2d(s, dt) for s in [synth.WINOGRAD_F32, synth.SMALL_F32, synth.TINY_WINOGRAD] + "
+            "[s for _, s, _ in synth.resnet50_layers(1)] for dt in ('f32', 'bf16')]))" % ROOT)
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, check=True, cwd=ROOT)
+    assert out.stdout.strip() == repr(first)
+
+
+def test_environment_hooks_apply_only_without_options():
+    desc = B.make_desc2d(40, 512, 512, 192, 96, 3, 3, 1, 1, 1)
+    code = ("import sys; sys.path.insert(0, %r); from dense_convolution_nhwc_b200 import binding as B; "
+            "d = B.make_desc2d(40, 512, 512, 192, 96, 3, 3, 1, 1, 1); p = B.ConvPlan(); "
+            "B.conv2d_plan_for_props(d, 0, B.DeviceProps(148, 10, 0, 183359 * 2 ** 20), None, p); "
+            "print(p.as_dict()['algo'], p.as_dict()['batch_tile'])" % ROOT)
+    env = dict(os.environ, B200CONV_WINOGRAD_TILE_BATCH="7")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, check=True, env=env, cwd=ROOT)
+    assert out.stdout.split() == ["winograd", "7"]
+    env = dict(os.environ, B200CONV_ALGO="direct")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, check=True, env=env, cwd=ROOT)
+    assert out.stdout.split()[0] == "direct"
+    env = dict(os.environ, B200CONV_WINOGRAD_WORKSPACE_BYTES=str(2 ** 20))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, check=True, env=env, cwd=ROOT)
+    assert out.stdout.split()[0] == "implicit"
+
+
+def test_conv3d_plan_depth_taps():
+    for s in synth.CONV3D_TAPS:
+        desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+        p = B.ConvPlan()
+        assert B.conv3d_plan_for_props(desc, B.DTYPE["bf16"], B200, None, p) == 0
+        d = p.as_dict()
+        assert d["taps"] == 3 and d["engine"] == "tcgen05"
+        out_bytes = s.od * s.oh * s.ow * s.o * 2
+        assert d["workspace_bytes"] >= out_bytes       # the tap scratch
+
+
+def test_conv3d_invalid():
+    desc = B.make_desc3d(1, 2, 8, 8, 4, 4, 3, 3, 3, 1, (0, 1, 1), 1)     # OD <= 0
+    p = B.ConvPlan()
+    assert B.conv3d_plan_for_props(desc, 0, B200, None, p) == 1
