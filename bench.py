@@ -1,0 +1,593 @@
+#!/usr/bin/env python
+"""Benchmark: convolution TFLOP/s on one B200 (or N replicas).
+
+Metric: direct-equivalent conv TFLOP/s, 2*N*OH*OW*O*C*KH*KW per second (Winograd
+counted at direct-equivalent FLOPs), and its fraction of the peak of the
+dominant kernel.  Default workload: the fp32 Winograd case of "Bound winograd
+conv2d working set by tiling the batch" (Testing): N=40, 512x512, 192->96,
+3x3, stride 1, pad 1, seeded uniform inputs, batch-tiled Winograd F(6x6,3x3).
+Other workloads (--workload) are measurement aids: the ResNet-50 layer set,
+the wide-channel implicit-GEMM sweep, the conv3d depth-tap cases, the small
+fp32 case.
+
+One step = one forward pass of the whole path over one batch with inputs
+resident in HBM.  Timed with CUDA events on the launching stream, W untimed
+warm-ups, K timed steps bracketed by a barrier and a synchronize; for N > 1
+each rank runs an independent replica (the forward pass needs no collective)
+and the slowest rank's time is reported.  `e2e` repeats the step through the
+same C ABI with host buffers: pinned host -> device copy of the inputs, the
+conv, device -> host copy of the output, all inside the timed region.
+
+--impl reference times the CPU oracle (the plain fp64 direct convolution) on
+host cores on a bounded pixel sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from dense_convolution_nhwc_b200 import synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FP32_LANES_PER_SM = 128
+BASELINE_CONTEXT = {
+    # direct-equivalent TFLOP/s of the pages' own measurement of the same workload
+    # (310 ms on an M2 Max: 2*40*512*512*96*192*9 / 0.310 s); context, another machine
+    "winograd_f32": 11.2,
+}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+class Conv:
+    """One conv2d or conv3d call of a workload."""
+
+    def __init__(self, shape, dtype, dist, algo="auto", name=None):
+        self.shape, self.dtype, self.dist, self.algo = shape, dtype, dist, algo
+        self.is3d = isinstance(shape, synth.Conv3dShape)
+        self.name = name or shape.name()
+
+    @property
+    def flops(self):
+        return self.shape.flops
+
+
+def workload(name):
+    if name == "winograd_f32":
+        return ("conv2d fp32 NHWC N=40 H=W=512 C=192->O=96 3x3 stride 1 pad 1 (Winograd, batch-tiled workspace)",
+                [Conv(synth.WINOGRAD_F32, "f32", "uniform")], "f32")
+    if name == "small_f32":
+        return ("conv2d fp32 NHWC N=2 H=W=16 C=32->O=32 3x3 stride 1 pad 1",
+                [Conv(synth.SMALL_F32, "f32", "uniform")], "f32")
+    if name.startswith("resnet50_"):
+        _, dt, b = name.split("_")
+        convs = []
+        for lname, shape, count in synth.resnet50_layers(int(b[1:])):
+            for i in range(count):
+                convs.append(Conv(shape, dt, "he", name=f"{lname}#{i}"))
+        return (f"ResNet-50 v1.5 conv layer set (53 convs) {dt} batch {b[1:]} 224x224", convs, dt)
+    if name.startswith("conv3d_"):
+        dt = name.split("_")[1]
+        return ("conv3d bf16 NDHWC 3x3x3 s1 spatial pad 1 depth pad 0 N=1 depth taps: 17x64x64 256->256, "
+                "41x60x104 256->256, 41x120x208 512->512", [Conv(s, dt, "normal") for s in synth.CONV3D_TAPS], dt)
+    if name.startswith("wide_"):
+        # wide_<dtype>: C_out >= 512 and M >= 16384 aligned members of the sweep
+        dt = name.split("_")[1]
+        shapes = [s for s in synth.wide_sweep(True) if s.o >= 512 and s.n * s.oh * s.ow >= 16384]
+        if not name.endswith("_all"):
+            shapes = [s for s in shapes if s.stride == (1, 1) and s.dilation == (1, 1)]
+        return (f"wide-channel implicit-GEMM sweep {dt}: C_out>=512, M>=16384, aligned ({len(shapes)} shapes)",
+                [Conv(s, dt, "normal") for s in shapes], dt)
+    raise SystemExit(f"unknown workload {name}")
+
+
+# ---------------------------------------------------------------------------
+# per-kernel algorithmic work (for the roofline)
+# ---------------------------------------------------------------------------
+
+def kernel_work(conv, plan):
+    """{kernel name: (flops, bytes)} of algorithmic work for one call, by the
+    plan the library will run."""
+    s = conv.shape
+    esz = 4 if conv.dtype == "f32" else 2
+    w = {}
+
+    def add(k, f=0.0, b=0.0):
+        f0, b0 = w.get(k, (0.0, 0.0))
+        w[k] = (f0 + f, b0 + b)
+
+    if conv.is3d:
+        frames_out = s.od
+        n2 = synth.Conv2dShape(frames_out, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride[1:], s.pad[1:], s.dilation[1:])
+        taps = s.kd
+        for t in range(taps):
+            for k, (f, b) in kernel_work(Conv(n2, conv.dtype, conv.dist), plan).items():
+                add(k, f * s.n, b * s.n)
+        out_bytes = s.n * s.od * s.oh * s.ow * s.o * esz
+        add("accumulate", 0.0, 3.0 * out_bytes * (taps - 1))
+        return w
+    M = s.n * s.oh * s.ow
+    K = s.c * s.kh * s.kw
+    in_b, w_b, out_b = s.n * s.h * s.w * s.c * esz, s.o * K * esz, M * s.o * esz
+    if plan["algo"] == "winograd":
+        m = plan["winograd_m"]
+        a2 = (m + 2) ** 2
+        T = s.n * math.ceil(s.oh / m) * math.ceil(s.ow / m)
+        st = 4 if plan["engine"] == "simt" else esz
+        add("wino_filter", 0.0, w_b + a2 * s.o * s.c * st)
+        add("wino_input", 0.0, in_b + a2 * T * s.c * st)
+        gk = "wino_gemm_tc" if plan["engine"] == "tcgen05" else "wino_gemm_simt"
+        add(gk, 2.0 * a2 * T * s.c * s.o, a2 * T * (s.c * st + s.o * 4))
+        add("wino_output", 0.0, a2 * T * s.o * 4 + out_b)
+    else:
+        k = "tc_conv" if plan["engine"] == "tcgen05" else "simt_conv"
+        add(k, 2.0 * M * s.o * K, in_b + w_b + out_b)
+        if plan["channel_pad"]:
+            cp = plan["channel_pad"]
+            add("channel_pad", 0.0, in_b + s.n * s.h * s.w * cp * esz + w_b + s.o * s.kh * s.kw * cp * esz)
+    return w
+
+
+def kernel_bound(name):
+    if name in ("tc_conv", "wino_gemm_tc"):
+        return "tensor"
+    if name in ("simt_conv", "wino_gemm_simt"):
+        return "alu"
+    return "hbm"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "dense_convolution_nhwc_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    try:
+        return json.load(open(p))
+    except Exception:
+        return {}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if getattr(self, "fh", None):
+            self.fh.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1])]
+        smax = max((num(r[2]) or 0) for r in rows)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower() == "active":
+                    reasons.add(n)
+        power = [num(r[3]) for r in rows if num(r[3])]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x, world, device):
+    """Max over ranks (the slowest replica sets the time)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline
+# ---------------------------------------------------------------------------
+
+METRIC = "conv TFLOP/s (direct-equivalent FLOPs) and fraction of the dominant kernel's peak"
+
+
+def oracle_sample_rate(conv, x_host, w_host, target_s, seed=0):
+    """Time the oracle on a pixel sample sized for about target_s seconds.
+    Returns (TFLOP/s, cores, description, seconds of the timed pass)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    s = conv.shape
+    per_px = 2.0 * s.o * s.c * s.kh * s.kw * (s.kd if conv.is3d else 1)
+
+    def run(npx):
+        import torch
+        g = torch.Generator().manual_seed(seed)
+        if conv.is3d:
+            nimg = x_host.shape[0]
+            idx = torch.randint(0, nimg * s.od * s.oh * s.ow, (npx,), generator=g)
+            ow_, r = idx % s.ow, idx // s.ow
+            oh_, r = r % s.oh, r // s.oh
+            od_, n_ = r % s.od, r // s.od
+            pix = torch.stack([n_, od_, oh_, ow_], 1).int().numpy()
+            t0 = time.perf_counter()
+            oracle.conv3d(x_host, w_host, conv.dtype, s.stride, s.pad, s.dilation, pixels=pix, threads=cores)
+        else:
+            nimg = x_host.shape[0]
+            idx = torch.randint(0, nimg * s.oh * s.ow, (npx,), generator=g)
+            ow_, r = idx % s.ow, idx // s.ow
+            oh_, n_ = r % s.oh, r // s.oh
+            pix = torch.stack([n_, oh_, ow_], 1).int().numpy()
+            t0 = time.perf_counter()
+            oracle.conv2d(x_host, w_host, conv.dtype, s.stride, s.pad, s.dilation, pixels=pix, threads=cores)
+        return time.perf_counter() - t0
+
+    npx = 64
+    dt = run(npx)
+    while dt < 0.5 and npx < 1 << 22:
+        npx *= 4
+        dt = run(npx)
+    npx = max(1, int(npx * target_s / max(dt, 1e-6)))
+    dt = run(npx)
+    return (per_px * npx / dt / 1e12, cores,
+            f"{npx} seeded output pixels (with replacement) x all {s.o} channels of {conv.name}, one pass", dt)
+
+
+def run_reference(args, wl_name):
+    """The CPU oracle as it stands, on the host cores, on a bounded sample."""
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    import torch
+    desc, convs, dtype = workload(wl_name)
+    conv = max(convs, key=lambda c: c.flops)
+    s = conv.shape
+    # one image (frame stack) of the workload, seeded, on the host
+    if conv.is3d:
+        one = synth.Conv3dShape(1, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+        x, w = synth.conv3d_inputs(one, dtype, conv.dist, 0, "cpu")
+    else:
+        one = synth.Conv2dShape(1, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
+        x, w = synth.conv2d_inputs(one, dtype, conv.dist, 0, "cpu")
+    per_step_s = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    rates, secs = [], []
+    desc_s = ""
+    cores = len(os.sched_getaffinity(0))
+    for i in range(args.warmup + args.steps):
+        r, cores, desc_s, sec = oracle_sample_rate(conv, x, w, per_step_s, seed=i)
+        if i >= args.warmup:
+            rates.append(r)
+            secs.append(sec)
+    value = statistics.mean(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(secs) * 1000.0, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"f32": "f64 (fp32 inputs)", "f16": "f64 (fp16 inputs)",
+                                         "bf16": "f64 (bf16 inputs)"}[dtype],
+        "data": "synthetic", "config": {"workload": desc, "sample_of": conv.name},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc_s},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="winograd_f32")
+    ap.add_argument("--algo", default="auto", choices=["auto", "implicit", "winograd", "direct"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--per-conv", action="store_true", help="also print one line per conv of the workload")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, args.workload)
+        return
+
+    import torch
+    from dense_convolution_nhwc_b200 import binding as B
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    desc, convs, dtype = workload(args.workload)
+    opts = B.make_options(args.algo)
+
+    # resident inputs, outputs and workspaces
+    items = []
+    ws_max = 0
+    for i, cv in enumerate(convs):
+        s = cv.shape
+        if cv.is3d:
+            x, w = synth.conv3d_inputs(s, cv.dtype, cv.dist, i, dev)
+            d = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+            plan = B.plan3d(d, cv.dtype, local, opts)
+            out = torch.empty((s.n, s.od, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
+        else:
+            x, w = synth.conv2d_inputs(s, cv.dtype, cv.dist, i, dev)
+            d = B.make_desc2d(s.n, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
+            plan = B.plan2d(d, cv.dtype, local, opts)
+            out = torch.empty((s.n, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
+        ws_max = max(ws_max, plan["workspace_bytes"])
+        items.append((cv, x, w, d, plan, out))
+    ws = torch.empty(max(ws_max, 256), dtype=torch.uint8, device=dev)
+    dt_code = B.DTYPE[dtype]
+    fwd = B.conv3d_forward if convs[0].is3d else B.conv2d_forward
+    sptr = stream.cuda_stream
+
+    def step(xs=None, outs=None):
+        for j, (cv, x, w, d, plan, out) in enumerate(items):
+            xp = xs[j].data_ptr() if xs is not None else x.data_ptr()
+            op = outs[j].data_ptr() if outs is not None else out.data_ptr()
+            st = fwd(xp, w.data_ptr(), op, d, dt_code, opts, ws.data_ptr(), ws.numel(), sptr)
+            if st != 0:
+                raise B.ConvError(st, cv.name)
+
+    in_bytes = sum(x.numel() * x.element_size() for _, x, _, _, _, _ in items)
+    flush_needed = in_bytes < 2 * L2_BYTES
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush_needed else None
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert B.conv_check(sptr) == 0
+
+    # timed region (device time of the steps; an L2 flush between steps is outside the events)
+    total_flops = sum(cv.flops for cv, *_ in items)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        B.conv_profile_begin()
+        for k in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        prof = B.profile_end()
+    barrier(world)
+    assert B.conv_check(sptr) == 0
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ms = reduce_max(ms, world, dev)
+    value = world * total_flops / (ms * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # roofline of the dominant kernel (the one with the largest event time)
+    work = {}
+    for cv, x, w, d, plan, out in items:
+        for k, (f, b) in kernel_work(cv, plan).items():
+            f0, b0 = work.get(k, (0.0, 0.0))
+            work[k] = (f0 + f, b0 + b)
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    kernels = {}
+    for name, (launches, tot) in prof.items():
+        per_launch_ms = tot / max(launches, 1)
+        f, b = work.get(name, (0.0, 0.0))
+        kernels[name] = {"launches_per_step": launches / args.steps, "ms_per_step": tot / args.steps,
+                         "share": tot / max(1e-9, sum(t for _, t in prof.values())),
+                         "flops_per_step": f, "bytes_per_step": b, "per_launch_ms": per_launch_ms}
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    kd = kernels[dom]
+    bound = kernel_bound(dom)
+    launches_step = kd["launches_per_step"]
+    if bound == "hbm":
+        achieved = kd["bytes_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e9
+        peak = peaks.get("hbm_gbs", 6650.0)
+        unit, peak_src = "GB/s", "measured (MEASURED_PEAKS.json hbm_gbs)" if peaks else "fallback"
+    elif bound == "tensor":
+        achieved = kd["flops_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops", 1590.0)
+        unit, peak_src = "TFLOP/s", "measured burst bf16 (MEASURED_PEAKS.json); fp16 same nominal rate"
+    else:
+        achieved = kd["flops_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e12
+        smax = peaks.get("sm_max_mhz", 1965.0)
+        peak = 148 * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
+        unit, peak_src = "TFLOP/s", f"derived: 148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"
+    traffic_db = load_traffic()
+    tr = traffic_db.get(f"{args.workload}:{dom}")
+    traffic = None
+    if tr and tr.get("source_hash") == source_hash():
+        traffic = tr.get("bytes_per_launch")
+    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+            "algorithmic_per_launch": (kd["bytes_per_step"] if bound == "hbm" else kd["flops_per_step"]) / launches_step}
+    gpu_launches = int(round(sum(l for l, _ in prof.values())))
+
+    # e2e through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = [x.cpu().pin_memory() for _, x, *_ in items]
+        hw = [w.cpu().pin_memory() for _, _, w, *_ in items]
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for *_, out in items]
+        dx = [torch.empty_like(x) for _, x, *_ in items]
+        dw = [torch.empty_like(w) for _, _, w, *_ in items]
+        k_e2e = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            for j in range(len(items)):
+                dx[j].copy_(hx[j], non_blocking=True)
+                dw[j].copy_(hw[j], non_blocking=True)
+            for j, (cv, x, w, d, plan, out) in enumerate(items):
+                st = fwd(dx[j].data_ptr(), dw[j].data_ptr(), out.data_ptr(), d, dt_code, opts, ws.data_ptr(),
+                         ws.numel(), sptr)
+                if st != 0:
+                    raise B.ConvError(st, cv.name)
+            for j, (*_, out) in enumerate(items):
+                hout[j].copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ems = reduce_max(a.elapsed_time(b) / k_e2e, world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in hx + hw)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        e2e = {"value": world * total_flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e}
+        del hx, hw, hout, dx, dw
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        big = max(items, key=lambda it: it[0].flops)
+        cv, x, w = big[0], big[1], big[2]
+        xh = x[:1].cpu()
+        r, cores, sample, _ = oracle_sample_rate(cv, xh, w.cpu(), 15.0)
+        cpu = {"value": r, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        plan0 = items[0][4]
+        line = {
+            "metric": METRIC,
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": (value / BASELINE_CONTEXT[args.workload]) if args.workload in BASELINE_CONTEXT else None,
+            "dtype": dtype, "data": "synthetic",
+            "config": {"workload": desc, "plan": {k: plan0[k] for k in ("algo", "engine", "winograd_m", "batch_tile",
+                                                                          "num_batch_tiles", "tile_n")},
+                       "convs_per_step": len(items), "flops_per_step": total_flops,
+                       "l2": "L2 flushed between steps (outside the events)" if flush_needed
+                       else f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": gpu_launches * 1,
+            "gpu_launches_per_step": gpu_launches / args.steps,
+            "e2e": e2e, "cpu_baseline": cpu,
+        }
+        if args.workload in BASELINE_CONTEXT:
+            line["vs_baseline_note"] = "pages' 310 ms on an M2 Max for the same workload (context, other hardware)"
+        print(json.dumps(line))
+        if args.per_conv:
+            for cv, x, w, d, plan, out in items:
+                evs = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                fwd_one = lambda: fwd(x.data_ptr(), w.data_ptr(), out.data_ptr(), d, dt_code, opts,
+                                      ws.data_ptr(), ws.numel(), sptr)
+                for _ in range(3):
+                    fwd_one()
+                reps = 10
+                if flush is not None:
+                    times = []
+                    for _ in range(reps):
+                        flush.zero_()
+                        evs[0].record(stream)
+                        fwd_one()
+                        evs[1].record(stream)
+                        torch.cuda.synchronize()
+                        times.append(evs[0].elapsed_time(evs[1]))
+                    t = statistics.median(times)
+                else:
+                    evs[0].record(stream)
+                    for _ in range(reps):
+                        fwd_one()
+                    evs[1].record(stream)
+                    torch.cuda.synchronize()
+                    t = evs[0].elapsed_time(evs[1]) / reps
+                print(json.dumps({"conv": cv.name, "dtype": cv.dtype, "algo": plan["algo"], "engine": plan["engine"],
+                                  "tile_n": plan["tile_n"], "ms": t, "tflops": cv.flops / (t * 1e-3) / 1e12,
+                                  "frac_of_bf16_peak": cv.flops / (t * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0)}))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

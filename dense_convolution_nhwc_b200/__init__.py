@@ -11,7 +11,8 @@ _BINDING_NAMES = frozenset({
     "conv2d_forward", "conv3d_forward", "conv2d_plan", "conv3d_plan",
     "conv2d_plan_for_props", "conv3d_plan_for_props",
     "conv2d_workspace_size", "conv3d_workspace_size", "conv_check",
-    "conv_status_string", "conv_device_props", "conv_accumulate",
+    "conv_status_string", "conv_device_props", "conv_accumulate", "conv_profile_begin", "conv_profile_end",
+    "profile_end", "KernelTime",
     # types and helpers
     "ConvError", "Conv2dDesc", "Conv3dDesc", "ConvPlan", "ConvOptions", "DeviceProps",
     "ALGO", "DTYPE", "STATUS", "ENGINE", "library_path", "make_desc2d", "make_desc3d", "make_options",

@@ -103,6 +103,14 @@ _conv_check = _sig("conv_check", _I, _P)
 _conv_status_string = _sig("conv_status_string", ctypes.c_char_p, _I)
 
 
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+_conv_profile_begin = _sig("conv_profile_begin", _I)
+_conv_profile_end = _sig("conv_profile_end", _I, ctypes.POINTER(KernelTime), _I)
+
+
 class ConvError(RuntimeError):
     def __init__(self, status: int, where: str = ""):
         self.status = status
@@ -169,6 +177,23 @@ def conv_accumulate(out: int, tap: int, count: int, dtype: int, stream: int) -> 
 
 def conv_check(stream: int) -> int:
     return _conv_check(stream or None)
+
+
+def conv_profile_begin() -> int:
+    return _conv_profile_begin()
+
+
+def conv_profile_end(out, max_entries: int) -> int:
+    return _conv_profile_end(out, max_entries)
+
+
+def profile_end() -> dict:
+    """Stop kernel timing; {kernel name: (launches, total ms)} since conv_profile_begin()."""
+    buf = (KernelTime * 32)()
+    n = conv_profile_end(buf, 32)
+    if n < 0:
+        raise ConvError(5, "conv_profile_end")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n)}
 
 
 # ---------------------------------------------------------------------------

@@ -21,6 +21,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "internal.h"
 
@@ -71,6 +72,55 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 long long out_extent(long long in, int k, int s, int p, int d) {
   return (in + 2LL * p - (long long)d * (k - 1) - 1) / s + 1;
 }
+
+// ------------------------------ profiling ------------------------------------
+// Opt-in: each kernel launch is bracketed by two events on its stream.
+
+enum Kind { K_TC_CONV, K_SIMT_CONV, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
+            K_WINO_OUTPUT, K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
+const char* const kKindName[K_COUNT] = {"tc_conv", "simt_conv", "wino_filter", "wino_input", "wino_gemm_tc",
+                                        "wino_gemm_simt", "wino_output", "accumulate", "channel_pad", "fill"};
+
+struct ProfRecord {
+  int kind;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  std::vector<ProfRecord> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+} g_prof;
+
+struct ProfScope {
+  cudaStream_t s;
+  bool active = false;
+  ProfRecord r{};
+  ProfScope(int kind, cudaStream_t st) : s(st) {
+    if (!g_prof.on) return;
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    r.kind = kind;
+    r.a = g_prof.get();
+    r.b = g_prof.get();
+    if (r.a && r.b && cudaEventRecord(r.a, s) == cudaSuccess) active = true;
+  }
+  ~ProfScope() {
+    if (!active) return;
+    cudaEventRecord(r.b, s);
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.recs.push_back(r);
+  }
+};
 
 // ----------------------------- options ---------------------------------------
 
@@ -269,20 +319,33 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     void* v = base + u_bytes;
     float* mb = reinterpret_cast<float*>(
         base + u_bytes + align256((size_t)a2 * s.nb * tiles_per_img * g.c * dtype_size(s.wino_store)));
-    cudaError_t e = launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
+    cudaError_t e;
+    {
+      ProfScope ps(K_WINO_FILTER, st);
+      e = launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
+    }
     if (e != cudaSuccess) return CONV_ERR_CUDA;
     for (int n0 = 0; n0 < g.n; n0 += s.nb) {
       const int nbi = std::min(s.nb, g.n - n0);
       const long long t = (long long)nbi * tiles_per_img;
-      e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
+      {
+        ProfScope ps(K_WINO_INPUT, st);
+        e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
+      }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
       BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb};
-      if (s.engine == CONV_ENGINE_TCGEN05)
+      if (s.engine == CONV_ENGINE_TCGEN05) {
+        ProfScope ps(K_WINO_GEMM_TC, st);
         e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
-      else
+      } else {
+        ProfScope ps(K_WINO_GEMM_SIMT, st);
         e = launch_simt_batched_gemm(bg, st);
+      }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
-      e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, false, st);
+      {
+        ProfScope ps(K_WINO_OUTPUT, st);
+        e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, false, st);
+      }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
     }
     return CONV_OK;
@@ -293,23 +356,33 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
       const int esz = dtype_size(dt);
       void* pin = base;
       void* pw = base + align256((size_t)g.n * g.h * g.w * s.cpad * esz);
-      cudaError_t e = launch_channel_pad(in, g.n, (long long)g.h * g.w, g.c, g.in_img_stride, pin, s.cpad, dt, st);
-      if (e == cudaSuccess)
+      cudaError_t e;
+      {
+        ProfScope ps(K_CHANNEL_PAD, st);
+        e = launch_channel_pad(in, g.n, (long long)g.h * g.w, g.c, g.in_img_stride, pin, s.cpad, dt, st);
+      }
+      if (e == cudaSuccess) {
+        ProfScope ps(K_CHANNEL_PAD, st);
         e = launch_channel_pad(w, g.o, (long long)g.kh * g.kw, g.c, g.w_row_stride, pw, s.cpad, dt, st);
+      }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
       Geom gp = g;
       gp.c = s.cpad;
       gp.in_img_stride = (long long)g.h * g.w * s.cpad;
       gp.w_row_stride = (long long)g.kh * g.kw * s.cpad;
+      ProfScope ps(K_TC_CONV, st);
       return cuda_status(launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, st));
     }
-    if (tc_conv_supported(g, dt, in, w))
+    if (tc_conv_supported(g, dt, in, w)) {
+      ProfScope ps(K_TC_CONV, st);
       return cuda_status(launch_tc_conv(in, w, out, g, dt, s.tile_n, d.props.sm_count, d.err_word, st));
+    }
     // Misaligned pointers: the any-alignment path below.
   }
   const bool vec = s.algo != CONV_ALGO_DIRECT && g.c % 4 == 0 &&
                    (g.in_img_stride % 4 == 0) && (g.w_row_stride % 4 == 0) &&
                    aligned16(in) && aligned16(w);
+  ProfScope ps(K_SIMT_CONV, st);
   return cuda_status(launch_simt_conv(in, w, out, g, dt, vec, false, st));
 }
 
@@ -519,6 +592,7 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
     const uint8_t* in_n = static_cast<const uint8_t*>(in) + (size_t)n * desc->d * frame_in * esz;
     uint8_t* out_n = static_cast<uint8_t*>(out) + (size_t)n * od * frame_out * esz;
     if (!first_covers_all) {
+      ProfScope ps(K_FILL, st_);
       if (launch_fill_zero(out_n, (size_t)od * frame_out * esz, st_) != cudaSuccess) return CONV_ERR_CUDA;
     }
     for (int i = 0; i < ntaps; ++i) {
@@ -533,6 +607,7 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
       st = run2d(in_view, w_slice, dst, g, dtype, s, ws2, *d, st_);
       if (st != CONV_OK) return st;
       if (!direct_write) {
+        ProfScope ps(K_ACCUMULATE, st_);
         if (launch_accumulate(out_view, tap_buf, (size_t)g.n * frame_out, dtype, st_) != cudaSuccess)
           return CONV_ERR_CUDA;
       }
@@ -547,7 +622,45 @@ conv_status_t conv_accumulate(void* out, const void* tap, size_t count, conv_dty
   if (!out || !tap) return CONV_ERR_INVALID;
   const size_t bytes = count * dtype_size(dtype);
   if (overlaps(out, bytes, tap, bytes)) return CONV_ERR_INVALID;
+  ProfScope ps(K_ACCUMULATE, static_cast<cudaStream_t>(stream));
   return cuda_status(launch_accumulate(out, tap, count, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+conv_status_t conv_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  for (auto& r : g_prof.recs) {
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  g_prof.on = true;
+  return CONV_OK;
+}
+
+int conv_profile_end(conv_kernel_time_t* out, int max_entries) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.on = false;
+  int launches[K_COUNT] = {0};
+  double ms[K_COUNT] = {0};
+  bool failed = false;
+  for (auto& r : g_prof.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      failed = true;
+    launches[r.kind] += 1;
+    ms[r.kind] += t;
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.recs.clear();
+  if (failed) return -1;
+  int n = 0;
+  for (int k = 0; k < K_COUNT; ++k) {
+    if (!launches[k]) continue;
+    if (out && n < max_entries) out[n] = conv_kernel_time_t{kKindName[k], launches[k], ms[k]};
+    ++n;
+  }
+  return std::min(n, max_entries);
 }
 
 conv_status_t conv_check(void* stream) {

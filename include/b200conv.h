@@ -199,6 +199,24 @@ B200CONV_API conv_status_t conv_accumulate(void *out, const void *tap, size_t co
  */
 B200CONV_API conv_status_t conv_check(void *stream);
 
+/*
+ * Opt-in kernel timing, for benchmarks.  Between conv_profile_begin() and
+ * conv_profile_end() every kernel the library launches on the current device
+ * is bracketed by a pair of CUDA events recorded on its launch stream.
+ * conv_profile_end() waits for those events, stops recording and writes up to
+ * max_entries per-kernel summaries (one per kernel kind that ran: its name,
+ * launch count and summed event time), returning how many it wrote (or -1 on
+ * a CUDA error).  Recording is process-wide and not meant for concurrent use
+ * from several threads.
+ */
+typedef struct {
+    const char *name;       /* static string, e.g. "tc_conv" */
+    int launches;
+    double total_ms;
+} conv_kernel_time_t;
+B200CONV_API conv_status_t conv_profile_begin(void);
+B200CONV_API int conv_profile_end(conv_kernel_time_t *out, int max_entries);
+
 /* Static description of a status code. */
 B200CONV_API const char *conv_status_string(conv_status_t status);
 
