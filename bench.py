@@ -65,6 +65,12 @@ class Conv:
 
 
 def workload(name):
+    if name.startswith("conv2d:"):
+        # conv2d:<n>,<h>,<w>,<c>,<o>,<k>,<stride>,<pad>,<dilation>:<dtype>  (a single conv, e.g. for ncu)
+        _, dims, dt = name.split(":")
+        n, h, w, c, o, k, st, pd, dl = (int(v) for v in dims.split(","))
+        shape = synth.Conv2dShape(n, h, w, c, o, k, k, (st, st), (pd, pd), (dl, dl))
+        return f"conv2d {dt} NHWC {shape.name()}", [Conv(shape, dt, "uniform" if dt == "f32" else "normal")], dt
     if name == "winograd_f32":
         return ("conv2d fp32 NHWC N=40 H=W=512 C=192->O=96 3x3 stride 1 pad 1 (Winograd, batch-tiled workspace)",
                 [Conv(synth.WINOGRAD_F32, "f32", "uniform")], "f32")
