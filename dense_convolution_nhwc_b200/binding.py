@@ -99,6 +99,8 @@ _conv3d_workspace_size = _sig("conv3d_workspace_size", ctypes.c_size_t, ctypes.P
 _conv3d_forward = _sig("conv3d_forward", _I, _P, _P, _P, ctypes.POINTER(Conv3dDesc), _I,
                        ctypes.POINTER(ConvOptions), _P, ctypes.c_size_t, _P)
 _conv_accumulate = _sig("conv_accumulate", _I, _P, _P, ctypes.c_size_t, _I, _P)
+_conv2d_forward_winograd_static = _sig("conv2d_forward_winograd_static", _I, _P, _P, _P,
+                                       ctypes.POINTER(Conv2dDesc), _I, _P)
 _conv_check = _sig("conv_check", _I, _P)
 _conv_status_string = _sig("conv_status_string", ctypes.c_char_p, _I)
 
@@ -169,6 +171,11 @@ def conv3d_forward(inp: int, w: int, out: int, desc: Conv3dDesc, dtype: int, opt
                    workspace: int, workspace_bytes: int, stream: int) -> int:
     return _conv3d_forward(inp, w, out, ctypes.byref(desc), dtype, _opt(opts), workspace or None,
                            workspace_bytes, stream or None)
+
+
+def conv2d_forward_winograd_static(inp: int, w: int, out: int, desc: Conv2dDesc, dtype: int, stream: int) -> int:
+    """Winograd conv2d with the library's fixed 64 MiB device scratch: no workspace, no allocation."""
+    return _conv2d_forward_winograd_static(inp, w, out, ctypes.byref(desc), dtype, stream or None)
 
 
 def conv_accumulate(out: int, tap: int, count: int, dtype: int, stream: int) -> int:

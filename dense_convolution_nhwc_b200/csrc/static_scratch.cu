@@ -1,0 +1,93 @@
+// static_scratch.cu -- a Winograd conv2d entry point that allocates nothing.
+//
+// conv2d_forward needs a caller-provided workspace for the Winograd path (the
+// transformed filter, and the transformed input and GEMM output of one batch
+// tile).  Some callers cannot provide one: code that runs inside another
+// runtime's hooks with no access to an allocator, code that must not
+// allocate once it is running (real-time or fixed-footprint services), and
+// callers that receive only borrowed input/output pointers.  For them this file
+// holds the scratch in a fixed device array compiled into the library, and the
+// entry point below runs the Winograd path with it.
+//
+// The array is 64 MiB.  Every GPU that loads the library holds it until the
+// process exits.  All calls share it and it keeps the last call's contents;
+// the Winograd path writes every scratch element it reads, so nothing needs
+// clearing between calls.  Two calls whose work overlaps on the GPU (on
+// different streams, or from several host threads) race on the array.
+//
+// The batch is tiled so that the transformed filter plus one batch tile fit in
+// the array, exactly as the budgeted Winograd path tiles it, so results equal
+// conv2d_forward's Winograd results bit for bit.  A conv whose transformed
+// filter plus a single image's transform buffers do not fit is rejected with
+// CONV_ERR_WORKSPACE before anything is launched.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.h"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+constexpr int kMaxDevices = 64;
+
+// Host code must never use this name as a device address: it is a host-side
+// stand-in.  The device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+void* g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Once per device, with that device current: look up the array's device
+// address.  This is the first call's set-up; it makes no allocation.
+conv_status_t scratch_address(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return CONV_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return CONV_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return CONV_OK;
+}
+
+}  // namespace
+
+extern "C" conv_status_t conv2d_forward_winograd_static(const void* in, const void* w, void* out,
+                                                        const conv2d_desc_t* desc, conv_dtype_t dtype,
+                                                        void* stream) {
+  if (!desc) return CONV_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+  void* scratch = nullptr;
+  conv_status_t st = scratch_address(dev, &scratch);
+  if (st != CONV_OK) return st;
+
+  // Is the shape one the Winograd path runs at all (3x3, stride 1, dilation 1)?
+  conv_options_t o{CONV_ALGO_WINOGRAD, 1LL << 60, 1};
+  conv_plan_t plan{};
+  st = conv2d_plan(desc, dtype, dev, &o, &plan);
+  if (st != CONV_OK) return st;
+  if (desc->n == 0) return CONV_OK;
+
+  // Largest batch tile whose scratch (filter + tile buffers) fits the array:
+  // start from the tile the array's size allows for the transform buffers and
+  // shrink it until the filter fits beside it.  Forcing the tile size keeps
+  // small tiles on the Winograd path.
+  o.winograd_budget_bytes = (long long)kStaticScratchBytes;
+  o.winograd_tile_batch = desc->n;
+  for (int i = 0; i <= desc->n + 1; ++i) {
+    st = conv2d_plan(desc, dtype, dev, &o, &plan);
+    if (st == CONV_ERR_UNSUPPORTED) return CONV_ERR_WORKSPACE;   // not even one image fits
+    if (st != CONV_OK) return st;
+    if (plan.workspace_bytes <= kStaticScratchBytes) break;
+    if (plan.batch_tile <= 1) return CONV_ERR_WORKSPACE;
+    // drop at least one image; per-image share estimated from the plan
+    const double per_img = (double)plan.workspace_bytes / plan.batch_tile;
+    int drop = (int)((double)(plan.workspace_bytes - kStaticScratchBytes) / per_img) + 1;
+    o.winograd_tile_batch = plan.batch_tile - drop > 1 ? plan.batch_tile - drop : 1;
+  }
+  if (plan.algo != CONV_ALGO_WINOGRAD || plan.workspace_bytes > kStaticScratchBytes) return CONV_ERR_WORKSPACE;
+  return conv2d_forward(in, w, out, desc, dtype, &o, scratch, kStaticScratchBytes, stream);
+}

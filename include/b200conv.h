@@ -200,6 +200,29 @@ B200CONV_API conv_status_t conv_accumulate(void *out, const void *tap, size_t co
 B200CONV_API conv_status_t conv_check(void *stream);
 
 /*
+ * Winograd conv2d that allocates nothing.  The pages have no counterpart of
+ * this entry point; it serves callers that cannot allocate device memory or
+ * hand the library a workspace (code running inside another runtime's hooks
+ * with no allocator, services that must not allocate once running, callers
+ * that hold only borrowed input/output pointers).  Its scratch is a 64 MiB
+ * device array compiled into the library, held by every GPU that loads it
+ * until the process exits.  in/w/out and their layouts are as for
+ * conv2d_forward.  The shape must be 3x3, stride 1, dilation 1
+ * (CONV_ERR_UNSUPPORTED otherwise).  The batch is tiled so that the transformed
+ * filter and one batch tile fit in the array; a conv whose filter plus one
+ * image's transform buffers exceed 64 MiB is rejected with CONV_ERR_WORKSPACE
+ * and nothing is launched.  Output equals conv2d_forward with
+ * CONV_ALGO_WINOGRAD at the same tile size.  No cudaMalloc or cudaFree is
+ * called.  The first call on each device looks up the array's address; make
+ * that first call before any stream capture.  All calls share the array and
+ * it keeps the last call's contents (nothing needs clearing); calls whose work
+ * overlaps on the GPU race on it.
+ */
+B200CONV_API conv_status_t conv2d_forward_winograd_static(const void *in, const void *w, void *out,
+                                                          const conv2d_desc_t *desc, conv_dtype_t dtype,
+                                                          void *stream);
+
+/*
  * Opt-in kernel timing, for benchmarks.  Between conv_profile_begin() and
  * conv_profile_end() every kernel the library launches on the current device
  * is bracketed by a pair of CUDA events recorded on its launch stream.
