@@ -102,6 +102,7 @@ _conv_accumulate = _sig("conv_accumulate", _I, _P, _P, ctypes.c_size_t, _I, _P)
 _conv2d_forward_winograd_static = _sig("conv2d_forward_winograd_static", _I, _P, _P, _P,
                                        ctypes.POINTER(Conv2dDesc), _I, _P)
 _conv_check = _sig("conv_check", _I, _P)
+_conv_selftest_timeout = _sig("conv_selftest_timeout", _I, ctypes.c_longlong, _P)
 _conv_status_string = _sig("conv_status_string", ctypes.c_char_p, _I)
 
 
@@ -184,6 +185,10 @@ def conv_accumulate(out: int, tap: int, count: int, dtype: int, stream: int) -> 
 
 def conv_check(stream: int) -> int:
     return _conv_check(stream or None)
+
+
+def conv_selftest_timeout(limit_ns: int, stream: int) -> int:
+    return _conv_selftest_timeout(limit_ns, stream or None)
 
 
 def conv_profile_begin() -> int:

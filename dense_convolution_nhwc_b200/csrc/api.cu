@@ -626,6 +626,16 @@ conv_status_t conv_accumulate(void* out, const void* tap, size_t count, conv_dty
   return cuda_status(launch_accumulate(out, tap, count, dtype, static_cast<cudaStream_t>(stream)));
 }
 
+conv_status_t conv_selftest_timeout(long long limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 100000000LL) return CONV_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
+  DeviceState* d = nullptr;
+  conv_status_t st = device_state(dev, &d);
+  if (st != CONV_OK) return st;
+  return cuda_status(launch_wait_selftest(d->err_word, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 conv_status_t conv_profile_begin(void) {
   std::lock_guard<std::mutex> lk(g_prof.mu);
   for (auto& r : g_prof.recs) {

@@ -17,6 +17,7 @@ enum DevErr : int {
   DEVERR_TIMEOUT_MMA_FULL = 0x102,   // MMA issuer waited too long for a loaded stage
   DEVERR_TIMEOUT_MMA_TMEM = 0x103,   // MMA issuer waited too long for a drained accumulator
   DEVERR_TIMEOUT_EPILOGUE = 0x104,   // epilogue waited too long for a finished accumulator
+  DEVERR_TIMEOUT_SELFTEST = 0x1ff,   // the watchdog self-test's deliberate wait
 };
 
 inline int dtype_size(conv_dtype_t t) { return t == CONV_F32 ? 4 : 2; }
@@ -61,6 +62,9 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
 // tcgen05 batched GEMM for 16-bit operands with fp32 D (Winograd 16-bit path).
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n,
                                    int sm_count, int* err_word, cudaStream_t s);
+
+// Watchdog self-test: one bounded wait on a barrier nothing arrives on.
+cudaError_t launch_wait_selftest(int* err_word, long long limit_ns, cudaStream_t s);
 
 // Winograd transforms (fp32 arithmetic; V/U stored in `store_dt`).
 cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int c, int m,

@@ -99,17 +99,17 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: true when the phase completed; false after the time limit or
-// when another role raised the abort flag.
+// Bounded wait: true when the phase completed; false after limit_ns of
+// %globaltimer or when another role raised the abort flag.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int* err, int code) {
+                                       int* err, int code, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (*abort_flag) return false;
-      if (gtimer() - t0 > kWaitLimitNs) {
+      if (gtimer() - t0 > limit_ns) {
         *abort_flag = 1;
         if (code) atomicCAS(err, 0, code);
         return false;
@@ -420,6 +420,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// Watchdog self-test: wait on an mbarrier phase that nothing completes, with a
+// short limit, so the timeout path (error word, abort, return) is exercised
+// without any risk of a hang.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), err, DEVERR_TIMEOUT_SELFTEST,
+              limit_ns);
+}
+
 // ------------------------------- host side ----------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
@@ -489,6 +506,11 @@ cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcAr
 }
 
 }  // namespace
+
+cudaError_t launch_wait_selftest(int* err_word, long long limit_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(err_word, (unsigned long long)limit_ns);
+  return cudaGetLastError();
+}
 
 bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w) {
   if (dt == CONV_F32) return false;

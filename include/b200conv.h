@@ -240,6 +240,17 @@ typedef struct {
 B200CONV_API conv_status_t conv_profile_begin(void);
 B200CONV_API int conv_profile_end(conv_kernel_time_t *out, int max_entries);
 
+/*
+ * Watchdog self-test.  Launches one tiny kernel that waits, through the same
+ * bounded-wait routine the tensor-core pipeline uses, on an mbarrier phase that
+ * nothing completes; after limit_ns nanoseconds (1 us .. 100 ms, else
+ * CONV_ERR_INVALID) the wait gives up, records a timeout in the device error
+ * word and the kernel returns.  The next conv_check() then reports
+ * CONV_ERR_TIMEOUT (and clears it).  Used by the tests to show that a stuck
+ * pipeline ends with a status instead of a hang.
+ */
+B200CONV_API conv_status_t conv_selftest_timeout(long long limit_ns, void *stream);
+
 /* Static description of a status code. */
 B200CONV_API const char *conv_status_string(conv_status_t status);
 

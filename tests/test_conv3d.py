@@ -1,0 +1,118 @@
+"""conv3d as depth-tap 2D convs ("Decompose small kernel-depth 3D convs into 2D
+convs", Change, Tests).
+
+* the fast path against the oracle over shapes with Cout != Cin,
+  KD in {1, 2, 3, 5} and a 1x1-spatial case;
+* the cases the page sends to its fallback -- depth stride > 1, depth padding,
+  non-multiple-of-16 channels, N > 1, kernel depth dilation, KD > 7 -- stay
+  correct here because the taps are generalised instead;
+* the depth-tap result equals a manual loop of conv2d_forward over frame views
+  plus conv_accumulate, bit for bit (the page's "numerically identical to"
+  per-frame 2D);
+* the workload's three shapes on sampled pixels.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dense_convolution_nhwc_b200 import binding as B
+from dense_convolution_nhwc_b200 import synth
+from tests.gpu_util import TOL, as_f64, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run3d(x, w, s, options=None):
+    out = torch.full((s.n, s.od, s.oh, s.ow, s.o), float("nan"), dtype=x.dtype, device=x.device)
+    out = B.conv3d(x, w, s.stride, s.pad, s.dilation, options=options, out=out)
+    torch.cuda.synchronize()
+    assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    return out
+
+
+def check3d(s, dtype, dist="normal", options=None, sample=None):
+    x, w = synth.conv3d_inputs(s, dtype, dist, 0, device="cuda")
+    out = run3d(x, w, s, options)
+    if sample:
+        pix = synth.sample_pixels(s.n, s.oh, s.ow, sample, 0, od=s.od)
+        ref = oracle.conv3d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation, pixels=pix.numpy())
+        p = pix.long()
+        got = as_f64(out[p[:, 0], p[:, 1], p[:, 2], p[:, 3]])
+    else:
+        ref = oracle.conv3d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
+        got = as_f64(out)
+    return assert_close(got, ref, dtype, s.name())
+
+
+FAST = [
+    synth.Conv3dShape(1, 6, 10, 12, 32, 48, 1, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),
+    synth.Conv3dShape(1, 7, 9, 9, 48, 32, 2, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),
+    synth.Conv3dShape(1, 8, 12, 10, 64, 64, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),
+    synth.Conv3dShape(1, 9, 6, 7, 32, 64, 5, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),
+    synth.Conv3dShape(1, 6, 1, 1, 64, 32, 3, 1, 1, (1, 1, 1), (0, 0, 0), (1, 1, 1)),   # 1x1 spatial
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("s", FAST, ids=lambda s: s.name())
+def test_depth_taps_against_oracle(s, dtype):
+    check3d(s, dtype)
+
+
+FALLBACK_CASES = [
+    synth.Conv3dShape(1, 9, 8, 8, 32, 32, 3, 3, 3, (2, 1, 1), (0, 1, 1), (1, 1, 1)),   # depth stride 2
+    synth.Conv3dShape(1, 6, 8, 8, 32, 32, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1)),   # depth pad 1
+    synth.Conv3dShape(1, 6, 8, 8, 20, 13, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),   # non-mod-16 channels
+    synth.Conv3dShape(3, 5, 7, 6, 32, 16, 2, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),   # N > 1
+    synth.Conv3dShape(1, 9, 6, 6, 16, 16, 3, 3, 3, (1, 2, 2), (2, 1, 1), (2, 1, 1)),   # depth dilation, pads
+    synth.Conv3dShape(1, 12, 5, 5, 16, 16, 9, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),  # KD > 7
+    synth.Conv3dShape(2, 7, 9, 11, 24, 40, 3, 3, 5, (3, 2, 1), (2, 0, 2), (1, 1, 2)),  # everything at once
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("s", FALLBACK_CASES, ids=lambda s: s.name())
+def test_generalised_taps(s, dtype):
+    check3d(s, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_taps_equal_manual_per_frame_loop(dtype):
+    """conv3d == for kd: conv2d_forward(frame view kd, w[:, kd]) then an in-place add."""
+    s = synth.Conv3dShape(1, 9, 14, 12, 64, 48, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    x, w = synth.conv3d_inputs(s, dtype, "normal", 5, device="cuda")
+    got = run3d(x, w, s)
+    OD = s.od
+    acc = None
+    for kd in range(s.kd):
+        view = x[0, kd:kd + OD]                     # [OD, H, W, C], contiguous frames
+        wk = w[:, kd].contiguous()                  # [O, KH, KW, C]
+        tap = B.conv2d(view, wk, s.stride[1:], s.pad[1:], s.dilation[1:])
+        if acc is None:
+            acc = tap
+        else:
+            st = B.conv_accumulate(acc.data_ptr(), tap.data_ptr(), acc.numel(), B.DTYPE[dtype],
+                                   torch.cuda.current_stream().cuda_stream)
+            assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(got[0], acc)
+
+
+@pytest.mark.parametrize("s", synth.CONV3D_TAPS, ids=lambda s: s.name())
+def test_workload_shapes_sampled(s):
+    check3d(s, "bf16", sample=2048)
+
+
+def test_accumulate_rounds_once_per_add():
+    """out = round(out + tap) with an fp32 add, every dtype, ragged length."""
+    for dt, tt in (("f32", torch.float32), ("f16", torch.float16), ("bf16", torch.bfloat16)):
+        n = 1000003
+        g = torch.Generator(device="cuda").manual_seed(9)
+        a = torch.randn(n, generator=g, device="cuda").to(tt)
+        b = torch.randn(n, generator=g, device="cuda").to(tt)
+        want = (a.float() + b.float()).to(tt)
+        st = B.conv_accumulate(a.data_ptr(), b.data_ptr(), n, B.DTYPE[dt], torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert torch.equal(a, want), dt

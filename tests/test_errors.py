@@ -1,0 +1,142 @@
+"""Error paths on the GPU.
+
+The failure the Winograd page fixes is a silent one: an out-of-memory during
+the conv was dropped and the output came back all zeros ("Bound winograd
+conv2d working set by tiling the batch", Problem).  Here every call returns a
+status, an undersized workspace is refused before anything runs (the output
+keeps its poison), overlapping buffers are refused, misaligned pointers take
+the any-alignment path and stay correct, and N = 0 is a no-op.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dense_convolution_nhwc_b200 import binding as B
+from dense_convolution_nhwc_b200 import synth
+from tests.gpu_util import TOL, as_f64, assert_close
+
+pytestmark = pytest.mark.gpu
+
+S = synth.Conv2dShape(3, 18, 18, 64, 96, 3, 3, (1, 1), (1, 1), (1, 1))
+
+
+def desc(s):
+    return B.make_desc2d(s.n, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
+
+
+def stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def test_undersized_workspace_is_refused_and_nothing_runs():
+    x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
+    opts = B.make_options("winograd")
+    need = B.conv2d_workspace_size(desc(S), 0, 0, opts)
+    assert need > 0
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    out = torch.full((S.n, S.oh, S.ow, S.o), float("nan"), device="cuda")
+    st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), out.data_ptr(), desc(S), 0, opts, ws.data_ptr(),
+                          ws.numel(), stream())
+    assert st == 4       # CONV_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all()      # never a partial or zeroed result
+    st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), out.data_ptr(), desc(S), 0, opts, 0, 0, stream())
+    assert st == 4
+
+
+def test_overlapping_output_is_refused():
+    x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
+    st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), x.data_ptr(), desc(S), 0, None, 0, 0, stream())
+    assert st == 1
+    st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), w.data_ptr(), desc(S), 0, None, 0, 0, stream())
+    assert st == 1
+
+
+def test_null_pointers_are_refused():
+    assert B.conv2d_forward(0, 0, 0, desc(S), 0, None, 0, 0, stream()) == 1
+
+
+def test_empty_batch_is_a_no_op():
+    d = desc(synth.Conv2dShape(0, 18, 18, 64, 96, 3, 3, (1, 1), (1, 1), (1, 1)))
+    assert B.conv2d_forward(0, 0, 0, d, 0, None, 0, 0, stream()) == 0
+    d3 = B.make_desc3d(0, 4, 8, 8, 16, 16, 3, 3, 3, 1, (0, 1, 1), 1)
+    assert B.conv3d_forward(0, 0, 0, d3, 2, None, 0, 0, stream()) == 0
+
+
+def test_invalid_shape_on_device():
+    d = desc(synth.Conv2dShape(1, 2, 2, 4, 4, 5, 5))
+    assert B.conv2d_forward(1, 1, 1, d, 0, None, 0, 0, stream()) == 1
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+def test_misaligned_pointers_take_the_any_alignment_path(dtype):
+    """Inputs that start 2 (16-bit) or 4 (fp32) bytes past a 16-byte boundary:
+    no TMA or vector load may touch them; the result is still correct."""
+    s = synth.Conv2dShape(2, 13, 11, 24, 40, 3, 3, (1, 1), (1, 1), (1, 1))
+    x, w = synth.conv2d_inputs(s, dtype, "normal", 4, device="cuda")
+    xb = torch.empty(x.numel() + 8, dtype=x.dtype, device="cuda")
+    wb = torch.empty(w.numel() + 8, dtype=w.dtype, device="cuda")
+    xm = xb[1:1 + x.numel()].view(x.shape)
+    wm = wb[1:1 + w.numel()].view(w.shape)
+    xm.copy_(x)
+    wm.copy_(w)
+    assert xm.data_ptr() % 16 != 0 and wm.data_ptr() % 16 != 0
+    out = torch.full((s.n, s.oh, s.ow, s.o), float("nan"), dtype=x.dtype, device="cuda")
+    st = B.conv2d_forward(xm.data_ptr(), wm.data_ptr(), out.data_ptr(), desc(s), B.DTYPE[dtype], None, 0, 0, stream())
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = oracle.conv2d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
+    assert_close(as_f64(out), ref, dtype, "misaligned")
+
+
+def test_forced_winograd_on_other_shapes_is_unsupported():
+    s = synth.Conv2dShape(1, 16, 16, 32, 32, 3, 3, (2, 2), (1, 1), (1, 1))
+    x, w = synth.conv2d_inputs(s, "f32", "normal", 0, device="cuda")
+    with pytest.raises(B.ConvError) as e:
+        B.conv2d(x, w, s.stride, s.pad, s.dilation, options=B.make_options("winograd"))
+    assert e.value.status == 2
+
+
+def test_conv_check_is_clean_after_normal_work():
+    x, w = synth.conv2d_inputs(S, "bf16", "normal", 0, device="cuda")
+    B.conv2d(x, w, S.stride, S.pad, S.dilation)
+    assert B.conv_check(stream()) == 0
+
+
+def test_plan_matches_props_selector():
+    p = B.DeviceProps()
+    assert B.conv_device_props(0, p) == 0
+    assert p.sm_count > 0 and p.total_global_mem > 0
+    for shape in (S, synth.WINOGRAD_F32, synth.TINY_WINOGRAD):
+        for dt in ("f32", "bf16"):
+            a, b = B.ConvPlan(), B.ConvPlan()
+            assert B.conv2d_plan(desc(shape), B.DTYPE[dt], 0, None, a) == 0
+            assert B.conv2d_plan_for_props(desc(shape), B.DTYPE[dt], p, None, b) == 0
+            assert a.as_dict() == b.as_dict()
+
+
+def test_plan_ignores_current_memory_use():
+    """The selector never looks at free memory: allocate a large block and re-plan."""
+    before = B.plan2d(desc(synth.WINOGRAD_F32), "f32")
+    free, total = torch.cuda.mem_get_info()
+    hog = torch.empty(int(min(free * 0.5, 60e9)), dtype=torch.uint8, device="cuda")
+    after = B.plan2d(desc(synth.WINOGRAD_F32), "f32")
+    del hog
+    torch.cuda.empty_cache()
+    assert before == after
+
+
+def test_bounded_wait_reports_timeout_instead_of_hanging():
+    """A kernel waits on an mbarrier that nothing completes, with a 2 ms limit:
+    it returns, and conv_check reports CONV_ERR_TIMEOUT once, then clears it."""
+    s = stream()
+    assert B.conv_check(s) == 0
+    assert B.conv_selftest_timeout(2_000_000, s) == 0
+    assert B.conv_check(s) == 6      # CONV_ERR_TIMEOUT
+    assert B.conv_check(s) == 0
+    # the context is still usable
+    x, w = synth.conv2d_inputs(S, "bf16", "normal", 0, device="cuda")
+    B.conv2d(x, w, S.stride, S.pad, S.dilation)
+    assert B.conv_check(s) == 0
+    assert B.conv_selftest_timeout(10, s) == 1     # limit out of range
