@@ -154,12 +154,22 @@ def kernel_bound(name):
     return "hbm"
 
 
-def source_hash():
+KERNEL_SOURCES = {
+    "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["simt_conv.cu", "common.cuh"],
+    "tc_conv": ["tc_conv.cu", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "common.cuh"],
+    "wino_input": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
+    "wino_output": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
+    "wino_filter": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
+    "accumulate": ["elementwise.cu", "common.cuh"], "channel_pad": ["elementwise.cu", "common.cuh"],
+}
+
+
+def source_hash(kernel):
+    """Hash of the source files a kernel is built from (ncu traffic is void once it changes)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dense_convolution_nhwc_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES.get(kernel, []):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -488,7 +498,7 @@ def main():
     traffic_db = load_traffic()
     tr = traffic_db.get(f"{args.workload}:{dom}")
     traffic = None
-    if tr and tr.get("source_hash") == source_hash():
+    if tr and tr.get("source_hash") == source_hash(dom):
         traffic = tr.get("bytes_per_launch")
     roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
