@@ -118,11 +118,12 @@ def kernel_work(conv, plan):
         frames_out = s.od
         n2 = synth.Conv2dShape(frames_out, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride[1:], s.pad[1:], s.dilation[1:])
         taps = s.kd
+        out_bytes = s.n * s.od * s.oh * s.ow * s.o * esz
         for t in range(taps):
             for k, (f, b) in kernel_work(Conv(n2, conv.dtype, conv.dist), plan).items():
-                add(k, f * s.n, b * s.n)
-        out_bytes = s.n * s.od * s.oh * s.ow * s.o * esz
-        add("accumulate", 0.0, 3.0 * out_bytes * (taps - 1))
+                # taps after the first also read the output they add into
+                extra = out_bytes if (t > 0 and k in ("tc_conv", "simt_conv", "wino_output")) else 0.0
+                add(k, f * s.n, b * s.n + extra)
         return w
     M = s.n * s.oh * s.ow
     K = s.c * s.kh * s.kw
@@ -155,7 +156,7 @@ def kernel_bound(name):
 
 
 KERNEL_SOURCES = {
-    "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["simt_conv.cu", "common.cuh"],
+    "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["wino_gemm_f32.cu"],
     "tc_conv": ["tc_conv.cu", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "common.cuh"],
     "wino_input": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
     "wino_output": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],

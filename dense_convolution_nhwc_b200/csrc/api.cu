@@ -198,12 +198,43 @@ int tc_tile_n(const Geom& g, const conv_device_props_t& p) {
   return tiles256 < p.sm_count ? 128 : 256;
 }
 
-void winograd_sizes(const Geom& g, conv_dtype_t store, int m, size_t* u_bytes, size_t* per_img) {
-  const int a = m + 2;
-  const long long tiles = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+long long round4(long long x) { return (x + 3) & ~3LL; }
+
+// V layout of the fp32 (FFMA) Winograd path: tile-major [a2][T][C] lets the
+// input transform write whole pixels' channels contiguously; the GEMM stages
+// it through swizzled shared rows.
+#ifndef B200CONV_F32_V_TILE_MAJOR
+#define B200CONV_F32_V_TILE_MAJOR 1
+#endif
+constexpr bool kF32VTileMajor = B200CONV_F32_V_TILE_MAJOR != 0;
+
+// Workspace layout of the Winograd path for batch tiles of nb images.
+//   tensor-core GEMM (16-bit operands): U [a2][O][C], V [a2][T][C], M [a2][T][O] fp32
+//   FFMA GEMM (fp32 operands):          U [a2][C][O4], V [a2][T][C] (tile-major) or
+//                                       [a2][C][T4] (channel-major), M [a2][T][O] fp32
+// (O4, T4 = O, T rounded up to 4 so rows start 16-byte aligned).
+struct WinoLayout {
+  size_t u_bytes = 0, v_bytes = 0, m_bytes = 0;
+  long long tiles_per_img = 0;
+  size_t per_img = 0;   // V + M bytes per image (the budget unit)
+};
+
+WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb) {
+  WinoLayout L;
+  const long long a2 = (long long)(m + 2) * (m + 2);
+  L.tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
   const int esz = dtype_size(store);
-  *u_bytes = align256((size_t)a * a * g.o * g.c * esz);
-  *per_img = (size_t)a * a * tiles * ((size_t)g.c * esz + (size_t)g.o * 4);
+  L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * esz + (size_t)g.o * 4);
+  const long long t = nb * L.tiles_per_img;
+  if (cmajor) {
+    L.u_bytes = align256((size_t)(a2 * g.c * round4(g.o)) * esz);
+    L.v_bytes = align256((size_t)(a2 * g.c * ((kF32VTileMajor && g.c % 4 == 0) ? t : round4(t))) * esz);
+  } else {
+    L.u_bytes = align256((size_t)(a2 * g.o * g.c) * esz);
+    L.v_bytes = align256((size_t)(a2 * t * g.c) * esz);
+  }
+  L.m_bytes = align256((size_t)(a2 * t * g.o) * 4);
+  return L;
 }
 
 conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t& p,
@@ -226,9 +257,9 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     // 16-byte rule, else the transforms store fp32 for the FFMA engine.
     const bool tc_gemm = dt != CONV_F32 && p.cc_major == 10 && g.c % 8 == 0;
     const conv_dtype_t store = (dt == CONV_F32 || !tc_gemm) ? CONV_F32 : dt;
-    size_t u_bytes, per_img;
-    winograd_sizes(g, store, m, &u_bytes, &per_img);
-    const long long tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+    const WinoLayout L1 = winograd_layout(g, store, !tc_gemm, m, 1);
+    const size_t u_bytes = L1.u_bytes, per_img = L1.per_img;
+    const long long tiles_per_img = L1.tiles_per_img;
     long long budget;
     if (o.winograd_budget_bytes >= 0) {
       budget = o.winograd_budget_bytes;
@@ -252,11 +283,9 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
       s->tile_m = 128;
-      s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : (g.o <= 64 ? 64 : g.o <= 96 ? 96 : 128);
-      const long long t_tile = nb * tiles_per_img;
-      const int a2 = (m + 2) * (m + 2);
-      s->ws = u_bytes + align256((size_t)a2 * t_tile * g.c * dtype_size(store)) +
-              align256((size_t)a2 * t_tile * g.o * 4);
+      s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
+      const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb);
+      s->ws = L.u_bytes + L.v_bytes + L.m_bytes;
       s->cpad = 0;
       return CONV_OK;
     }
@@ -305,46 +334,52 @@ conv_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CONV_OK : C
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Run one planned 2D conv.  ws holds at least s.ws bytes.
+// Run one planned 2D conv.  ws holds at least s.ws bytes.  accumulate: add the
+// result into out (out = round(out + round(result))), the depth-tap sum fused
+// into the conv's output stage.
 conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt, const Sel& s,
-                    void* ws, const DeviceState& d, cudaStream_t st) {
+                    void* ws, const DeviceState& d, cudaStream_t st, bool accumulate = false) {
   if (g.n == 0) return CONV_OK;
   if (s.algo == CONV_ALGO_WINOGRAD) {
     const int m = s.wino_m, a2 = (m + 2) * (m + 2);
-    const long long tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
-    size_t u_bytes, per_img;
-    winograd_sizes(g, s.wino_store, m, &u_bytes, &per_img);
+    const bool cmajor = s.engine == CONV_ENGINE_SIMT;
+    const WinoLayout L = winograd_layout(g, s.wino_store, cmajor, m, s.nb);
     uint8_t* base = static_cast<uint8_t*>(ws);
     void* u = base;
-    void* v = base + u_bytes;
-    float* mb = reinterpret_cast<float*>(
-        base + u_bytes + align256((size_t)a2 * s.nb * tiles_per_img * g.c * dtype_size(s.wino_store)));
+    void* v = base + L.u_bytes;
+    float* mb = reinterpret_cast<float*>(base + L.u_bytes + L.v_bytes);
     cudaError_t e;
     {
       ProfScope ps(K_WINO_FILTER, st);
-      e = launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
+      e = cmajor ? launch_wino_filter_cmajor(w, g.w_row_stride, g.o, g.c, m, dt, round4(g.o), static_cast<float*>(u), st)
+                 : launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
     }
     if (e != cudaSuccess) return CONV_ERR_CUDA;
     for (int n0 = 0; n0 < g.n; n0 += s.nb) {
       const int nbi = std::min(s.nb, g.n - n0);
-      const long long t = (long long)nbi * tiles_per_img;
+      const long long t = (long long)nbi * L.tiles_per_img;
       {
         ProfScope ps(K_WINO_INPUT, st);
-        e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
+        if (cmajor && !(kF32VTileMajor && g.c % 4 == 0))
+          e = launch_wino_input_cmajor(in, g, n0, nbi, m, dt, static_cast<float*>(v), round4(t), st);
+        else
+          e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
       }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
-      BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb};
-      if (s.engine == CONV_ENGINE_TCGEN05) {
+      if (cmajor) {
+        ProfScope ps(K_WINO_GEMM_SIMT, st);
+        const bool tmajor = kF32VTileMajor && g.c % 4 == 0;
+        e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), mb, a2, (int)t, g.c, g.o,
+                                 tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
+      } else {
+        BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb};
         ProfScope ps(K_WINO_GEMM_TC, st);
         e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
-      } else {
-        ProfScope ps(K_WINO_GEMM_SIMT, st);
-        e = launch_simt_batched_gemm(bg, st);
       }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
       {
         ProfScope ps(K_WINO_OUTPUT, st);
-        e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, false, st);
+        e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, accumulate, st);
       }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
     }
@@ -371,11 +406,13 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
       gp.in_img_stride = (long long)g.h * g.w * s.cpad;
       gp.w_row_stride = (long long)g.kh * g.kw * s.cpad;
       ProfScope ps(K_TC_CONV, st);
-      return cuda_status(launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, st));
+      return cuda_status(
+          launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
     }
     if (tc_conv_supported(g, dt, in, w)) {
       ProfScope ps(K_TC_CONV, st);
-      return cuda_status(launch_tc_conv(in, w, out, g, dt, s.tile_n, d.props.sm_count, d.err_word, st));
+      return cuda_status(
+          launch_tc_conv(in, w, out, g, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
     }
     // Misaligned pointers: the any-alignment path below.
   }
@@ -383,7 +420,7 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
                    (g.in_img_stride % 4 == 0) && (g.w_row_stride % 4 == 0) &&
                    aligned16(in) && aligned16(w);
   ProfScope ps(K_SIMT_CONV, st);
-  return cuda_status(launch_simt_conv(in, w, out, g, dt, vec, false, st));
+  return cuda_status(launch_simt_conv(in, w, out, g, dt, vec, accumulate, st));
 }
 
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
@@ -441,9 +478,9 @@ conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_de
   if (st != CONV_OK) return st;
   st = select2d(*g2, dt, p, o, s);
   if (st != CONV_OK) return st;
-  // Scratch for the taps that are added (all but a first tap that covers every frame).
-  *tap_bytes = d->kd > 1 || d->pad[0] > 0 ? align256((size_t)*od * g2->oh * g2->ow * g2->o * dtype_size(dt)) : 0;
-  *ws_total = *tap_bytes + s->ws;
+  // Taps after the first add into out inside their own output stage: no tap scratch.
+  *tap_bytes = 0;
+  *ws_total = s->ws;
   return CONV_OK;
 }
 
@@ -583,9 +620,6 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
   Tap taps[1024];
   if (desc->kd > 1024) return CONV_ERR_UNSUPPORTED;
   const int ntaps = taps3d(desc, od, taps);
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  void* tap_buf = tap_bytes ? wsb : nullptr;
-  void* ws2 = tap_bytes ? wsb + tap_bytes : workspace;
   const bool first_covers_all = ntaps > 0 && taps[0].od_lo == 0 && taps[0].od_hi == od - 1;
 
   for (int n = 0; n < desc->n; ++n) {
@@ -602,15 +636,10 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
       const void* in_view = in_n + (size_t)t.id_lo * frame_in * esz;
       const void* w_slice = static_cast<const uint8_t*>(w) + (size_t)t.kd * desc->kh * desc->kw * desc->c * esz;
       uint8_t* out_view = out_n + (size_t)t.od_lo * frame_out * esz;
-      const bool direct_write = i == 0 && first_covers_all;
-      void* dst = direct_write ? static_cast<void*>(out_view) : tap_buf;
-      st = run2d(in_view, w_slice, dst, g, dtype, s, ws2, *d, st_);
+      // tap 0 writes (when it covers every frame); the others add in ascending kd order
+      const bool accumulate = !(i == 0 && first_covers_all);
+      st = run2d(in_view, w_slice, out_view, g, dtype, s, workspace, *d, st_, accumulate);
       if (st != CONV_OK) return st;
-      if (!direct_write) {
-        ProfScope ps(K_ACCUMULATE, st_);
-        if (launch_accumulate(out_view, tap_buf, (size_t)g.n * frame_out, dtype, st_) != cudaSuccess)
-          return CONV_ERR_CUDA;
-      }
     }
   }
   return CONV_OK;

@@ -83,10 +83,11 @@ def _lit(q: Fr) -> str:
     return s + "f"
 
 
-def _expr(row, src):
+def _expr(row, src, pick=None):
+    """Sum of row[k] * src[k] as C; pick limits the terms to a parity (0/1)."""
     terms = []
     for k, c in enumerate(row):
-        if c == 0:
+        if c == 0 or (pick is not None and k % 2 != pick):
             continue
         if c == 1:
             terms.append(f"+ {src}[{k}]")
@@ -102,29 +103,114 @@ def _expr(row, src):
     return s[2:] if s.startswith("+ ") else "-" + s[2:]
 
 
+def _row_pairs(M):
+    """Pairs (p, q, s_even, s_odd) with M[q][n] = s_even*M[p][n] for even n and
+    s_odd*M[p][n] for odd n, s_even = -s_odd: rows of a +-a point pair."""
+    used, pairs = set(), []
+    for p in range(len(M)):
+        if p in used:
+            continue
+        for q in range(p + 1, len(M)):
+            if q in used:
+                continue
+            for se in (1, -1):
+                so = -se
+                if all(M[q][n] == (se if n % 2 == 0 else so) * M[p][n] for n in range(len(M[p]))) and \
+                        any(M[p][n] != 0 for n in range(0, len(M[p]), 2)) and \
+                        any(M[p][n] != 0 for n in range(1, len(M[p]), 2)):
+                    pairs.append((p, q, se, so))
+                    used.update((p, q))
+                    break
+            if p in used:
+                break
+    return pairs
+
+
+def _emit_rows(name, M, n_in):
+    """y = M x with paired rows sharing their even / odd partial sums."""
+    out = [f"__device__ __forceinline__ void {name}(const float* x, float* y) {{"]
+    pairs = _row_pairs(M)
+    done = set()
+    for (p, q, se, so) in pairs:
+        out.append(f"  {{ const float e = {_expr(M[p], 'x', 0)}, o = {_expr(M[p], 'x', 1)};")
+        out.append(f"    y[{p}] = e + o;")
+        out.append(f"    y[{q}] = {'' if se > 0 else '-'}e {'-' if se > 0 else '+'} o; }}")
+        done.update((p, q))
+    for r in range(len(M)):
+        if r not in done:
+            out.append(f"  y[{r}] = {_expr(M[r], 'x')};")
+    out.append("}")
+    return out
+
+
+def _col_pairs(M):
+    """Column pairs (p, q) with M[i][q] = M[i][p] for even i and -M[i][p] for odd i."""
+    cols = len(M[0])
+    used, pairs = set(), []
+    for p in range(cols):
+        if p in used:
+            continue
+        for q in range(p + 1, cols):
+            if q in used:
+                continue
+            if all(M[i][q] == (1 if i % 2 == 0 else -1) * M[i][p] for i in range(len(M))) and \
+                    any(M[i][p] != 0 for i in range(len(M))):
+                pairs.append((p, q))
+                used.update((p, q))
+                break
+    return pairs
+
+
+def _emit_cols(name, M):
+    """y = M x with paired columns combined first: s = x_p + x_q, d = x_p - x_q."""
+    out = [f"__device__ __forceinline__ void {name}(const float* x, float* y) {{"]
+    pairs = _col_pairs(M)
+    paired = {}
+    for k, (p, q) in enumerate(pairs):
+        out.append(f"  const float s{k} = x[{p}] + x[{q}], d{k} = x[{p}] - x[{q}];")
+        paired[p] = k
+    lone = [c for c in range(len(M[0])) if all(c not in pq for pq in pairs)]
+    for i, row in enumerate(M):
+        terms = []
+        for c in lone:
+            if row[c] != 0:
+                terms.append((row[c], f"x[{c}]"))
+        for p, k in paired.items():
+            if row[p] != 0:
+                terms.append((row[p], f"{'s' if i % 2 == 0 else 'd'}{k}"))
+        parts = []
+        for c, v in terms:
+            if c == 1:
+                parts.append(f"+ {v}")
+            elif c == -1:
+                parts.append(f"- {v}")
+            elif c > 0:
+                parts.append(f"+ {_lit(c)} * {v}")
+            else:
+                parts.append(f"- {_lit(-c)} * {v}")
+        e = " ".join(parts) if parts else "0.0f"
+        e = e[2:] if e.startswith("+ ") else ("-" + e[2:] if e.startswith("- ") else e)
+        out.append(f"  y[{i}] = {e};")
+    out.append("}")
+    return out
+
+
 def emit() -> str:
     out = []
     out.append("// GENERATED by gen_winograd.py -- do not edit by hand.")
     out.append("// 1D Winograd F(m, 3) transforms, from the exact Cook-Toom matrices:")
     out.append("//   *_bt: y = B^T x (alpha -> alpha), *_g: y = G x (3 -> alpha), *_at: y = A^T x (alpha -> m).")
+    out.append("// Rows (B^T, G) or columns (A^T) belonging to a +-a point pair share their")
+    out.append("// even / odd partial sums, which halves the arithmetic.")
     out.append("#pragma once")
     out.append("")
     for m in sorted(POINTS):
         AT, G, BT = matrices(m)
         a = m + R - 1
         out.append(f"// F({m}x{m}, 3x3): alpha = {a}")
-        out.append(f"__device__ __forceinline__ void wino{m}_bt(const float* x, float* y) {{")
-        for j in range(a):
-            out.append(f"  y[{j}] = {_expr(BT[j], 'x')};")
-        out.append("}")
-        out.append(f"__device__ __forceinline__ void wino{m}_g(const float* x, float* y) {{")
-        for j in range(a):
-            out.append(f"  y[{j}] = {_expr(G[j], 'x')};")
-        out.append("}")
-        out.append(f"__device__ __forceinline__ void wino{m}_at(const float* x, float* y) {{")
-        for i in range(m):
-            out.append(f"  y[{i}] = {_expr(AT[i], 'x')};")
-        out.append("}")
+        out += _emit_rows(f"wino{m}_bt", BT, a)
+        out += _emit_rows(f"wino{m}_g", G, R)
+        out += _emit_cols(f"wino{m}_at", AT)
         out.append("")
     return "\n".join(out) + "\n"
 

@@ -47,7 +47,7 @@ struct BatchedGemm {
 // ---- kernel launchers (return a CUDA error; never synchronise) ----
 
 // SIMT implicit GEMM (FFMA, fp32 accumulate): any dtype, any alignment when
-// vec == false.  accumulate: out = round(out + result).
+// vec == false.  accumulate: out = round(out + round(result)).
 cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geom& g,
                              conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s);
 // SIMT batched GEMM on fp32 operands (Winograd fp32 path).
@@ -56,9 +56,10 @@ cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s);
 // tcgen05 implicit GEMM for 16-bit dtypes (TMA im2col staging, TMEM accumulators).
 // Returns cudaErrorNotSupported if the shape cannot be encoded as TMA maps.
 bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w);
+// accumulate: out = round(out + round(result)), the unfused depth-tap add's arithmetic.
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
                            conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
-                           cudaStream_t s);
+                           bool accumulate, cudaStream_t s);
 // tcgen05 batched GEMM for 16-bit operands with fp32 D (Winograd 16-bit path).
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n,
                                    int sm_count, int* err_word, cudaStream_t s);
@@ -72,6 +73,16 @@ cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int
 cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int m,
                               conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_tile,
                               cudaStream_t s);
+// Channel-major fp32 variants for the FFMA GEMM: U[xi][c][o_pad], V[xi][c][t_stride].
+cudaError_t launch_wino_filter_cmajor(const void* w, long long w_row_stride, int o, int c, int m,
+                                      conv_dtype_t in_dt, long long o_pad, float* u, cudaStream_t s);
+cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int nb, int m, conv_dtype_t in_dt,
+                                     float* v, long long t_stride, cudaStream_t s);
+// Batched FFMA GEMM D[b][t][o] = sum_c A[b][.][.] * B[b][c][o]; A is [C][lda] (channel-major)
+// or, with a_tmajor, [T][lda] (tile-major); B row stride ldb.
+cudaError_t launch_wino_gemm_f32(const float* a, const float* b, float* d, int batches, int t, int c, int o,
+                                 long long lda, long long ldb, bool a_tmajor, cudaStream_t s);
+int wino_gemm_f32_tile_n(int o);
 cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb, int m,
                                long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
                                cudaStream_t s);

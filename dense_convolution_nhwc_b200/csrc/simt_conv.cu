@@ -201,7 +201,7 @@ simt_conv_kernel(const SimtArgs a) {
       int o = n0 + 32 * (j >> 1) + tx * 2 + (j & 1);
       if (o < a.o) {
         float v = acc[i][j];
-        if (a.accumulate) v += Store<T>::to_f32(orow[o]);
+        if (a.accumulate) v = Store<T>::to_f32(orow[o]) + Store<T>::to_f32(Store<T>::from_f32(v));
         orow[o] = Store<T>::from_f32(v);
       }
     }

@@ -65,6 +65,7 @@ struct TcArgs {
   void* out;
   long long ldo;               // elements between output rows
   long long out_batch;         // elements between batches
+  int accumulate;              // out = round(out + round(acc)) instead of out = round(acc)
   int* err;
 };
 
@@ -374,7 +375,33 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (c0 >= a.ocols) continue;
         TOut* p = orow + c0;
         const bool full = c0 + 32 <= a.ocols;
-        if constexpr (sizeof(TOut) == 4) {
+        if (a.accumulate) {
+          // depth-tap accumulate: round the tap to the storage type, add in fp32, round again
+          constexpr int E = 16 / sizeof(TOut);                 // elements per 16-byte vector
+          if (full && ((reinterpret_cast<uintptr_t>(p) & 15) == 0)) {
+            uint4 old[32 / E];
+#pragma unroll
+            for (int v = 0; v < 32 / E; ++v) old[v] = reinterpret_cast<const uint4*>(p)[v];
+#pragma unroll
+            for (int v = 0; v < 32 / E; ++v) {
+              TOut* e = reinterpret_cast<TOut*>(&old[v]);
+#pragma unroll
+              for (int k = 0; k < E; ++k) {
+                const float tap = Store<TOut>::to_f32(Store<TOut>::from_f32(__uint_as_float(r[v * E + k])));
+                e[k] = Store<TOut>::from_f32(Store<TOut>::to_f32(e[k]) + tap);
+              }
+              reinterpret_cast<uint4*>(p)[v] = old[v];
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < a.ocols) {
+                const float tap = Store<TOut>::to_f32(Store<TOut>::from_f32(__uint_as_float(r[j])));
+                p[j] = Store<TOut>::from_f32(Store<TOut>::to_f32(p[j]) + tap);
+              }
+            }
+          }
+        } else if constexpr (sizeof(TOut) == 4) {
           if (full && ((reinterpret_cast<uintptr_t>(p) & 15) == 0)) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
@@ -529,7 +556,7 @@ bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const voi
 }
 
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt,
-                           int tile_n, int sm_count, int* err_word, cudaStream_t s) {
+                           int tile_n, int sm_count, int* err_word, bool accumulate, cudaStream_t s) {
   if (!tc_conv_supported(g, dt, in, w)) return cudaErrorNotSupported;
   const long long M = (long long)g.n * g.oh * g.ow;
   if (M == 0) return cudaSuccess;
@@ -565,6 +592,7 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   a.out = out;
   a.ldo = g.o;
   a.out_batch = 0;
+  a.accumulate = accumulate ? 1 : 0;
   a.err = err_word;
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, true, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)

@@ -195,10 +195,152 @@ wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __re
       if (xo < a.ow) {
         Tout* p = op + ((long long)y * a.ow + xo) * a.o;
         float val = res[j];
-        if (a.accumulate) val += Store<Tout>::to_f32(*p);
+        if (a.accumulate) val = Store<Tout>::to_f32(*p) + Store<Tout>::to_f32(Store<Tout>::from_f32(val));
         *p = Store<Tout>::from_f32(val);
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Channel-major variants for the FFMA GEMM: U[xi][c][o] (row stride O_pad) and
+// V[xi][c][t] (row stride T_pad), fp32.  Rows of both are contiguous in the
+// GEMM's m / n direction, so the GEMM stages them with 16-byte copies.
+// ---------------------------------------------------------------------------
+template <int M, typename Tin>
+__global__ void wino_filter_cmajor_kernel(const Tin* __restrict__ w, long long w_row_stride, int O, int C,
+                                          long long o_pad, float* __restrict__ u) {
+  constexpr int A = Wino<M>::A;
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)O * C) return;
+  const int c = (int)(idx / O), o = (int)(idx - (long long)c * O);    // o fastest: coalesced stores
+  const Tin* wp = w + (long long)o * w_row_stride + c;
+  float g[3][3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) g[i][j] = Store<Tin>::to_f32(wp[(long long)(i * 3 + j) * C]);
+  float t[A][3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    float col[3] = {g[0][j], g[1][j], g[2][j]}, r[A];
+    Wino<M>::g(col, r);
+#pragma unroll
+    for (int i = 0; i < A; ++i) t[i][j] = r[i];
+  }
+  const long long plane = (long long)C * o_pad;
+  float* up = u + (long long)c * o_pad + o;
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    float r[A];
+    Wino<M>::g(t[i], r);
+#pragma unroll
+    for (int j = 0; j < A; ++j) up[(long long)(i * A + j) * plane] = r[j];
+  }
+}
+
+// Input transform, channel-major output.  A block transforms a strip of
+// kStripTiles consecutive tiles of one tile row, for kStripChans channels:
+// the strip's alpha rows x (kStripTiles*m + 2) columns x channels are staged
+// in shared memory ([c][y][x]) with sector-sized global reads, then thread
+// (tile, channel) transforms its alpha x alpha patch and writes V[xi][c][t]
+// with consecutive threads on consecutive tiles (128-byte rows).
+constexpr int kStripTiles = 32;
+constexpr int kStripChans = 8;
+
+template <int M>
+struct Strip {
+  static constexpr int A = M + 2;
+  static constexpr int W = kStripTiles * M + 2;               // staged columns
+  static constexpr int WP = W + ((1 - W) % 4 + 4) % 4;        // padded row: WP = 1 (mod 4)
+  static constexpr int BYTES = kStripChans * A * WP * 4;
+};
+
+struct WinoInCArgs {
+  int h, w, c, ph, pw, tiles_h, tiles_w, strips_w;
+  long long in_img_stride;
+  int n0;
+  long long t_stride;     // row stride of V (T_pad)
+};
+
+template <int M, typename Tin>
+__global__ void __launch_bounds__(256)
+wino_input_cmajor_kernel(const Tin* __restrict__ in, const WinoInCArgs a, float* __restrict__ v) {
+  constexpr int A = Wino<M>::A;
+  using S = Strip<M>;
+  extern __shared__ float sm[];     // [kStripChans][A][S::WP]
+  const int tid = threadIdx.x;
+  // blockIdx.x -> (image, tile row, strip, channel group), channel group fastest so
+  // that concurrently running blocks together read whole pixels (C contiguous).
+  const int cgroups = (a.c + kStripChans - 1) / kStripChans;
+  const long long bid = blockIdx.x;
+  const int cg = (int)(bid % cgroups);
+  const long long strip = bid / cgroups;
+  const int strips_per_img = a.tiles_h * a.strips_w;
+  const int nl = (int)(strip / strips_per_img);
+  const int r = (int)(strip - (long long)nl * strips_per_img);
+  const int ty = r / a.strips_w, sx = r - (r / a.strips_w) * a.strips_w;
+  const int c0 = cg * kStripChans;
+  const int y0 = ty * M - a.ph, x0 = sx * kStripTiles * M - a.pw;
+  const Tin* base = in + (long long)(a.n0 + nl) * a.in_img_stride;
+
+  // Stage: 4 channels per load (16 bytes for fp32) when the rows allow it.
+  const bool vec4 = (a.c % 4 == 0) && ((reinterpret_cast<uintptr_t>(in) & (4 * sizeof(Tin) - 1)) == 0) &&
+                    (a.in_img_stride % 4 == 0);
+  constexpr int Q = kStripChans / 4;
+  for (int idx = tid; idx < A * S::W * Q; idx += 256) {
+    const int q = idx % Q;
+    const int rest = idx / Q;
+    const int x = rest % S::W, y = rest / S::W;
+    const int gy = y0 + y, gx = x0 + x, c = c0 + 4 * q;
+    float val[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (gy >= 0 && gy < a.h && gx >= 0 && gx < a.w && c < a.c) {
+      const Tin* p = base + ((long long)gy * a.w + gx) * a.c + c;
+      if (vec4) {
+        if constexpr (sizeof(Tin) == 4) {
+          const float4 f = __ldg(reinterpret_cast<const float4*>(p));
+          val[0] = f.x; val[1] = f.y; val[2] = f.z; val[3] = f.w;
+        } else {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+          const Tin* e = reinterpret_cast<const Tin*>(&u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) val[k] = Store<Tin>::to_f32(e[k]);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (c + k < a.c) val[k] = Store<Tin>::to_f32(p[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sm[((4 * q + k) * A + y) * S::WP + x] = val[k];
+  }
+  __syncthreads();
+
+  const int txl = tid % kStripTiles, cl = tid / kStripTiles;
+  const int tx = sx * kStripTiles + txl;
+  const int c = c0 + cl;
+  if (tx >= a.tiles_w || c >= a.c) return;
+  const float* sp = sm + cl * A * S::WP + txl * M;
+  float tt[A][A];
+#pragma unroll
+  for (int j = 0; j < A; ++j) {
+    float col[A], res[A];
+#pragma unroll
+    for (int i = 0; i < A; ++i) col[i] = sp[i * S::WP + j];
+    Wino<M>::bt(col, res);
+#pragma unroll
+    for (int i = 0; i < A; ++i) tt[i][j] = res[i];
+  }
+  const long long t = (long long)nl * a.tiles_h * a.tiles_w + (long long)ty * a.tiles_w + tx;
+  const long long plane = (long long)a.c * a.t_stride;
+  float* vp = v + (long long)c * a.t_stride + t;
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    float res[A];
+    Wino<M>::bt(tt[i], res);
+#pragma unroll
+    for (int j = 0; j < A; ++j) vp[(long long)(i * A + j) * plane] = res[j];
   }
 }
 
@@ -269,6 +411,49 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
                                                               static_cast<Tst*>(v));
         return cudaGetLastError();
       });
+    });
+  });
+}
+
+cudaError_t launch_wino_filter_cmajor(const void* w, long long w_row_stride, int o, int c, int m,
+                                      conv_dtype_t in_dt, long long o_pad, float* u, cudaStream_t s) {
+  long long n = (long long)o * c;
+  if (n == 0) return cudaSuccess;
+  unsigned blocks = (unsigned)((n + 255) / 256);
+  return by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return by_dt(in_dt, [&](auto ti) {
+      using Tin = decltype(ti);
+      wino_filter_cmajor_kernel<M, Tin><<<blocks, 256, 0, s>>>(static_cast<const Tin*>(w), w_row_stride, o, c,
+                                                                o_pad, u);
+      return cudaGetLastError();
+    });
+  });
+}
+
+cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int nb, int m, conv_dtype_t in_dt,
+                                     float* v, long long t_stride, cudaStream_t s) {
+  WinoInCArgs a{};
+  a.h = g.h; a.w = g.w; a.c = g.c; a.ph = g.ph; a.pw = g.pw;
+  a.tiles_h = (g.oh + m - 1) / m;
+  a.tiles_w = (g.ow + m - 1) / m;
+  a.strips_w = (a.tiles_w + kStripTiles - 1) / kStripTiles;
+  a.in_img_stride = g.in_img_stride;
+  a.n0 = n0;
+  a.t_stride = t_stride;
+  const long long blocks = (long long)nb * a.tiles_h * a.strips_w * ((g.c + kStripChans - 1) / kStripChans);
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)blocks);
+  return by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return by_dt(in_dt, [&](auto ti) {
+      using Tin = decltype(ti);
+      auto k = wino_input_cmajor_kernel<M, Tin>;
+      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Strip<M>::BYTES);
+      if (e != cudaSuccess) return e;
+      k<<<grid, 256, Strip<M>::BYTES, s>>>(static_cast<const Tin*>(in), a, v);
+      return cudaGetLastError();
     });
   });
 }
