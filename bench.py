@@ -88,12 +88,14 @@ def workload(name):
         dt = name.split("_")[1]
         return ("conv3d bf16 NDHWC 3x3x3 s1 spatial pad 1 depth pad 0 N=1 depth taps: 17x64x64 256->256, "
                 "41x60x104 256->256, 41x120x208 512->512", [Conv(s, dt, "normal") for s in synth.CONV3D_TAPS], dt)
-    if name.startswith("wide_"):
+    if name.startswith("wide_") or name.startswith("wide3_"):
         # wide_<dtype>: C_out >= 512 and M >= 16384 aligned members of the sweep
         dt = name.split("_")[1]
         shapes = [s for s in synth.wide_sweep(True) if s.o >= 512 and s.n * s.oh * s.ow >= 16384]
         if not name.endswith("_all"):
             shapes = [s for s in shapes if s.stride == (1, 1) and s.dilation == (1, 1)]
+        if name.startswith("wide3_"):     # the 3x3 members (the ones Winograd can also run)
+            shapes = [s for s in shapes if s.kh == 3]
         return (f"wide-channel implicit-GEMM sweep {dt}: C_out>=512, M>=16384, aligned ({len(shapes)} shapes)",
                 [Conv(s, dt, "normal") for s in shapes], dt)
     raise SystemExit(f"unknown workload {name}")
@@ -114,6 +116,13 @@ def kernel_work(conv, plan):
         f0, b0 = w.get(k, (0.0, 0.0))
         w[k] = (f0 + f, b0 + b)
 
+    if conv.is3d and plan["taps"] == 1 and plan["engine"] == "tcgen05":
+        # native K-fused 3D implicit GEMM: one pass, output written once
+        M = s.n * s.od * s.oh * s.ow
+        K = s.c * s.kd * s.kh * s.kw
+        add("tc_conv3d", 2.0 * M * s.o * K,
+            (s.n * s.d * s.h * s.w * s.c + s.o * K + M * s.o) * esz)
+        return w
     if conv.is3d:
         frames_out = s.od
         n2 = synth.Conv2dShape(frames_out, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride[1:], s.pad[1:], s.dilation[1:])
@@ -148,7 +157,7 @@ def kernel_work(conv, plan):
 
 
 def kernel_bound(name):
-    if name in ("tc_conv", "wino_gemm_tc"):
+    if name in ("tc_conv", "tc_conv3d", "wino_gemm_tc"):
         return "tensor"
     if name in ("simt_conv", "wino_gemm_simt"):
         return "alu"
@@ -158,6 +167,7 @@ def kernel_bound(name):
 KERNEL_SOURCES = {
     "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["wino_gemm_f32.cu"],
     "tc_conv": ["tc_conv.cu", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "common.cuh"],
+    "tc_conv3d": ["tc_conv.cu", "common.cuh"],
     "wino_input": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
     "wino_output": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
     "wino_filter": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
@@ -506,7 +516,10 @@ def main():
             "algorithmic_per_launch": (kd["bytes_per_step"] if bound == "hbm" else kd["flops_per_step"]) / launches_step}
     gpu_launches = int(round(sum(l for l, _ in prof.values())))
 
-    # e2e through the C ABI with host buffers
+    # e2e through the C ABI with host buffers.  Images are independent, so each
+    # conv's batch is cut into chunks that flow through three streams: the
+    # host->device copy of chunk i+1 and the device->host copy of chunk i-1
+    # overlap the conv of chunk i (copy engines and SMs work at the same time).
     e2e = None
     if not args.no_e2e:
         hx = [x.cpu().pin_memory() for _, x, *_ in items]
@@ -515,18 +528,48 @@ def main():
         dx = [torch.empty_like(x) for _, x, *_ in items]
         dw = [torch.empty_like(w) for _, _, w, *_ in items]
         k_e2e = max(1, min(args.steps, 3))
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        chunk_descs = []
+        for j, (cv, x, w, d, plan, out) in enumerate(items):
+            s = cv.shape
+            nchunk = min(s.n, 8) if not cv.is3d else 1
+            bounds = [round(i * s.n / nchunk) for i in range(nchunk + 1)]
+            cds = []
+            for c0, c1 in zip(bounds[:-1], bounds[1:]):
+                if c1 <= c0:
+                    continue
+                if cv.is3d:
+                    dd = d
+                else:
+                    dd = B.make_desc2d(c1 - c0, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
+                cds.append((c0, c1, dd))
+            chunk_descs.append(cds)
 
         def e2e_step():
-            for j in range(len(items)):
-                dx[j].copy_(hx[j], non_blocking=True)
-                dw[j].copy_(hw[j], non_blocking=True)
             for j, (cv, x, w, d, plan, out) in enumerate(items):
-                st = fwd(dx[j].data_ptr(), dw[j].data_ptr(), out.data_ptr(), d, dt_code, opts, ws.data_ptr(),
-                         ws.numel(), sptr)
-                if st != 0:
-                    raise B.ConvError(st, cv.name)
-            for j, (*_, out) in enumerate(items):
-                hout[j].copy_(out, non_blocking=True)
+                ev_in = []
+                with torch.cuda.stream(s_in):
+                    dw[j].copy_(hw[j], non_blocking=True)
+                    for (c0, c1, dd) in chunk_descs[j]:
+                        dx[j][c0:c1].copy_(hx[j][c0:c1], non_blocking=True)
+                        e = torch.cuda.Event()
+                        e.record(s_in)
+                        ev_in.append(e)
+                for (c0, c1, dd), e in zip(chunk_descs[j], ev_in):
+                    stream.wait_event(e)
+                    st = fwd(dx[j][c0:c1].data_ptr(), dw[j].data_ptr(), out[c0:c1].data_ptr(), dd, dt_code, opts,
+                             ws.data_ptr(), ws.numel(), sptr)
+                    if st != 0:
+                        raise B.ConvError(st, cv.name)
+                    e2 = torch.cuda.Event()
+                    e2.record(stream)
+                    s_out.wait_event(e2)
+                    with torch.cuda.stream(s_out):
+                        hout[j][c0:c1].copy_(out[c0:c1], non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(s_out)
+            stream.wait_event(done)
+            s_in.wait_stream(stream)   # the next step's uploads wait for this step's convs
 
         e2e_step()
         torch.cuda.synchronize()
@@ -541,7 +584,9 @@ def main():
         h2d = sum(t.numel() * t.element_size() for t in hx + hw)
         d2h = sum(t.numel() * t.element_size() for t in hout)
         e2e = {"value": world * total_flops / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": k_e2e,
+               "how": "per conv, the batch in up to 8 chunks; H2D of chunk i+1 and D2H of chunk i-1 overlap the "
+                      "conv of chunk i on separate streams; pinned host buffers"}
         del hx, hw, hout, dx, dw
 
     cpu = None
@@ -598,9 +643,22 @@ def main():
                     evs[1].record(stream)
                     torch.cuda.synchronize()
                     t = evs[0].elapsed_time(evs[1]) / reps
+                B.conv_profile_begin()
+                for _ in range(reps):
+                    fwd_one()
+                torch.cuda.synchronize()
+                kp = B.profile_end()
+                kw = kernel_work(cv, plan)
+                ker = {}
+                for kn, (nl, tot) in kp.items():
+                    kms = tot / reps
+                    f, b = kw.get(kn, (0.0, 0.0))
+                    ker[kn] = {"ms": kms, "tflops": f / (kms * 1e-3) / 1e12 if f else None,
+                               "gbs": b / (kms * 1e-3) / 1e9 if b else None}
                 print(json.dumps({"conv": cv.name, "dtype": cv.dtype, "algo": plan["algo"], "engine": plan["engine"],
                                   "tile_n": plan["tile_n"], "ms": t, "tflops": cv.flops / (t * 1e-3) / 1e12,
-                                  "frac_of_bf16_peak": cv.flops / (t * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0)}))
+                                  "frac_of_bf16_peak": cv.flops / (t * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0),
+                                  "kernels": ker}))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -76,9 +76,9 @@ long long out_extent(long long in, int k, int s, int p, int d) {
 // ------------------------------ profiling ------------------------------------
 // Opt-in: each kernel launch is bracketed by two events on its stream.
 
-enum Kind { K_TC_CONV, K_SIMT_CONV, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
+enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
             K_WINO_OUTPUT, K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
-const char* const kKindName[K_COUNT] = {"tc_conv", "simt_conv", "wino_filter", "wino_input", "wino_gemm_tc",
+const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "wino_filter", "wino_input", "wino_gemm_tc",
                                         "wino_gemm_simt", "wino_output", "accumulate", "channel_pad", "fill"};
 
 struct ProfRecord {
@@ -470,16 +470,66 @@ int taps3d(const conv3d_desc_t* d, long long od, Tap* taps) {
   return n;
 }
 
+Geom3 geom3_of(const conv3d_desc_t* d, long long od, const Geom& g2) {
+  Geom3 g{};
+  g.n = d->n; g.d = d->d; g.h = d->h; g.w = d->w; g.c = d->c; g.o = d->o;
+  g.kd = d->kd; g.kh = d->kh; g.kw = d->kw;
+  g.sd = d->stride[0]; g.sh = d->stride[1]; g.sw = d->stride[2];
+  g.pd = d->pad[0]; g.ph = d->pad[1]; g.pw = d->pad[2];
+  g.dd = d->dilation[0]; g.dh = d->dilation[1]; g.dw = d->dilation[2];
+  g.od = (int)od; g.oh = g2.oh; g.ow = g2.ow;
+  return g;
+}
+
+// The depth-tap page's guard ("Decompose small kernel-depth 3D convs into 2D
+// convs", Change): N == 1, KD <= 7, depth stride 1, kernel dilation 1, no depth
+// padding, channel counts that are multiples of 16.
+bool depth_tap_guard(const conv3d_desc_t* d) {
+  return d->n == 1 && d->kd <= 7 && d->stride[0] == 1 && d->dilation[0] == 1 && d->dilation[1] == 1 &&
+         d->dilation[2] == 1 && d->pad[0] == 0 && d->c % 16 == 0 && d->o % 16 == 0;
+}
+
+// The native 3D implicit GEMM can express this shape (pointers are checked at launch).
+bool native3d_shape_ok(const Geom3& g, conv_dtype_t dt, const conv_device_props_t& p) {
+  if (dt == CONV_F32 || p.cc_major != 10 || g.c % 8 != 0) return false;
+  if (g.sd > 8 || g.sh > 8 || g.sw > 8) return false;
+  const int lo[3] = {-g.pw, -g.ph, -g.pd};
+  const int up[3] = {g.pw - g.dw * (g.kw - 1), g.ph - g.dh * (g.kh - 1), g.pd - g.dd * (g.kd - 1)};
+  for (int i = 0; i < 3; ++i)
+    if (lo[i] < -16 || lo[i] > 15 || up[i] < -16 || up[i] > 15) return false;
+  return (long long)g.dw * (g.kw - 1) <= 65535 && (long long)g.dh * (g.kh - 1) <= 65535 &&
+         (long long)g.dd * (g.kd - 1) <= 65535;
+}
+
 conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_device_props_t& p,
                           const conv_options_t& o, Sel* s, Geom* g2, long long* od, size_t* ws_total,
-                          size_t* tap_bytes) {
+                          bool* native) {
   if (!valid_dtype(dt)) return CONV_ERR_INVALID;
   conv_status_t st = geom3d(d, od, g2);
   if (st != CONV_OK) return st;
+  const Geom3 g3 = geom3_of(d, *od, *g2);
+  const bool can_native = native3d_shape_ok(g3, dt, p);
+  // Auto: the page's guard keeps the depth taps; the cases it sends to a native
+  // 3D kernel go to the K-fused tcgen05 implicit GEMM.  Forcing the implicit
+  // GEMM asks for the native kernel whenever it can run the shape.
+  *native = can_native && ((o.algo == CONV_ALGO_AUTO && !depth_tap_guard(d)) || o.algo == CONV_ALGO_IMPLICIT_GEMM);
+  if (*native) {
+    s->algo = CONV_ALGO_IMPLICIT_GEMM;
+    s->engine = CONV_ENGINE_TCGEN05;
+    s->tile_m = 128;
+    const long long m_tiles = ((long long)d->n * *od * g2->oh * g2->ow + 127) / 128;
+    s->tile_n = d->o <= 128 || m_tiles * ((d->o + 255) / 256) < p.sm_count ? 128 : 256;
+    s->wino_m = 0;
+    s->nb = d->n;
+    s->ntiles = 1;
+    s->cpad = 0;
+    s->ws = 0;
+    *ws_total = 0;
+    return CONV_OK;
+  }
   st = select2d(*g2, dt, p, o, s);
   if (st != CONV_OK) return st;
   // Taps after the first add into out inside their own output stage: no tap scratch.
-  *tap_bytes = 0;
   *ws_total = s->ws;
   return CONV_OK;
 }
@@ -571,10 +621,11 @@ conv_status_t conv3d_plan_for_props(const conv3d_desc_t* desc, conv_dtype_t dtyp
   Sel s;
   Geom g2;
   long long od;
-  size_t ws, tap_bytes;
-  conv_status_t st = plan3d_impl(desc, dtype, *props, effective_options(opts), &s, &g2, &od, &ws, &tap_bytes);
+  size_t ws;
+  bool native = false;
+  conv_status_t st = plan3d_impl(desc, dtype, *props, effective_options(opts), &s, &g2, &od, &ws, &native);
   if (st != CONV_OK) return st;
-  fill_plan(s, plan, desc->kd, ws);
+  fill_plan(s, plan, native ? 1 : desc->kd, ws);
   return CONV_OK;
 }
 
@@ -601,8 +652,9 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
   Sel s;
   Geom g2;
   long long od;
-  size_t ws, tap_bytes;
-  st = plan3d_impl(desc, dtype, d->props, effective_options(opts), &s, &g2, &od, &ws, &tap_bytes);
+  size_t ws;
+  bool native = false;
+  st = plan3d_impl(desc, dtype, d->props, effective_options(opts), &s, &g2, &od, &ws, &native);
   if (st != CONV_OK) return st;
   if (desc->n == 0) return CONV_OK;
   if (!in || !w || !out) return CONV_ERR_INVALID;
@@ -617,6 +669,18 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
     return CONV_ERR_INVALID;
 
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  if (native) {
+    const Geom3 g3 = geom3_of(desc, od, g2);
+    if (tc_conv3d_supported(g3, dtype, in, w)) {
+      ProfScope ps(K_TC_CONV3D, st_);
+      return cuda_status(launch_tc_conv3d(in, w, out, g3, dtype, s.tile_n, d->props.sm_count, d->err_word, st_));
+    }
+    // misaligned pointers: depth taps on the any-alignment path
+    conv_options_t o2 = effective_options(opts);
+    o2.algo = CONV_ALGO_DIRECT;
+    st = select2d(g2, dtype, d->props, o2, &s);
+    if (st != CONV_OK) return st;
+  }
   Tap taps[1024];
   if (desc->kd > 1024) return CONV_ERR_UNSUPPORTED;
   const int ntaps = taps3d(desc, od, taps);

@@ -35,6 +35,13 @@ struct Geom {
   long long out_img_stride;   // elements (OH*OW*O for a dense NHWC output)
 };
 
+// One 3D convolution (NDHWC input, O,KD,KH,KW,I weights, dense NDHWC output).
+struct Geom3 {
+  int n, d, h, w, c, o, kd, kh, kw;
+  int sd, sh, sw, pd, ph, pw, dd, dh, dw;
+  int od, oh, ow;
+};
+
 // Batched GEMM view used by the Winograd path: for b < batches,
 //   D_b[t][o] = sum_c A_b[t][c] * B_b[o][c]   (A: [batches][T][C], B: [batches][O][C])
 struct BatchedGemm {
@@ -60,6 +67,11 @@ bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const voi
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
                            conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
                            bool accumulate, cudaStream_t s);
+// Native 3D implicit GEMM on tcgen05: K = KD*KH*KW*C in one main loop, the A
+// tiles gathered by a 5D TMA im2col map (corners limited to [-16, 15]).
+bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w);
+cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geom3& g, conv_dtype_t dt, int tile_n,
+                             int sm_count, int* err_word, cudaStream_t s);
 // tcgen05 batched GEMM for 16-bit operands with fp32 D (Winograd 16-bit path).
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n,
                                    int sm_count, int* err_word, cudaStream_t s);

@@ -60,6 +60,7 @@ struct TcArgs {
   int kb_per_tap, taps;
   int kw, dh, dw;
   int oh, ow, sh, sw, ph, pw;
+  int kh, od, sd, pd, dd;      // depth axis of the native 3D mode (kh splits a tap into kd, kh, kw)
   long long m_rows;            // rows per batch
   int ocols;                   // output columns (O)
   void* out;
@@ -138,6 +139,17 @@ __device__ __forceinline__ void tma_load_im2col_4d(uint32_t dst, const CUtensorM
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_im2col_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                   int c, int w, int h, int d, int n, uint16_t off_w,
+                                                   uint16_t off_h, uint16_t off_d) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], {%8, %9, %10};" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c), "r"(w), "r"(h), "r"(d), "r"(n), "h"(off_w),
+      "h"(off_h), "h"(off_d)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -191,7 +203,8 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt) {
 
 // --------------------------------- kernel -----------------------------------
 
-template <int BN, bool IM2COL, typename TIn, typename TOut>
+// MODE 0: batched GEMM (tiled A); 1: conv2d (4D im2col A); 2: conv3d (5D im2col A).
+template <int BN, int MODE, typename TIn, typename TOut>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcArgs a) {
@@ -255,15 +268,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const long long rest = tile / a.n_tiles;
         const int mt = (int)(rest % a.m_tiles);
         const int b = (int)(rest / a.m_tiles);
-        int img = 0, wx = 0, hy = 0;
-        if (IM2COL) {
+        int img = 0, wx = 0, hy = 0, dz = 0;
+        if (MODE != 0) {
+          // first output pixel of the tile -> its window's corner in the input
           const long long m0 = (long long)mt * BM;
           const long long ohw = (long long)a.oh * a.ow;
-          img = (int)(m0 / ohw);
-          const int rem = (int)(m0 - (long long)img * ohw);
+          long long fr = m0 / ohw;                   // image (2D) or image*OD + od (3D)
+          const int rem = (int)(m0 - fr * ohw);
           const int oy = rem / a.ow, ox = rem - (rem / a.ow) * a.ow;
           wx = ox * a.sw - a.pw;
           hy = oy * a.sh - a.ph;
+          if (MODE == 2) {
+            const int odz = (int)(fr % a.od);
+            fr /= a.od;
+            dz = odz * a.sd - a.pd;
+          }
+          img = (int)fr;
         }
         for (int ks = 0; ks < ksteps; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err, DEVERR_TIMEOUT_PRODUCER)) {
@@ -276,10 +296,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           mbar_expect_tx(fb, C::STAGE_BYTES);
           const uint32_t dA = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t dB = smem_u32(sB + stage * C::B_BYTES);
-          if (IM2COL) {
+          if (MODE == 1) {
             const int ky = tap / a.kw, kx = tap - (tap / a.kw) * a.kw;
             tma_load_im2col_4d(dA, &tmA, fb, kb * BK, wx, hy, img, (uint16_t)(kx * a.dw),
                                (uint16_t)(ky * a.dh));
+            tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
+          } else if (MODE == 2) {
+            const int khw = a.kh * a.kw;
+            const int kz = tap / khw, r2 = tap - kz * khw;
+            const int ky = r2 / a.kw, kx = r2 - (r2 / a.kw) * a.kw;
+            tma_load_im2col_5d(dA, &tmA, fb, kb * BK, wx, hy, dz, img, (uint16_t)(kx * a.dw),
+                               (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
             tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
           } else {
             tma_load_3d(dA, &tmA, fb, kb * BK, mt * BM, b);
@@ -519,10 +546,10 @@ cudaError_t set_smem(K kernel, int bytes) {
   return e;
 }
 
-template <int BN, bool IM2COL, typename TIn, typename TOut>
+template <int BN, int MODE, typename TIn, typename TOut>
 cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int sm_count,
                           cudaStream_t s) {
-  auto k = tc_gemm_kernel<BN, IM2COL, TIn, TOut>;
+  auto k = tc_gemm_kernel<BN, MODE, TIn, TOut>;
   cudaError_t e = set_smem(k, Cfg<BN>::SMEM);
   if (e != cudaSuccess) return e;
   long long tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
@@ -595,10 +622,72 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   a.accumulate = accumulate ? 1 : 0;
   a.err = err_word;
   if (dt == CONV_BF16)
-    return tile_n == 256 ? launch_kernel<256, true, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, true, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
-  return tile_n == 256 ? launch_kernel<256, true, __half, __half>(tA, tB, a, sm_count, s)
-                       : launch_kernel<128, true, __half, __half>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
+  return tile_n == 256 ? launch_kernel<256, 1, __half, __half>(tA, tB, a, sm_count, s)
+                       : launch_kernel<128, 1, __half, __half>(tA, tB, a, sm_count, s);
+}
+
+bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w) {
+  if (dt == CONV_F32) return false;
+  if (!driver_fns()) return false;
+  if (g.c % 8 != 0) return false;
+  if ((reinterpret_cast<uintptr_t>(in) & 15) || (reinterpret_cast<uintptr_t>(w) & 15)) return false;
+  if (g.sd > 8 || g.sh > 8 || g.sw > 8) return false;
+  // 5D im2col bounding-box corners are limited to [-16, 15] per axis
+  const int lo[3] = {-g.pw, -g.ph, -g.pd};
+  const int up[3] = {g.pw - g.dw * (g.kw - 1), g.ph - g.dh * (g.kh - 1), g.pd - g.dd * (g.kd - 1)};
+  for (int i = 0; i < 3; ++i)
+    if (lo[i] < -16 || lo[i] > 15 || up[i] < -16 || up[i] > 15) return false;
+  if ((long long)g.dw * (g.kw - 1) > 65535 || (long long)g.dh * (g.kh - 1) > 65535 ||
+      (long long)g.dd * (g.kd - 1) > 65535)
+    return false;
+  return g.n > 0 && g.od > 0 && g.oh > 0 && g.ow > 0;
+}
+
+cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geom3& g, conv_dtype_t dt, int tile_n,
+                             int sm_count, int* err_word, cudaStream_t s) {
+  if (!tc_conv3d_supported(g, dt, in, w)) return cudaErrorNotSupported;
+  const long long M = (long long)g.n * g.od * g.oh * g.ow;
+  if (M == 0) return cudaSuccess;
+  CUtensorMap tA, tB;
+  {
+    // A: im2col view of the NDHWC input (C, W, H, D, N)
+    cuuint64_t dims[5] = {(cuuint64_t)g.c, (cuuint64_t)g.w, (cuuint64_t)g.h, (cuuint64_t)g.d, (cuuint64_t)g.n};
+    cuuint64_t strides[4] = {(cuuint64_t)g.c * 2, (cuuint64_t)g.w * g.c * 2, (cuuint64_t)g.h * g.w * g.c * 2,
+                             (cuuint64_t)g.d * g.h * g.w * g.c * 2};
+    int lower[3] = {-g.pw, -g.ph, -g.pd};
+    int upper[3] = {g.pw - g.dw * (g.kw - 1), g.ph - g.dh * (g.kh - 1), g.pd - g.dd * (g.kd - 1)};
+    cuuint32_t es[5] = {1, (cuuint32_t)g.sw, (cuuint32_t)g.sh, (cuuint32_t)g.sd, 1};
+    CUresult r = g_encode_im2col(&tA, tmap_dtype(dt), 5, const_cast<void*>(in), dims, strides, lower, upper, BK, BM,
+                                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  const int taps = g.kd * g.kh * g.kw;
+  if (!encode_3d(&tB, dt, w, g.c, taps, g.o, (uint64_t)g.c * 2, (uint64_t)taps * g.c * 2, BK, 1, tile_n))
+    return cudaErrorInvalidValue;
+  TcArgs a{};
+  a.m_tiles = (int)((M + BM - 1) / BM);
+  a.n_tiles = (g.o + tile_n - 1) / tile_n;
+  a.batches = 1;
+  a.kb_per_tap = (g.c + BK - 1) / BK;
+  a.taps = taps;
+  a.kw = g.kw; a.dh = g.dh; a.dw = g.dw;
+  a.oh = g.oh; a.ow = g.ow; a.sh = g.sh; a.sw = g.sw; a.ph = g.ph; a.pw = g.pw;
+  a.kh = g.kh; a.od = g.od; a.sd = g.sd; a.pd = g.pd; a.dd = g.dd;
+  a.m_rows = M;
+  a.ocols = g.o;
+  a.out = out;
+  a.ldo = g.o;
+  a.out_batch = 0;
+  a.accumulate = 0;
+  a.err = err_word;
+  if (dt == CONV_BF16)
+    return tile_n == 256 ? launch_kernel<256, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
+  return tile_n == 256 ? launch_kernel<256, 2, __half, __half>(tA, tB, a, sm_count, s)
+                       : launch_kernel<128, 2, __half, __half>(tA, tB, a, sm_count, s);
 }
 
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n, int sm_count,
@@ -629,10 +718,10 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   a.out_batch = (long long)bg.t * bg.o;
   a.err = err_word;
   if (dt == CONV_BF16)
-    return tile_n == 256 ? launch_kernel<256, false, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, false, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
-  return tile_n == 256 ? launch_kernel<256, false, __half, float>(tA, tB, a, sm_count, s)
-                       : launch_kernel<128, false, __half, float>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
+  return tile_n == 256 ? launch_kernel<256, 0, __half, float>(tA, tB, a, sm_count, s)
+                       : launch_kernel<128, 0, __half, float>(tA, tB, a, sm_count, s);
 }
 
 }  // namespace b200conv

@@ -138,32 +138,52 @@ wino_gemm_f32_kernel(const WgArgs p) {
     cp_commit();
     const float* as = As + (kt % STAGES) * BK * BM;
     const float* bs = Bs + (kt % STAGES) * BK * BN;
+    if constexpr (A_TMAJOR) {
+      // one 128-bit load per A row covers 4 k-steps (rows are contiguous in k)
 #pragma unroll
-    for (int k = 0; k < BK; ++k) {
-      float av[8], bv[TN];
-      if (A_TMAJOR) {
-        // rows tr*4 + i and 64 + tr*4 + i share the swizzle tr % 4
-        const int off = (((k >> 2) ^ (tr & 3)) << 2) + (k & 3);
+      for (int k4 = 0; k4 < BK / 4; ++k4) {
+        float4 a4[8];
+        const int off = (k4 ^ (tr & 3)) << 2;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          av[i] = as[(tr * 4 + i) * BK + off];
-          av[4 + i] = as[(64 + tr * 4 + i) * BK + off];
+          a4[i] = *reinterpret_cast<const float4*>(as + (tr * 4 + i) * BK + off);
+          a4[4 + i] = *reinterpret_cast<const float4*>(as + (64 + tr * 4 + i) * BK + off);
         }
-      } else {
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int k = 4 * k4 + kq;
+          float bv[TN];
+#pragma unroll
+          for (int j = 0; j < TN / 4; ++j) {
+            const float4 b = *reinterpret_cast<const float4*>(bs + k * BN + 32 * j + tc * 4);
+            bv[4 * j] = b.x; bv[4 * j + 1] = b.y; bv[4 * j + 2] = b.z; bv[4 * j + 3] = b.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float av = kq == 0 ? a4[i].x : kq == 1 ? a4[i].y : kq == 2 ? a4[i].z : a4[i].w;
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av, bv[j], acc[i][j]);
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < BK; ++k) {
+        float av[8], bv[TN];
         const float4 a0 = *reinterpret_cast<const float4*>(as + k * BM + tr * 4);
         const float4 a1 = *reinterpret_cast<const float4*>(as + k * BM + 64 + tr * 4);
         av[0] = a0.x; av[1] = a0.y; av[2] = a0.z; av[3] = a0.w;
         av[4] = a1.x; av[5] = a1.y; av[6] = a1.z; av[7] = a1.w;
+#pragma unroll
+        for (int j = 0; j < TN / 4; ++j) {
+          const float4 b = *reinterpret_cast<const float4*>(bs + k * BN + 32 * j + tc * 4);
+          bv[4 * j] = b.x; bv[4 * j + 1] = b.y; bv[4 * j + 2] = b.z; bv[4 * j + 3] = b.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
       }
-#pragma unroll
-      for (int j = 0; j < TN / 4; ++j) {
-        const float4 b = *reinterpret_cast<const float4*>(bs + k * BN + 32 * j + tc * 4);
-        bv[4 * j] = b.x; bv[4 * j + 1] = b.y; bv[4 * j + 2] = b.z; bv[4 * j + 3] = b.w;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
   cp_wait<0>();

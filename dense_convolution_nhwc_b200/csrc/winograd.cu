@@ -97,8 +97,13 @@ template <int M, typename Tin, typename Tst>
 __global__ void __launch_bounds__(256)
 wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restrict__ v) {
   constexpr int A = Wino<M>::A;
-  const int c = blockIdx.y * blockDim.x + threadIdx.x;
-  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  // channel group fastest across blocks, so one tile's V rows are written by
+  // blocks that run together
+  const int cgroups = (a.c + blockDim.x - 1) / blockDim.x;
+  const int cg = (int)(blockIdx.x % cgroups);
+  const long long tg = blockIdx.x / cgroups;
+  const int c = cg * blockDim.x + threadIdx.x;
+  const long long t = tg * blockDim.y + threadIdx.y;
   if (c >= a.c || t >= a.t_count) return;
   const int per_img = a.tiles_h * a.tiles_w;
   const int nl = (int)(t / per_img);
@@ -399,8 +404,9 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   if (a.t_count == 0) return cudaSuccess;
   int bx = g.c >= 64 ? 64 : 32;
   dim3 block(bx, 256 / bx);
-  dim3 grid((unsigned)((a.t_count + block.y - 1) / block.y), (g.c + bx - 1) / bx);
-  if (grid.y > 65535) return cudaErrorInvalidValue;
+  const long long blocks = ((a.t_count + block.y - 1) / block.y) * ((g.c + bx - 1) / bx);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)blocks);
   return by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return by_dt(in_dt, [&](auto ti) {

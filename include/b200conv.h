@@ -163,13 +163,24 @@ B200CONV_API conv_status_t conv2d_forward(const void *in, const void *w, void *o
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * conv3d as depth taps ("Decompose small kernel-depth 3D convs into 2D
- * convs", Change): for each kd, a 2D conv over the zero-copy view of the input
- * frames at depth offset kd*dd (frame stride sd*H*W*C) with the weight slice
- * w[:, kd] (row stride KD*KH*KW*C); tap 0 writes out, taps 1..KD-1 are added
- * in ascending order.  Depth padding, depth stride/dilation, N > 1 and any KD
- * are handled by restricting each tap to the output frames whose input frame
- * exists.  in [N,D,H,W,C], w [O,KD,KH,KW,C], out [N,OD,OH,OW,O].
+ * conv3d, in[N,D,H,W,C], w[O,KD,KH,KW,C], out[N,OD,OH,OW,O].  Two algorithms:
+ *  - depth taps ("Decompose small kernel-depth 3D convs into 2D convs",
+ *    Change): for each kd, a 2D conv over the zero-copy view of the input
+ *    frames at depth offset kd*dd (frame stride sd*H*W*C) with the weight slice
+ *    w[:, kd] (row stride KD*KH*KW*C); tap 0 writes out and taps 1..KD-1 add in
+ *    ascending order inside their own output stage (round the tap, add in
+ *    fp32, round).  Depth padding, depth stride/dilation, N > 1 and any KD are
+ *    handled by restricting each tap to the output frames whose input frame
+ *    exists.
+ *  - a native 3D implicit GEMM (16-bit, tensor cores): K = KD*KH*KW*C in one
+ *    main loop, A tiles gathered by a 5D TMA im2col map; output written once.
+ * With CONV_ALGO_AUTO the page's guard (N == 1, KD <= 7, depth stride 1,
+ * kernel dilation 1, no depth padding, C and O multiples of 16) selects the
+ * depth taps and the other shapes take the native GEMM when it can express them
+ * (16-bit, C % 8 == 0, 5D box corners within [-16, 15]), else the depth taps.
+ * CONV_ALGO_IMPLICIT_GEMM asks for the native GEMM whenever it can run;
+ * CONV_ALGO_WINOGRAD / CONV_ALGO_DIRECT pick the depth taps' 2D algorithm.
+ * plan->taps is KD for depth taps and 1 for the native GEMM.
  */
 B200CONV_API conv_status_t conv3d_plan(const conv3d_desc_t *desc, conv_dtype_t dtype, int device,
                           const conv_options_t *opts, conv_plan_t *plan);

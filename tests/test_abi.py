@@ -187,3 +187,32 @@ def test_conv3d_invalid():
     desc = B.make_desc3d(1, 2, 8, 8, 4, 4, 3, 3, 3, 1, (0, 1, 1), 1)     # OD <= 0
     p = B.ConvPlan()
     assert B.conv3d_plan_for_props(desc, 0, B200, None, p) == 1
+
+
+def plan3d(s, dtype="bf16", **opt):
+    desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+    p = B.ConvPlan()
+    st = B.conv3d_plan_for_props(desc, B.DTYPE[dtype], B200, B.make_options(**opt) if opt else B.make_options(), p)
+    return st, p.as_dict()
+
+
+def test_conv3d_guard_selects_depth_taps_or_native_gemm():
+    """The depth-tap page's guard keeps the taps; what it sends elsewhere goes to
+    the native K-fused 3D GEMM (16-bit) when a 5D im2col map can express it."""
+    guarded = synth.Conv3dShape(1, 9, 16, 16, 64, 64, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    st, p = plan3d(guarded)
+    assert st == 0 and p["taps"] == 3
+    for other in [synth.Conv3dShape(2, 9, 16, 16, 64, 64, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),   # N > 1
+                  synth.Conv3dShape(1, 9, 16, 16, 64, 64, 3, 3, 3, (2, 1, 1), (0, 1, 1), (1, 1, 1)),   # depth stride
+                  synth.Conv3dShape(1, 9, 16, 16, 64, 64, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1)),   # depth pad
+                  synth.Conv3dShape(1, 12, 8, 8, 64, 64, 9, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))]:  # KD > 7
+        st, p = plan3d(other)
+        assert st == 0 and p["taps"] == 1 and p["engine"] == "tcgen05" and p["workspace_bytes"] == 0, other
+        st, p = plan3d(other, "f32")                 # fp32: always depth taps (FFMA)
+        assert st == 0 and p["taps"] == other.kd
+    # a depth pad beyond the 5D box-corner range stays on depth taps
+    st, p = plan3d(synth.Conv3dShape(1, 40, 8, 8, 64, 64, 3, 3, 3, (1, 1, 1), (17, 1, 1), (1, 1, 1)))
+    assert st == 0 and p["taps"] == 3
+    # forcing the implicit GEMM takes the native kernel even inside the guard
+    st, p = plan3d(guarded, algo="implicit")
+    assert st == 0 and p["taps"] == 1

@@ -1,5 +1,5 @@
 """conv3d as depth-tap 2D convs ("Decompose small kernel-depth 3D convs into 2D
-convs", Change, Tests).
+convs", Change, Tests) and as the native K-fused 3D implicit GEMM.
 
 * the fast path against the oracle over shapes with Cout != Cin,
   KD in {1, 2, 3, 5} and a 1x1-spatial case;
@@ -9,7 +9,9 @@ convs", Change, Tests).
 * the depth-tap result equals a manual loop of conv2d_forward over frame views
   plus conv_accumulate, bit for bit (the page's "numerically identical to"
   per-frame 2D);
-* the workload's three shapes on sampled pixels.
+* the workload's three shapes on sampled pixels;
+* the native tcgen05 3D GEMM (5D TMA im2col) against the oracle, and against
+  the depth taps.
 """
 import numpy as np
 import pytest
@@ -116,3 +118,22 @@ def test_accumulate_rounds_once_per_add():
         assert st == 0
         torch.cuda.synchronize()
         assert torch.equal(a, want), dt
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("s", FAST[1:4] + FALLBACK_CASES[:2], ids=lambda s: s.name())
+def test_native_3d_gemm_against_oracle(s, dtype):
+    """The K-fused tcgen05 3D implicit GEMM (forced) against the oracle."""
+    desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+    assert B.plan3d(desc, dtype, 0, B.make_options("implicit"))["taps"] == 1
+    check3d(s, dtype, options=B.make_options("implicit"))
+
+
+def test_native_and_taps_agree():
+    s = synth.Conv3dShape(2, 7, 12, 10, 64, 96, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1))
+    x, w = synth.conv3d_inputs(s, "bf16", "normal", 7, device="cuda")
+    a = run3d(x, w, s, B.make_options("implicit"))
+    b = run3d(x, w, s, B.make_options("direct"))
+    ref = oracle.conv3d(x.cpu(), w.cpu(), "bf16", s.stride, s.pad, s.dilation)
+    assert_close(as_f64(a), ref, "bf16", "native")
+    assert_close(as_f64(b), ref, "bf16", "taps")
