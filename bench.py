@@ -396,6 +396,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--per-conv", action="store_true", help="also print one line per conv of the workload")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step as a CUDA graph and time its replays (removes host launch gaps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -452,6 +454,22 @@ def main():
     torch.cuda.synchronize()
     assert B.conv_check(sptr) == 0
 
+    run_step = step
+    graph = None
+    if args.graph:
+        g_stream = torch.cuda.Stream(dev)
+        g_stream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(g_stream):
+            sptr_saved = sptr
+            sptr = g_stream.cuda_stream
+            with torch.cuda.graph(graph, stream=g_stream):
+                step()
+            sptr = sptr_saved
+        stream.wait_stream(g_stream)
+        torch.cuda.synchronize()
+        run_step = graph.replay
+
     # timed region (device time of the steps; an L2 flush between steps is outside the events)
     total_flops = sum(cv.flops for cv, *_ in items)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -463,8 +481,15 @@ def main():
             if flush is not None:
                 flush.zero_()
             ev[k][0].record(stream)
-            step()
+            run_step()
             ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        prof = B.profile_end()
+    if graph is not None:
+        # graph replays record no per-kernel events: take the kernel breakdown from plain steps
+        B.conv_profile_begin()
+        for k in range(args.steps):
+            step()
         torch.cuda.synchronize()
         prof = B.profile_end()
     barrier(world)
@@ -610,7 +635,8 @@ def main():
                        "convs_per_step": len(items), "flops_per_step": total_flops,
                        "l2": "L2 flushed between steps (outside the events)" if flush_needed
                        else f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "cuda_graph": bool(args.graph)},
             "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": gpu_launches * 1,
             "gpu_launches_per_step": gpu_launches / args.steps,
             "e2e": e2e, "cpu_baseline": cpu,

@@ -8,16 +8,16 @@ fallback.
 """
 _BINDING_NAMES = frozenset({
     # C-ABI entry points (same names as include/b200conv.h)
-    "conv2d_forward", "conv3d_forward", "conv2d_forward_winograd_static", "conv2d_plan", "conv3d_plan",
+    "conv2d_forward", "conv3d_forward", "conv1d_forward", "conv1d_plan", "conv1d_workspace_size", "conv2d_forward_winograd_static", "conv2d_plan", "conv3d_plan",
     "conv2d_plan_for_props", "conv3d_plan_for_props",
     "conv2d_workspace_size", "conv3d_workspace_size", "conv_check", "conv_selftest_timeout",
     "conv_status_string", "conv_device_props", "conv_accumulate", "conv_profile_begin", "conv_profile_end",
     "profile_end", "KernelTime",
     # types and helpers
-    "ConvError", "Conv2dDesc", "Conv3dDesc", "ConvPlan", "ConvOptions", "DeviceProps",
+    "ConvError", "Conv1dDesc", "Conv2dDesc", "Conv3dDesc", "ConvPlan", "ConvOptions", "DeviceProps",
     "ALGO", "DTYPE", "STATUS", "ENGINE", "library_path", "make_desc2d", "make_desc3d", "make_options",
     # torch conveniences
-    "conv2d", "conv3d", "plan2d", "plan3d",
+    "conv1d", "conv2d", "conv3d", "plan2d", "plan3d",
 })
 
 

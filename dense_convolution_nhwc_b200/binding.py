@@ -45,6 +45,11 @@ class Conv3dDesc(ctypes.Structure):
                 ("dilation", ctypes.c_int * 3)]
 
 
+class Conv1dDesc(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int), ("l", ctypes.c_int), ("c", ctypes.c_int), ("o", ctypes.c_int),
+                ("k", ctypes.c_int), ("stride", ctypes.c_int), ("pad", ctypes.c_int), ("dilation", ctypes.c_int)]
+
+
 class DeviceProps(ctypes.Structure):
     _fields_ = [("sm_count", ctypes.c_int), ("cc_major", ctypes.c_int), ("cc_minor", ctypes.c_int),
                 ("total_global_mem", ctypes.c_ulonglong)]
@@ -97,6 +102,12 @@ _conv3d_plan_for_props = _sig("conv3d_plan_for_props", _I, ctypes.POINTER(Conv3d
 _conv3d_workspace_size = _sig("conv3d_workspace_size", ctypes.c_size_t, ctypes.POINTER(Conv3dDesc), _I, _I,
                               ctypes.POINTER(ConvOptions))
 _conv3d_forward = _sig("conv3d_forward", _I, _P, _P, _P, ctypes.POINTER(Conv3dDesc), _I,
+                       ctypes.POINTER(ConvOptions), _P, ctypes.c_size_t, _P)
+_conv1d_plan = _sig("conv1d_plan", _I, ctypes.POINTER(Conv1dDesc), _I, _I, ctypes.POINTER(ConvOptions),
+                    ctypes.POINTER(ConvPlan))
+_conv1d_workspace_size = _sig("conv1d_workspace_size", ctypes.c_size_t, ctypes.POINTER(Conv1dDesc), _I, _I,
+                              ctypes.POINTER(ConvOptions))
+_conv1d_forward = _sig("conv1d_forward", _I, _P, _P, _P, ctypes.POINTER(Conv1dDesc), _I,
                        ctypes.POINTER(ConvOptions), _P, ctypes.c_size_t, _P)
 _conv_accumulate = _sig("conv_accumulate", _I, _P, _P, ctypes.c_size_t, _I, _P)
 _conv2d_forward_winograd_static = _sig("conv2d_forward_winograd_static", _I, _P, _P, _P,
@@ -152,6 +163,20 @@ def conv2d_workspace_size(desc: Conv2dDesc, dtype: int, device: int, opts: Optio
 def conv2d_forward(inp: int, w: int, out: int, desc: Conv2dDesc, dtype: int, opts: Optional[ConvOptions],
                    workspace: int, workspace_bytes: int, stream: int) -> int:
     return _conv2d_forward(inp, w, out, ctypes.byref(desc), dtype, _opt(opts), workspace or None,
+                           workspace_bytes, stream or None)
+
+
+def conv1d_plan(desc: Conv1dDesc, dtype: int, device: int, opts: Optional[ConvOptions], plan: ConvPlan) -> int:
+    return _conv1d_plan(ctypes.byref(desc), dtype, device, _opt(opts), ctypes.byref(plan))
+
+
+def conv1d_workspace_size(desc: Conv1dDesc, dtype: int, device: int, opts: Optional[ConvOptions]) -> int:
+    return int(_conv1d_workspace_size(ctypes.byref(desc), dtype, device, _opt(opts)))
+
+
+def conv1d_forward(inp: int, w: int, out: int, desc: Conv1dDesc, dtype: int, opts: Optional[ConvOptions],
+                   workspace: int, workspace_bytes: int, stream: int) -> int:
+    return _conv1d_forward(inp, w, out, ctypes.byref(desc), dtype, _opt(opts), workspace or None,
                            workspace_bytes, stream or None)
 
 
@@ -316,6 +341,41 @@ def conv2d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
         st = conv2d_forward(x.data_ptr(), w.data_ptr(), out.data_ptr(), desc, dt, options, ws_ptr, ws_n, stream)
         if st != 0:
             raise ConvError(st, "conv2d_forward")
+    return out
+
+
+def conv1d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions] = None, out=None,
+           workspace=None):
+    """NLC conv1d: x [N,L,C], w [O,K,C] -> [N,OL,O] on x's device (through conv1d_forward)."""
+    torch = _torch()
+    _check(x, "x")
+    _check(w, "w")
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must share a dtype")
+    N, L, C = x.shape
+    O, K, C2 = w.shape
+    if C2 != C:
+        raise ValueError("channel mismatch")
+    desc = Conv1dDesc(N, L, C, O, K, stride, padding, dilation)
+    dt = _dtype_code(x.dtype)
+    dev = x.device.index if x.device.index is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        plan = ConvPlan()
+        st = conv1d_plan(desc, dt, dev, options, plan)
+        if st != 0:
+            raise ConvError(st, "conv1d_plan")
+        OL = (L + 2 * padding - dilation * (K - 1) - 1) // stride + 1
+        if out is None:
+            out = torch.empty((N, OL, O), dtype=x.dtype, device=x.device)
+        ws_bytes = int(plan.workspace_bytes)
+        if workspace is None and ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        ws_ptr = workspace.data_ptr() if workspace is not None else 0
+        ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        stream = torch.cuda.current_stream(x.device).cuda_stream
+        st = conv1d_forward(x.data_ptr(), w.data_ptr(), out.data_ptr(), desc, dt, options, ws_ptr, ws_n, stream)
+        if st != 0:
+            raise ConvError(st, "conv1d_forward")
     return out
 
 

@@ -615,6 +615,36 @@ conv_status_t conv2d_forward(const void* in, const void* w, void* out, const con
   return run2d(in, w, out, g, dtype, s, workspace, *d, static_cast<cudaStream_t>(stream));
 }
 
+static bool desc2d_of(const conv1d_desc_t* d, conv2d_desc_t* d2) {
+  if (!d) return false;
+  *d2 = conv2d_desc_t{};
+  d2->n = d->n; d2->h = 1; d2->w = d->l; d2->c = d->c; d2->o = d->o; d2->kh = 1; d2->kw = d->k;
+  d2->stride[0] = 1; d2->stride[1] = d->stride;
+  d2->pad[0] = 0; d2->pad[1] = d->pad;
+  d2->dilation[0] = 1; d2->dilation[1] = d->dilation;
+  return true;
+}
+
+conv_status_t conv1d_plan(const conv1d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts,
+                          conv_plan_t* plan) {
+  conv2d_desc_t d2;
+  if (!desc2d_of(desc, &d2)) return CONV_ERR_INVALID;
+  return conv2d_plan(&d2, dtype, device, opts, plan);
+}
+
+size_t conv1d_workspace_size(const conv1d_desc_t* desc, conv_dtype_t dtype, int device, const conv_options_t* opts) {
+  conv2d_desc_t d2;
+  if (!desc2d_of(desc, &d2)) return 0;
+  return conv2d_workspace_size(&d2, dtype, device, opts);
+}
+
+conv_status_t conv1d_forward(const void* in, const void* w, void* out, const conv1d_desc_t* desc, conv_dtype_t dtype,
+                             const conv_options_t* opts, void* workspace, size_t workspace_bytes, void* stream) {
+  conv2d_desc_t d2;
+  if (!desc2d_of(desc, &d2)) return CONV_ERR_INVALID;
+  return conv2d_forward(in, w, out, &d2, dtype, opts, workspace, workspace_bytes, stream);
+}
+
 conv_status_t conv3d_plan_for_props(const conv3d_desc_t* desc, conv_dtype_t dtype, const conv_device_props_t* props,
                                     const conv_options_t* opts, conv_plan_t* plan) {
   if (!props || !plan) return CONV_ERR_INVALID;

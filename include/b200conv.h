@@ -97,6 +97,12 @@ typedef struct {
     int stride[3], pad[3], dilation[3];
 } conv3d_desc_t;
 
+/* 1D problem: in [N, L, C] (channels last), w [O, K, C], out [N, OL, O]. */
+typedef struct {
+    int n, l, c, o, k;
+    int stride, pad, dilation;
+} conv1d_desc_t;
+
 /* Constant device properties the selector may depend on. */
 typedef struct {
     int sm_count;
@@ -161,6 +167,23 @@ B200CONV_API conv_status_t conv2d_forward(const void *in, const void *w, void *o
                              const conv2d_desc_t *desc, conv_dtype_t dtype,
                              const conv_options_t *opts,
                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * conv1d through the 2D path, as the implicit-GEMM page's conv_1D_gpu routes
+ * 1D convolutions into the 2D dispatch ("Use the explicit gemm for wide convs
+ * on neural accelerators", the Whisper follow-up): a [N, L, C] input is the
+ * [N, 1, L, C] image of a 1 x K conv2d with stride (1, s), padding (0, p) and
+ * dilation (1, d).  Same selector, kernels, ownership and error behaviour as
+ * conv2d_*.
+ */
+B200CONV_API conv_status_t conv1d_plan(const conv1d_desc_t *desc, conv_dtype_t dtype, int device,
+                                       const conv_options_t *opts, conv_plan_t *plan);
+B200CONV_API size_t conv1d_workspace_size(const conv1d_desc_t *desc, conv_dtype_t dtype, int device,
+                                          const conv_options_t *opts);
+B200CONV_API conv_status_t conv1d_forward(const void *in, const void *w, void *out,
+                                          const conv1d_desc_t *desc, conv_dtype_t dtype,
+                                          const conv_options_t *opts,
+                                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * conv3d, in[N,D,H,W,C], w[O,KD,KH,KW,C], out[N,OD,OH,OW,O].  Two algorithms:

@@ -120,3 +120,25 @@ def test_wide_sweep_subset(dtype):
 def test_wide_sweep_unaligned(dtype):
     for shape in synth.wide_sweep(False)[::3]:
         check_conv2d(shape, dtype, sample=512)
+
+
+CONV1D = [
+    # Whisper-encoder-style pair (the implicit-GEMM page's conv1d follow-up): 80 -> 384, then stride 2
+    (1, 3000, 80, 384, 3, 1, 1, 1),
+    (1, 3000, 384, 384, 3, 2, 1, 1),
+    (3, 97, 13, 21, 5, 2, 2, 2),      # ragged, unaligned channels, dilation
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("case", CONV1D, ids=str)
+def test_conv1d_through_the_2d_path(case, dtype):
+    import numpy as np
+    import oracle
+    from tests.gpu_util import as_f64, assert_close
+    n, l, c, o, k, s, p, d = case
+    x, w = synth.make_inputs((n, l, c), (o, k, c), dtype, "normal", 11, device="cuda")
+    out = B.conv1d(x, w, s, p, d)
+    torch.cuda.synchronize()
+    ref = oracle.conv2d(x.cpu().reshape(n, 1, l, c), w.cpu().reshape(o, 1, k, c), dtype, (1, s), (0, p), (1, d))
+    assert_close(as_f64(out), ref.reshape(out.shape), dtype, f"conv1d {case}")
