@@ -298,7 +298,8 @@ def barrier(world):
 # CPU oracle baseline
 # ---------------------------------------------------------------------------
 
-METRIC = "conv TFLOP/s (direct-equivalent FLOPs) and fraction of the dominant kernel's peak"
+# the headline metric, verbatim; TFLOP/s are direct-equivalent (2*N*OH*OW*O*C*KH*KW per second)
+METRIC = "conv TFLOP/s per dtype and fraction of tensor (or FP32) peak, 1 B200"
 
 
 def oracle_sample_rate(conv, x_host, w_host, target_s, seed=0):

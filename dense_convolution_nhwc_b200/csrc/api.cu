@@ -169,6 +169,7 @@ struct Sel {
   conv_engine_t engine = CONV_ENGINE_SIMT;
   int tile_m = 128, tile_n = 128;
   int wino_m = 0, nb = 0, ntiles = 0, cpad = 0;
+  bool wpack = false;      // KW taps folded into cpad channels (a few-channel input)
   conv_dtype_t wino_store = CONV_F32;
   size_t ws = 0;
 };
@@ -302,7 +303,14 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     s->engine = CONV_ENGINE_TCGEN05;
     s->tile_m = 128;
     s->tile_n = tc_tile_n(g, p);
-    if (g.c % 8 != 0) {
+    s->wpack = false;
+    if (g.c % 8 != 0 && g.kw > 1 && g.kw * g.c <= 64) {
+      // a few channels: fold the KW taps into channels (KH x 1 conv over KW*C)
+      const int cp = (g.kw * g.c + 7) / 8 * 8;
+      s->cpad = cp;
+      s->wpack = true;
+      s->ws = align256((size_t)g.n * g.h * g.ow * cp * esz) + align256((size_t)g.o * g.kh * cp * esz);
+    } else if (g.c % 8 != 0) {
       const int cp = (g.c + 7) / 8 * 8;
       s->cpad = cp;
       s->ws = align256((size_t)g.n * g.h * g.w * cp * esz) + align256((size_t)g.o * g.kh * g.kw * cp * esz);
@@ -324,6 +332,7 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->batch_tile = s.nb;
   plan->num_batch_tiles = s.ntiles;
   plan->channel_pad = s.cpad;
+  plan->packed_taps = s.wpack ? 1 : 0;
   plan->taps = taps;
   plan->workspace_bytes = ws;
 }
@@ -386,6 +395,35 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     return CONV_OK;
   }
   if (s.engine == CONV_ENGINE_TCGEN05) {
+    if (s.wpack) {
+      uint8_t* base = static_cast<uint8_t*>(ws);
+      const int esz = dtype_size(dt);
+      void* pin = base;
+      void* pw = base + align256((size_t)g.n * g.h * g.ow * s.cpad * esz);
+      cudaError_t e;
+      {
+        ProfScope ps(K_CHANNEL_PAD, st);
+        e = launch_wpack(in, g.n, g.h, g.w, g.c, g.kw, g.sw, g.pw, g.dw, g.ow, g.in_img_stride, pin, s.cpad, dt, st);
+      }
+      if (e == cudaSuccess) {
+        // w[o][kh][kw][c] rows of KW*C channels -> [o][kh][cp]
+        ProfScope ps(K_CHANNEL_PAD, st);
+        e = launch_channel_pad(w, g.o, g.kh, g.kw * g.c, g.w_row_stride, pw, s.cpad, dt, st);
+      }
+      if (e != cudaSuccess) return CONV_ERR_CUDA;
+      Geom gp = g;
+      gp.w = g.ow;
+      gp.c = s.cpad;
+      gp.kw = 1;
+      gp.sw = 1;
+      gp.pw = 0;
+      gp.dw = 1;
+      gp.in_img_stride = (long long)g.h * g.ow * s.cpad;
+      gp.w_row_stride = (long long)g.kh * s.cpad;
+      ProfScope ps(K_TC_CONV, st);
+      return cuda_status(
+          launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
+    }
     if (s.cpad) {
       uint8_t* base = static_cast<uint8_t*>(ws);
       const int esz = dtype_size(dt);

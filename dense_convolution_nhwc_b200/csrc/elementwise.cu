@@ -6,7 +6,10 @@
 //    storage dtype; 16-byte vector accesses when both pointers allow it.
 //  * channel pad: copies NHWC (or OHWI) rows of C channels into rows of Cp
 //    channels with zeros after C, so that rows meet the tensor-memory-access
-//    16-byte stride rule (e.g. a 3-channel stem).
+//    16-byte stride rule.
+//  * tap packing: for a few channels (a 3-channel stem), folds the KW taps of
+//    each output column into channels so the tensor cores see a KH x 1 conv
+//    over KW*C packed channels instead of KH*KW mostly-empty 64-channel steps.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -78,7 +81,73 @@ __global__ void channel_pad_kernel(const T* __restrict__ src, long long outer, l
   }
 }
 
+// Tap packing for small C: P[n][h][ow][kw*C + c] = in[n][h][ow*sw - pw + kw*dw][c]
+// (zero outside the row and for channels >= KW*C), so the conv becomes KH x 1
+// over Cp = KW*C rounded up packed channels.
+template <typename T>
+__global__ void wpack_kernel(const T* __restrict__ src, long long pixels /* n*h*ow */, int w, int c, int kw, int sw,
+                             int pw, int dw, int ow, long long in_row_stride, long long in_img_stride, int h,
+                             T* __restrict__ dst, int cp) {
+  // one thread per output pixel (n, y, x); its cp packed channels are written in
+  // 8-element vectors (cp is a multiple of 8, rows 16-byte aligned)
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (; i < pixels; i += stride) {
+    const int x = (int)(i % ow);
+    const long long nh = i / ow;
+    const long long n = nh / h, y = nh - n * h;
+    const T* row = src + n * in_img_stride + y * in_row_stride;
+    const int x0 = x * sw - pw;
+    T* out = dst + i * cp;
+    for (int ch0 = 0; ch0 < cp; ch0 += 8) {
+      __align__(16) T v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int ch = ch0 + e;
+        float f = 0.0f;
+        if (ch < kw * c) {
+          const int k = ch / c, cc = ch - k * c;
+          const int ix = x0 + k * dw;
+          if (ix >= 0 && ix < w) f = Store<T>::to_f32(row[(long long)ix * c + cc]);
+        }
+        v[e] = Store<T>::from_f32(f);
+      }
+      if constexpr (sizeof(T) == 2) {
+        *reinterpret_cast<uint4*>(out + ch0) = *reinterpret_cast<const uint4*>(v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[ch0 + e] = v[e];
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,
+                         long long in_img_stride, void* dst, int cp, conv_dtype_t dt, cudaStream_t s) {
+  if (cp % 8 != 0) return cudaErrorInvalidValue;
+  const long long total = n * h * (long long)ow;     // output pixels
+  if (total == 0) return cudaSuccess;
+  unsigned blocks = (unsigned)((total + 255) / 256 < 148 * 32 ? (total + 255) / 256 : 148 * 32);
+  const long long rs = (long long)w * c;
+  switch (dt) {
+    case CONV_F32:
+      wpack_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(src), total, w, c, kw, sw, pw, dw, ow, rs,
+                                                 in_img_stride, h, static_cast<float*>(dst), cp);
+      break;
+    case CONV_F16:
+      wpack_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(src), total, w, c, kw, sw, pw, dw, ow, rs,
+                                                  in_img_stride, h, static_cast<__half*>(dst), cp);
+      break;
+    case CONV_BF16:
+      wpack_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), total, w, c, kw, sw,
+                                                         pw, dw, ow, rs, in_img_stride, h,
+                                                         static_cast<__nv_bfloat16*>(dst), cp);
+      break;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dt,
                               cudaStream_t s) {

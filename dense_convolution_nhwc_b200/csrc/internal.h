@@ -103,6 +103,10 @@ cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb,
 cudaError_t launch_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dt,
                               cudaStream_t s);
 cudaError_t launch_fill_zero(void* out, size_t bytes, cudaStream_t s);
+// Tap packing: dst[n][y][x][k*c + ch] = src[n][y][x*sw - pw + k*dw][ch] (zero outside the row and
+// for channels >= kw*c); dst is dense [n][h][ow][cp].
+cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,
+                         long long in_img_stride, void* dst, int cp, conv_dtype_t dt, cudaStream_t s);
 // Channel pad: dst[a][b][c'] = c' < c ? src[a*src_outer_stride + b*c + c'] : 0 for a < outer,
 // b < inner, c' < cp; dst is dense [outer][inner][cp].  Element strides.
 cudaError_t launch_channel_pad(const void* src, long long outer, long long inner, int c,

@@ -132,6 +132,7 @@ typedef struct {
     int batch_tile;            /* images per Winograd batch tile (= n when untiled) */
     int num_batch_tiles;       /* number of batch tiles */
     int channel_pad;           /* padded channel count of the pre-pass, 0 if none */
+    int packed_taps;           /* 1 if the KW taps are folded into channel_pad channels (few-channel inputs) */
     int taps;                  /* conv3d: number of depth taps (KD); 1 for conv2d */
     size_t workspace_bytes;    /* bytes the caller must pass to *_forward */
 } conv_plan_t;

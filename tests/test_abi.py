@@ -116,8 +116,8 @@ def test_sixteen_bit_takes_tensor_cores():
         for dt in ("f16", "bf16"):
             st, p = plan2d(shape, dt)
             assert st == 0 and p["algo"] == "implicit" and p["engine"] == "tcgen05", name
-            if shape.c == 3:
-                assert p["channel_pad"] == 8 and p["workspace_bytes"] > 0
+            if shape.c == 3:      # the stem: 7 taps x 3 channels folded into 24 channels
+                assert p["channel_pad"] == 24 and p["packed_taps"] == 1 and p["workspace_bytes"] > 0
             else:
                 assert p["channel_pad"] == 0 and p["workspace_bytes"] == 0
 
