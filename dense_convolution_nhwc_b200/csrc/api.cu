@@ -76,9 +76,9 @@ long long out_extent(long long in, int k, int s, int p, int d) {
 // ------------------------------ profiling ------------------------------------
 // Opt-in: each kernel launch is bracketed by two events on its stream.
 
-enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
+enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_SPLITK_REDUCE, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
             K_WINO_OUTPUT, K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
-const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "wino_filter", "wino_input", "wino_gemm_tc",
+const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "splitk_reduce", "wino_filter", "wino_input", "wino_gemm_tc",
                                         "wino_gemm_simt", "wino_output", "accumulate", "channel_pad", "fill"};
 
 struct ProfRecord {
@@ -170,6 +170,8 @@ struct Sel {
   int tile_m = 128, tile_n = 128;
   int wino_m = 0, nb = 0, ntiles = 0, cpad = 0;
   bool wpack = false;      // KW taps folded into cpad channels (a few-channel input)
+  int ksplit = 1;          // implicit GEMM: K range split over ksplit CTAs, fp32 partials reduced after
+  size_t split_off = 0;    // workspace offset of the partials
   conv_dtype_t wino_store = CONV_F32;
   size_t ws = 0;
 };
@@ -319,6 +321,36 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     s->engine = CONV_ENGINE_SIMT;
     s->tile_m = 128;
     s->tile_n = g.o <= 64 ? 64 : (g.o <= 96 ? 96 : 128);
+    s->wpack = false;
+    if (s->algo == CONV_ALGO_IMPLICIT_GEMM && g.c <= 8 && g.kw > 1 && g.kw * g.c <= 64) {
+      // a few channels: fold the KW taps into channels for the 16-wide k chunks too
+      const int cp = (g.kw * g.c + 7) / 8 * 8;
+      s->cpad = cp;
+      s->wpack = true;
+      s->ws = align256((size_t)g.n * g.h * g.ow * cp * esz) + align256((size_t)g.o * g.kh * cp * esz);
+    }
+  }
+  // Split-K for grids under half a wave with a long K loop: each split writes
+  // fp32 partials, reduced in a fixed order (deterministic for a given plan).
+  const long long M = (long long)g.n * g.oh * g.ow;
+  if (s->algo == CONV_ALGO_IMPLICIT_GEMM && M > 0) {
+    const int c_eff = s->cpad ? s->cpad : g.c;
+    const long long taps = s->wpack ? g.kh : (long long)g.kh * g.kw;
+    long long ks = 1;
+    if (s->engine == CONV_ENGINE_TCGEN05) {
+      const long long ksteps = taps * ((c_eff + 63) / 64);
+      const long long tiles = ((M + 127) / 128) * ((g.o + s->tile_n - 1) / s->tile_n);
+      if (tiles * 2 <= p.sm_count && ksteps >= 8) ks = std::min({(long long)p.sm_count / tiles, ksteps / 4, 16LL});
+    } else {
+      const long long steps = taps * ((c_eff + 15) / 16);
+      const long long blocks = ((M + 127) / 128) * ((g.o + s->tile_n - 1) / s->tile_n);
+      if (blocks * 2 <= p.sm_count && steps >= 16) ks = std::min({(long long)p.sm_count / blocks, steps / 8, 16LL});
+    }
+    if (ks >= 2) {
+      s->ksplit = (int)ks;
+      s->split_off = s->ws;
+      s->ws += align256((size_t)ks * M * g.o * 4);
+    }
   }
   return CONV_OK;
 }
@@ -333,6 +365,7 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->num_batch_tiles = s.ntiles;
   plan->channel_pad = s.cpad;
   plan->packed_taps = s.wpack ? 1 : 0;
+  plan->k_split = s.ksplit;
   plan->taps = taps;
   plan->workspace_bytes = ws;
 }
@@ -394,71 +427,80 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     }
     return CONV_OK;
   }
-  if (s.engine == CONV_ENGINE_TCGEN05) {
-    if (s.wpack) {
-      uint8_t* base = static_cast<uint8_t*>(ws);
-      const int esz = dtype_size(dt);
-      void* pin = base;
-      void* pw = base + align256((size_t)g.n * g.h * g.ow * s.cpad * esz);
-      cudaError_t e;
-      {
-        ProfScope ps(K_CHANNEL_PAD, st);
-        e = launch_wpack(in, g.n, g.h, g.w, g.c, g.kw, g.sw, g.pw, g.dw, g.ow, g.in_img_stride, pin, s.cpad, dt, st);
-      }
-      if (e == cudaSuccess) {
-        // w[o][kh][kw][c] rows of KW*C channels -> [o][kh][cp]
-        ProfScope ps(K_CHANNEL_PAD, st);
-        e = launch_channel_pad(w, g.o, g.kh, g.kw * g.c, g.w_row_stride, pw, s.cpad, dt, st);
-      }
-      if (e != cudaSuccess) return CONV_ERR_CUDA;
-      Geom gp = g;
-      gp.w = g.ow;
-      gp.c = s.cpad;
-      gp.kw = 1;
-      gp.sw = 1;
-      gp.pw = 0;
-      gp.dw = 1;
-      gp.in_img_stride = (long long)g.h * g.ow * s.cpad;
-      gp.w_row_stride = (long long)g.kh * s.cpad;
-      ProfScope ps(K_TC_CONV, st);
-      return cuda_status(
-          launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
+  // Implicit GEMM / direct: optional pre-pass (tap packing or channel pad),
+  // the GEMM engine, and the split-K reduction.
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int esz = dtype_size(dt);
+  const void* cin = in;
+  const void* cw = w;
+  Geom gg = g;
+  if (s.wpack) {
+    void* pin = base;
+    void* pw = base + align256((size_t)g.n * g.h * g.ow * s.cpad * esz);
+    cudaError_t e;
+    {
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_wpack(in, g.n, g.h, g.w, g.c, g.kw, g.sw, g.pw, g.dw, g.ow, g.in_img_stride, pin, s.cpad, dt, st);
     }
-    if (s.cpad) {
-      uint8_t* base = static_cast<uint8_t*>(ws);
-      const int esz = dtype_size(dt);
-      void* pin = base;
-      void* pw = base + align256((size_t)g.n * g.h * g.w * s.cpad * esz);
-      cudaError_t e;
-      {
-        ProfScope ps(K_CHANNEL_PAD, st);
-        e = launch_channel_pad(in, g.n, (long long)g.h * g.w, g.c, g.in_img_stride, pin, s.cpad, dt, st);
-      }
-      if (e == cudaSuccess) {
-        ProfScope ps(K_CHANNEL_PAD, st);
-        e = launch_channel_pad(w, g.o, (long long)g.kh * g.kw, g.c, g.w_row_stride, pw, s.cpad, dt, st);
-      }
-      if (e != cudaSuccess) return CONV_ERR_CUDA;
-      Geom gp = g;
-      gp.c = s.cpad;
-      gp.in_img_stride = (long long)g.h * g.w * s.cpad;
-      gp.w_row_stride = (long long)g.kh * g.kw * s.cpad;
-      ProfScope ps(K_TC_CONV, st);
-      return cuda_status(
-          launch_tc_conv(pin, pw, out, gp, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
+    if (e == cudaSuccess) {
+      // w[o][kh][kw][c] rows of KW*C channels -> [o][kh][cp]
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_channel_pad(w, g.o, g.kh, g.kw * g.c, g.w_row_stride, pw, s.cpad, dt, st);
     }
-    if (tc_conv_supported(g, dt, in, w)) {
-      ProfScope ps(K_TC_CONV, st);
-      return cuda_status(
-          launch_tc_conv(in, w, out, g, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st));
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    cin = pin;
+    cw = pw;
+    gg.w = g.ow;
+    gg.c = s.cpad;
+    gg.kw = 1;
+    gg.sw = 1;
+    gg.pw = 0;
+    gg.dw = 1;
+    gg.in_img_stride = (long long)g.h * g.ow * s.cpad;
+    gg.w_row_stride = (long long)g.kh * s.cpad;
+  } else if (s.cpad) {
+    void* pin = base;
+    void* pw = base + align256((size_t)g.n * g.h * g.w * s.cpad * esz);
+    cudaError_t e;
+    {
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_channel_pad(in, g.n, (long long)g.h * g.w, g.c, g.in_img_stride, pin, s.cpad, dt, st);
     }
-    // Misaligned pointers: the any-alignment path below.
+    if (e == cudaSuccess) {
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_channel_pad(w, g.o, (long long)g.kh * g.kw, g.c, g.w_row_stride, pw, s.cpad, dt, st);
+    }
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    cin = pin;
+    cw = pw;
+    gg.c = s.cpad;
+    gg.in_img_stride = (long long)g.h * g.w * s.cpad;
+    gg.w_row_stride = (long long)g.kh * g.kw * s.cpad;
   }
-  const bool vec = s.algo != CONV_ALGO_DIRECT && g.c % 4 == 0 &&
-                   (g.in_img_stride % 4 == 0) && (g.w_row_stride % 4 == 0) &&
-                   aligned16(in) && aligned16(w);
-  ProfScope ps(K_SIMT_CONV, st);
-  return cuda_status(launch_simt_conv(in, w, out, g, dt, vec, accumulate, st));
+  float* partial = s.ksplit > 1 ? reinterpret_cast<float*>(base + s.split_off) : nullptr;
+  bool done = false;
+  if (s.engine == CONV_ENGINE_TCGEN05 && tc_conv_supported(gg, dt, cin, cw)) {
+    ProfScope ps(K_TC_CONV, st);
+    if (launch_tc_conv(cin, cw, out, gg, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st, s.ksplit,
+                       partial) != cudaSuccess)
+      return CONV_ERR_CUDA;
+    done = true;
+  }
+  if (!done) {
+    // FFMA engine, or misaligned pointers on the tensor-core plan: the any-alignment path
+    const bool vec = s.algo != CONV_ALGO_DIRECT && gg.c % 4 == 0 && (gg.in_img_stride % 4 == 0) &&
+                     (gg.w_row_stride % 4 == 0) && aligned16(cin) && aligned16(cw);
+    ProfScope ps(K_SIMT_CONV, st);
+    if (launch_simt_conv(cin, cw, out, gg, dt, vec, accumulate, st, s.ksplit, partial) != cudaSuccess)
+      return CONV_ERR_CUDA;
+  }
+  if (s.ksplit > 1) {
+    ProfScope ps(K_SPLITK_REDUCE, st);
+    if (launch_splitk_reduce(partial, s.ksplit, (size_t)g.n * g.oh * g.ow * g.o, out, dt, accumulate, st) !=
+        cudaSuccess)
+      return CONV_ERR_CUDA;
+  }
+  return CONV_OK;
 }
 
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
@@ -643,13 +685,13 @@ conv_status_t conv2d_forward(const void* in, const void* w, void* out, const con
   Sel s;
   st = select2d(g, dtype, d->props, effective_options(opts), &s);
   if (st != CONV_OK) return st;
-  if (workspace_bytes < s.ws || (s.ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
   const int esz = dtype_size(dtype);
   const size_t out_bytes = (size_t)g.n * g.out_img_stride * esz;
   if (overlaps(out, out_bytes, in, (size_t)g.n * g.in_img_stride * esz) ||
-      overlaps(out, out_bytes, w, (size_t)g.o * g.w_row_stride * esz) ||
-      overlaps(out, out_bytes, workspace, s.ws))
+      overlaps(out, out_bytes, w, (size_t)g.o * g.w_row_stride * esz))
     return CONV_ERR_INVALID;
+  if (workspace_bytes < s.ws || (s.ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
+  if (overlaps(out, out_bytes, workspace, s.ws)) return CONV_ERR_INVALID;
   return run2d(in, w, out, g, dtype, s, workspace, *d, static_cast<cudaStream_t>(stream));
 }
 

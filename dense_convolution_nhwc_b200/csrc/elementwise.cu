@@ -122,7 +122,41 @@ __global__ void wpack_kernel(const T* __restrict__ src, long long pixels /* n*h*
   }
 }
 
+template <typename T>
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int ksplit, size_t count, T* __restrict__ out,
+                                     int accumulate) {
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (; i < count; i += stride) {
+    float sum = 0.0f;
+    for (int k = 0; k < ksplit; ++k) sum += __ldg(partial + (size_t)k * count + i);   // fixed order
+    float v = sum;
+    if (accumulate) v = Store<T>::to_f32(out[i]) + Store<T>::to_f32(Store<T>::from_f32(sum));
+    out[i] = Store<T>::from_f32(v);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count, void* out, conv_dtype_t dt,
+                                 bool accumulate, cudaStream_t s) {
+  if (count == 0) return cudaSuccess;
+  unsigned blocks = (unsigned)((count + 255) / 256 < 148 * 16 ? (count + 255) / 256 : 148 * 16);
+  const int acc = accumulate ? 1 : 0;
+  switch (dt) {
+    case CONV_F32:
+      splitk_reduce_kernel<float><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<float*>(out), acc);
+      break;
+    case CONV_F16:
+      splitk_reduce_kernel<__half><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<__half*>(out), acc);
+      break;
+    case CONV_BF16:
+      splitk_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(partial, ksplit, count,
+                                                                 static_cast<__nv_bfloat16*>(out), acc);
+      break;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,
                          long long in_img_stride, void* dst, int cp, conv_dtype_t dt, cudaStream_t s) {

@@ -55,8 +55,15 @@ struct BatchedGemm {
 
 // SIMT implicit GEMM (FFMA, fp32 accumulate): any dtype, any alignment when
 // vec == false.  accumulate: out = round(out + round(result)).
+// ksplit > 1: the K range is split over ksplit blocks that write fp32 partials
+// [ksplit][M][O] to `partial` (then launch_splitk_reduce).
 cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geom& g,
-                             conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s);
+                             conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s, int ksplit = 1,
+                             float* partial = nullptr);
+// out[i] = round(sum_s partial[s][i]) (s ascending), or with accumulate
+// out[i] = round(out[i] + round(sum)), for i < count.
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count, void* out, conv_dtype_t dt,
+                                 bool accumulate, cudaStream_t s);
 // SIMT batched GEMM on fp32 operands (Winograd fp32 path).
 cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s);
 
@@ -64,9 +71,10 @@ cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s);
 // Returns cudaErrorNotSupported if the shape cannot be encoded as TMA maps.
 bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w);
 // accumulate: out = round(out + round(result)), the unfused depth-tap add's arithmetic.
+// ksplit > 1: fp32 partials [ksplit][M][O] to `partial` (then launch_splitk_reduce).
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
                            conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
-                           bool accumulate, cudaStream_t s);
+                           bool accumulate, cudaStream_t s, int ksplit = 1, float* partial = nullptr);
 // Native 3D implicit GEMM on tcgen05: K = KD*KH*KW*C in one main loop, the A
 // tiles gathered by a 5D TMA im2col map (corners limited to [-16, 15]).
 bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w);

@@ -37,6 +37,8 @@ struct SimtArgs {
   long long w_row_stride;    // elements between weight rows
   long long a_batch, b_batch, d_batch;   // batch strides (grid.z), elements
   int accumulate;
+  int ksplit;                // > 1: blockIdx.z splits the K range; fp32 partials go to `partial`
+  float* partial;            // [ksplit][m][o] when ksplit > 1
 };
 
 // Loads 4 consecutive channels starting at p (all < C when full) as fp32.
@@ -73,7 +75,8 @@ simt_conv_kernel(const SimtArgs a) {
   const int tx = tid & 15, ty = tid >> 4;
   const long long m0 = (long long)blockIdx.x * BM;
   const int n0 = blockIdx.y * BN;
-  const int bz = blockIdx.z;
+  const int bz = a.ksplit > 1 ? 0 : blockIdx.z;
+  const int split = a.ksplit > 1 ? blockIdx.z : 0;
 
   const T* __restrict__ in = static_cast<const T*>(a.in) + (long long)bz * a.a_batch;
   const T* __restrict__ wt = static_cast<const T*>(a.w) + (long long)bz * a.b_batch;
@@ -99,12 +102,17 @@ simt_conv_kernel(const SimtArgs a) {
   }
 
   const int cchunks = (a.c + BK - 1) / BK;
-  const int steps = a.kh * a.kw * cchunks;
+  const int steps_all = a.kh * a.kw * cchunks;
+  // K range of this block: all of it, or split `split` of ksplit
+  const int step_lo = (int)((long long)steps_all * split / a.ksplit);
+  const int step_hi = (int)((long long)steps_all * (split + 1) / a.ksplit);
+  const int steps = step_hi - step_lo;
 
   float ra[2][4];
   float rb[B_PER_T][4];
 
-  auto load_tiles = [&](int step) {
+  auto load_tiles = [&](int step_rel) {
+    const int step = step_lo + step_rel;
     const int tap = step / cchunks;
     const int c0 = (step - tap * cchunks) * BK;
     const int ky = tap / a.kw, kx = tap - (tap / a.kw) * a.kw;
@@ -161,7 +169,12 @@ simt_conv_kernel(const SimtArgs a) {
 #pragma unroll
     for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
 
-  load_tiles(0);
+  if (steps > 0) load_tiles(0);
+  else ra[0][0] = ra[0][1] = ra[0][2] = ra[0][3] = ra[1][0] = ra[1][1] = ra[1][2] = ra[1][3] = 0.0f;
+  if (steps <= 0) {
+#pragma unroll
+    for (int r = 0; r < B_PER_T; ++r) rb[r][0] = rb[r][1] = rb[r][2] = rb[r][3] = 0.0f;
+  }
   store_tiles(0);
   __syncthreads();
 
@@ -195,6 +208,15 @@ simt_conv_kernel(const SimtArgs a) {
   for (int i = 0; i < 8; ++i) {
     long long m = m0 + 32 * (i >> 1) + ty * 2 + (i & 1);
     if (m >= a.m) continue;
+    if (a.ksplit > 1) {
+      float* prow = a.partial + (long long)split * a.m * a.o + m * a.o;
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        int o = n0 + 32 * (j >> 1) + tx * 2 + (j & 1);
+        if (o < a.o) prow[o] = acc[i][j];
+      }
+      continue;
+    }
     T* orow = out + m * a.o;
 #pragma unroll
     for (int j = 0; j < TN; ++j) {
@@ -237,7 +259,8 @@ cudaError_t launch_dt(const SimtArgs& a, conv_dtype_t dt, int batches, cudaStrea
 }  // namespace
 
 cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geom& g,
-                             conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s) {
+                             conv_dtype_t dt, bool vec, bool accumulate, cudaStream_t s, int ksplit,
+                             float* partial) {
   if (g.out_img_stride != (long long)g.oh * g.ow * g.o) return cudaErrorInvalidValue;
   SimtArgs a{};
   a.in = in; a.w = w; a.out = out;
@@ -249,8 +272,11 @@ cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geo
   a.w_row_stride = g.w_row_stride;
   a.a_batch = a.b_batch = a.d_batch = 0;
   a.accumulate = accumulate ? 1 : 0;
+  a.ksplit = ksplit > 1 ? ksplit : 1;
+  a.partial = partial;
   if (a.m == 0) return cudaSuccess;
-  return vec ? launch_dt<true>(a, dt, 1, s) : launch_dt<false>(a, dt, 1, s);
+  if (a.ksplit > 1 && !partial) return cudaErrorInvalidValue;
+  return vec ? launch_dt<true>(a, dt, a.ksplit, s) : launch_dt<false>(a, dt, a.ksplit, s);
 }
 
 cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s) {
@@ -267,6 +293,8 @@ cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s) {
   a.b_batch = (long long)bg.o * bg.c;
   a.d_batch = (long long)bg.t * bg.o;
   a.accumulate = 0;
+  a.ksplit = 1;
+  a.partial = nullptr;
   if (a.m == 0 || bg.batches == 0) return cudaSuccess;
   bool vec = (bg.c % 4 == 0) && ((reinterpret_cast<uintptr_t>(bg.a) & 15) == 0) &&
              ((reinterpret_cast<uintptr_t>(bg.b) & 15) == 0);

@@ -67,6 +67,7 @@ struct TcArgs {
   long long ldo;               // elements between output rows
   long long out_batch;         // elements between batches
   int accumulate;              // out = round(out + round(acc)) instead of out = round(acc)
+  int ksplit;                  // conv modes: > 1 splits the K range, the split index in the batch slot
   int* err;
 };
 
@@ -285,7 +286,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           img = (int)fr;
         }
-        for (int ks = 0; ks < ksteps; ++ks) {
+        int ks_lo = 0, ks_hi = ksteps;
+        if (MODE != 0 && a.ksplit > 1) {
+          ks_lo = (int)((long long)ksteps * b / a.ksplit);
+          ks_hi = (int)((long long)ksteps * (b + 1) / a.ksplit);
+        }
+        for (int ks = ks_lo; ks < ks_hi; ++ks) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, a.err, DEVERR_TIMEOUT_PRODUCER)) {
             ok = false;
             break;
@@ -348,7 +354,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int ks = 0; ks < ksteps; ++ks) {
+        int nks = ksteps;
+        if (MODE != 0 && a.ksplit > 1) {
+          const int b = (int)(tile / a.n_tiles / a.m_tiles);
+          nks = (int)((long long)ksteps * (b + 1) / a.ksplit) - (int)((long long)ksteps * b / a.ksplit);
+        }
+        for (int ks = 0; ks < nks; ++ks) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, a.err, DEVERR_TIMEOUT_MMA_FULL)) {
             ok = false;
             break;
@@ -583,7 +594,8 @@ bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const voi
 }
 
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt,
-                           int tile_n, int sm_count, int* err_word, bool accumulate, cudaStream_t s) {
+                           int tile_n, int sm_count, int* err_word, bool accumulate, cudaStream_t s, int ksplit,
+                           float* partial) {
   if (!tc_conv_supported(g, dt, in, w)) return cudaErrorNotSupported;
   const long long M = (long long)g.n * g.oh * g.ow;
   if (M == 0) return cudaSuccess;
@@ -620,7 +632,22 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   a.ldo = g.o;
   a.out_batch = 0;
   a.accumulate = accumulate ? 1 : 0;
+  a.ksplit = 1;
   a.err = err_word;
+  if (ksplit > 1) {
+    // split-K: ksplit partial fp32 results [ksplit][M][O], reduced by launch_splitk_reduce
+    if (!partial || ksplit > taps * a.kb_per_tap) return cudaErrorInvalidValue;
+    a.ksplit = ksplit;
+    a.batches = ksplit;
+    a.out = partial;
+    a.out_batch = M * g.o;
+    a.accumulate = 0;
+    if (dt == CONV_BF16)
+      return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
+                           : launch_kernel<128, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 1, __half, float>(tA, tB, a, sm_count, s)
+                         : launch_kernel<128, 1, __half, float>(tA, tB, a, sm_count, s);
+  }
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
                          : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
@@ -676,6 +703,7 @@ cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geo
   a.kw = g.kw; a.dh = g.dh; a.dw = g.dw;
   a.oh = g.oh; a.ow = g.ow; a.sh = g.sh; a.sw = g.sw; a.ph = g.ph; a.pw = g.pw;
   a.kh = g.kh; a.od = g.od; a.sd = g.sd; a.pd = g.pd; a.dd = g.dd;
+  a.ksplit = 1;
   a.m_rows = M;
   a.ocols = g.o;
   a.out = out;
@@ -716,6 +744,7 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   a.out = bg.d;
   a.ldo = bg.o;
   a.out_batch = (long long)bg.t * bg.o;
+  a.ksplit = 1;
   a.err = err_word;
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s)

@@ -79,7 +79,8 @@ def test_winograd_shape_plan():
 
 def test_small_shape_takes_implicit_gemm():
     st, p = plan2d(synth.SMALL_F32)       # C + O = 64 < 256
-    assert st == 0 and p["algo"] == "implicit" and p["engine"] == "simt" and p["workspace_bytes"] == 0
+    assert st == 0 and p["algo"] == "implicit" and p["engine"] == "simt"
+    assert (p["workspace_bytes"] == 0) == (p["k_split"] == 1)
 
 
 @pytest.mark.parametrize("budget,expect", [
@@ -119,7 +120,7 @@ def test_sixteen_bit_takes_tensor_cores():
             if shape.c == 3:      # the stem: 7 taps x 3 channels folded into 24 channels
                 assert p["channel_pad"] == 24 and p["packed_taps"] == 1 and p["workspace_bytes"] > 0
             else:
-                assert p["channel_pad"] == 0 and p["workspace_bytes"] == 0
+                assert p["channel_pad"] == 0 and (p["workspace_bytes"] == 0) == (p["k_split"] == 1)
 
 
 def test_sixteen_bit_forced_winograd_uses_f2x2():
@@ -216,3 +217,21 @@ def test_conv3d_guard_selects_depth_taps_or_native_gemm():
     # forcing the implicit GEMM takes the native kernel even inside the guard
     st, p = plan3d(guarded, algo="implicit")
     assert st == 0 and p["taps"] == 1
+
+
+def test_split_k_for_small_m_long_k():
+    """Under half a wave of tiles with a long K loop: the K range is split and
+    the workspace holds the fp32 partials; large grids are never split."""
+    small = synth.Conv2dShape(8, 14, 14, 512, 512, 3, 3, (2, 2), (1, 1), (1, 1))     # M = 392, K = 4608
+    for dt, tile in (("bf16", 128), ("f32", 128)):
+        st, p = plan2d(small, dt)
+        assert st == 0 and p["k_split"] >= 2
+        M = 8 * 7 * 7
+        assert p["workspace_bytes"] >= p["k_split"] * M * 512 * 4
+    big = synth.Conv2dShape(16, 64, 64, 512, 512, 3, 3, (1, 1), (1, 1), (1, 1))
+    for dt in ("bf16", "f32"):
+        st, p = plan2d(big, dt, algo="implicit")
+        assert st == 0 and p["k_split"] == 1 and p["workspace_bytes"] == 0
+    # Winograd plans never split (bit identity of batch tiling)
+    st, p = plan2d(synth.WINOGRAD_F32)
+    assert p["algo"] == "winograd" and p["k_split"] == 1

@@ -83,7 +83,10 @@ def test_misaligned_pointers_take_the_any_alignment_path(dtype):
     wm.copy_(w)
     assert xm.data_ptr() % 16 != 0 and wm.data_ptr() % 16 != 0
     out = torch.full((s.n, s.oh, s.ow, s.o), float("nan"), dtype=x.dtype, device="cuda")
-    st = B.conv2d_forward(xm.data_ptr(), wm.data_ptr(), out.data_ptr(), desc(s), B.DTYPE[dtype], None, 0, 0, stream())
+    need = B.conv2d_workspace_size(desc(s), B.DTYPE[dtype], 0, None)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    st = B.conv2d_forward(xm.data_ptr(), wm.data_ptr(), out.data_ptr(), desc(s), B.DTYPE[dtype], None,
+                          ws.data_ptr(), need, stream())
     assert st == 0
     torch.cuda.synchronize()
     ref = oracle.conv2d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
