@@ -122,9 +122,34 @@ __global__ void wpack_kernel(const T* __restrict__ src, long long pixels /* n*h*
   }
 }
 
+// Four elements per thread (count % 4 == 0, 16-byte aligned partials); the
+// partial sums are added in split order 0..ksplit-1 for every element.
 template <typename T>
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int ksplit, size_t count, T* __restrict__ out,
                                      int accumulate) {
+  const size_t n4 = count / 4;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (; i < n4; i += stride) {
+    float4 sum = __ldg(reinterpret_cast<const float4*>(partial) + i);
+    for (int k = 1; k < ksplit; ++k) {
+      const float4 p = __ldg(reinterpret_cast<const float4*>(partial + (size_t)k * count) + i);
+      sum.x += p.x; sum.y += p.y; sum.z += p.z; sum.w += p.w;
+    }
+    float v[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      T* o = out + 4 * i + e;
+      float r = v[e];
+      if (accumulate) r = Store<T>::to_f32(*o) + Store<T>::to_f32(Store<T>::from_f32(v[e]));
+      *o = Store<T>::from_f32(r);
+    }
+  }
+}
+
+template <typename T>
+__global__ void splitk_reduce_scalar_kernel(const float* __restrict__ partial, int ksplit, size_t count,
+                                            T* __restrict__ out, int accumulate) {
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (; i < count; i += stride) {
@@ -136,24 +161,54 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int kspl
   }
 }
 
+// dst[k][o] = w[o][k] (row strides w_row_stride, ldb), 32 x 32 tiles through shared memory.
+__global__ void transpose_weights_kernel(const float* __restrict__ w, int O, long long K, long long w_row_stride,
+                                         float* __restrict__ dst, long long ldb) {
+  __shared__ float tile[32][33];
+  const long long k0 = (long long)blockIdx.x * 32;
+  const int o0 = blockIdx.y * 32;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int o = o0 + r;
+    const long long k = k0 + threadIdx.x;
+    tile[r][threadIdx.x] = (o < O && k < K) ? w[(long long)o * w_row_stride + k] : 0.0f;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const long long k = k0 + r;
+    const int o = o0 + threadIdx.x;
+    if (k < K && o < O) dst[k * ldb + o] = tile[threadIdx.x][r];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_transpose_weights(const float* w, int o, long long k, long long w_row_stride, float* dst,
+                                     long long ldb, cudaStream_t s) {
+  if (o == 0 || k == 0) return cudaSuccess;
+  dim3 grid((unsigned)((k + 31) / 32), (o + 31) / 32);
+  if (grid.y > 65535) return cudaErrorInvalidValue;
+  transpose_weights_kernel<<<grid, dim3(32, 8), 0, s>>>(w, o, k, w_row_stride, dst, ldb);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count, void* out, conv_dtype_t dt,
                                  bool accumulate, cudaStream_t s) {
   if (count == 0) return cudaSuccess;
-  unsigned blocks = (unsigned)((count + 255) / 256 < 148 * 16 ? (count + 255) / 256 : 148 * 16);
   const int acc = accumulate ? 1 : 0;
+  const bool vec = count % 4 == 0 && (reinterpret_cast<uintptr_t>(partial) & 15) == 0;
+  const size_t items = vec ? count / 4 : count;
+  unsigned blocks = (unsigned)((items + 255) / 256 < 148 * 16 ? (items + 255) / 256 : 148 * 16);
+  auto run = [&](auto tag) {
+    using T = decltype(tag);
+    if (vec)
+      splitk_reduce_kernel<T><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<T*>(out), acc);
+    else
+      splitk_reduce_scalar_kernel<T><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<T*>(out), acc);
+  };
   switch (dt) {
-    case CONV_F32:
-      splitk_reduce_kernel<float><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<float*>(out), acc);
-      break;
-    case CONV_F16:
-      splitk_reduce_kernel<__half><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<__half*>(out), acc);
-      break;
-    case CONV_BF16:
-      splitk_reduce_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(partial, ksplit, count,
-                                                                 static_cast<__nv_bfloat16*>(out), acc);
-      break;
+    case CONV_F32: run(float{}); break;
+    case CONV_F16: run(__half{}); break;
+    case CONV_BF16: run(__nv_bfloat16{}); break;
   }
   return cudaGetLastError();
 }
