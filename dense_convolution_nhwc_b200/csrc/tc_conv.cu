@@ -32,6 +32,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -44,6 +45,9 @@ constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 x 16-bit = one 128-byte swizzle row
 constexpr int THREADS = 192;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+#ifndef TC_EPI_COLS
+#define TC_EPI_COLS 128        // accumulator columns an epilogue thread reads per TMEM wait
+#endif
 
 template <int BN> struct Cfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
@@ -52,7 +56,13 @@ template <int BN> struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  // fp32-output variants stage each epilogue warp's 32 x 32 chunk for a TMA
+  // store: 4 warps x 2 buffers x 4 KB, 128-byte swizzled
+  static constexpr int STORE_BYTES = 4 * 2 * 32 * 32 * 4;
+  template <typename TOut>
+  static constexpr int smem() {
+    return 1024 + STAGES * STAGE_BYTES + (sizeof(TOut) == 4 ? STORE_BYTES : 0) + BAR_BYTES;
+  }
 };
 
 struct TcArgs {
@@ -68,6 +78,7 @@ struct TcArgs {
   long long out_batch;         // elements between batches
   int accumulate;              // out = round(out + round(acc)) instead of out = round(acc)
   int ksplit;                  // conv modes: > 1 splits the K range, the split index in the batch slot
+  int tma_store;               // fp32 output: write 32 x 32 chunks with TMA stores through tmD
   int* err;
 };
 
@@ -151,6 +162,19 @@ __device__ __forceinline__ void tma_load_im2col_5d(uint32_t dst, const CUtensorM
       : "memory");
 }
 
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -208,15 +232,17 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt) {
 template <int BN, int MODE, typename TIn, typename TOut>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const TcArgs a) {
+               const __grid_constant__ CUtensorMap tmD, const TcArgs a) {
   using C = Cfg<BN>;
+  constexpr int STORE_BYTES = sizeof(TOut) == 4 ? C::STORE_BYTES : 0;
   constexpr uint32_t IDESC = make_idesc<BN>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint8_t* sStore = sB + C::STAGES * C::B_BYTES;        // fp32 output staging (1024-aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStore + STORE_BYTES);
   // bars: full[S], empty[S], tfull[2], tempty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -389,6 +415,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
     int it = 0;
+    int store_count = 0;                    // TMA-stored chunks of this warp (staging double buffer)
     for (long long tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
@@ -402,13 +429,52 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const bool row_ok = m < a.m_rows;
       TOut* orow = static_cast<TOut*>(a.out) + (long long)b * a.out_batch + (row_ok ? m : 0) * a.ldo;
       const int n0 = nt * BN;
+      // EPI columns per round: EPI/32 TMEM loads in flight behind one wait
+      constexpr int EPI = BN < TC_EPI_COLS ? BN : TC_EPI_COLS;
 #pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cc);
-        TMEM_LD32(taddr, r);
+      for (int cg = 0; cg < BN; cg += EPI) {
+        uint32_t rr[EPI / 32][32];
+#pragma unroll
+        for (int h = 0; h < EPI / 32; ++h) {
+          const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cg + 32 * h);
+          TMEM_LD32(taddr, rr[h]);
+        }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if constexpr (sizeof(TOut) == 4) {
+          if (a.tma_store) {
+            // stage row `lane` of this warp's 32 x 32 chunk (16-byte chunks XOR-swizzled by
+            // lane % 8, the TMA 128-byte swizzle), then one lane stores it; rows past the
+            // batch's last row and columns past O are clipped by the tensor map
+#pragma unroll
+            for (int h = 0; h < EPI / 32; ++h) {
+              const int c0 = n0 + cg + 32 * h;
+              if (c0 >= a.ocols) continue;
+              float* sb = reinterpret_cast<float*>(sStore + (q * 2 + (store_count & 1)) * 4096);
+              if (store_count >= 2) {
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+              }
+              float4* rowp = reinterpret_cast<float4*>(sb + lane * 32);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                rowp[k ^ (lane & 7)] = make_float4(__uint_as_float(rr[h][4 * k]), __uint_as_float(rr[h][4 * k + 1]),
+                                                   __uint_as_float(rr[h][4 * k + 2]), __uint_as_float(rr[h][4 * k + 3]));
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tmD, smem_u32(sb), c0, mt * BM + q * 32, b);
+                bulk_commit();
+              }
+              ++store_count;
+            }
+            continue;
+          }
+        }
         if (!row_ok) continue;
+#pragma unroll
+        for (int h = 0; h < EPI / 32; ++h) {
+        const uint32_t* r = rr[h];
+        const int cc = cg + 32 * h;
         const int c0 = n0 + cc;
         if (c0 >= a.ocols) continue;
         TOut* p = orow + c0;
@@ -469,9 +535,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               if (c0 + j < a.ocols) p[j] = Store<TOut>::from_f32(__uint_as_float(r[j]));
           }
         }
+        }
       }
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
+    }
+    if constexpr (sizeof(TOut) == 4) {
+      if (a.tma_store && lane == 0) bulk_wait_all();   // the last stores have landed
+      __syncwarp();
     }
   }
 
@@ -559,15 +630,31 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 template <int BN, int MODE, typename TIn, typename TOut>
 cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int sm_count,
-                          cudaStream_t s) {
+                          cudaStream_t s, const CUtensorMap* D = nullptr) {
   auto k = tc_gemm_kernel<BN, MODE, TIn, TOut>;
-  cudaError_t e = set_smem(k, Cfg<BN>::SMEM);
+  constexpr int smem = Cfg<BN>::template smem<TOut>();
+  static_assert(smem <= 232448, "shared memory budget");
+  cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
   long long tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
   if (tiles == 0) return cudaSuccess;
   int grid = (int)(tiles < sm_count ? tiles : sm_count);
-  k<<<grid, THREADS, Cfg<BN>::SMEM, s>>>(A, B, a);
+  CUtensorMap none;
+  memset(&none, 0, sizeof(none));
+  k<<<grid, THREADS, smem, s>>>(A, B, D ? *D : none, a);
   return cudaGetLastError();
+}
+
+// 3D fp32 map over D [batches][rows][cols] for the epilogue's TMA stores (box 32 x 32, 128-byte swizzle).
+bool encode_store_map(CUtensorMap* m, const float* d, long long cols, long long rows, long long batches) {
+  if (cols % 4 != 0 || (reinterpret_cast<uintptr_t>(d) & 15)) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batches};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)rows * cols * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(d), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -642,11 +729,13 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
     a.out = partial;
     a.out_batch = M * g.o;
     a.accumulate = 0;
+    CUtensorMap tD;
+    a.tma_store = encode_store_map(&tD, partial, g.o, M, ksplit) ? 1 : 0;
     if (dt == CONV_BF16)
-      return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
-                           : launch_kernel<128, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
-    return tile_n == 256 ? launch_kernel<256, 1, __half, float>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, 1, __half, float>(tA, tB, a, sm_count, s);
+      return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
+                           : launch_kernel<128, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
+    return tile_n == 256 ? launch_kernel<256, 1, __half, float>(tA, tB, a, sm_count, s, &tD)
+                         : launch_kernel<128, 1, __half, float>(tA, tB, a, sm_count, s, &tD);
   }
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
@@ -746,11 +835,13 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   a.out_batch = (long long)bg.t * bg.o;
   a.ksplit = 1;
   a.err = err_word;
+  CUtensorMap tD;
+  a.tma_store = encode_store_map(&tD, bg.d, bg.o, bg.t, bg.batches) ? 1 : 0;
   if (dt == CONV_BF16)
-    return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s);
-  return tile_n == 256 ? launch_kernel<256, 0, __half, float>(tA, tB, a, sm_count, s)
-                       : launch_kernel<128, 0, __half, float>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
+                         : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
+  return tile_n == 256 ? launch_kernel<256, 0, __half, float>(tA, tB, a, sm_count, s, &tD)
+                       : launch_kernel<128, 0, __half, float>(tA, tB, a, sm_count, s, &tD);
 }
 
 }  // namespace b200conv
