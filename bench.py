@@ -86,7 +86,7 @@ def workload(name):
         return (f"ResNet-50 v1.5 conv layer set (53 convs) {dt} batch {b[1:]} 224x224", convs, dt)
     if name.startswith("conv3d_"):
         dt = name.split("_")[1]
-        return ("conv3d bf16 NDHWC 3x3x3 s1 spatial pad 1 depth pad 0 N=1 depth taps: 17x64x64 256->256, "
+        return (f"conv3d {dt} NDHWC 3x3x3 s1 spatial pad 1 depth pad 0 N=1: 17x64x64 256->256, "
                 "41x60x104 256->256, 41x120x208 512->512", [Conv(s, dt, "normal") for s in synth.CONV3D_TAPS], dt)
     if name.startswith("wide_") or name.startswith("wide3_"):
         # wide_<dtype>: C_out >= 512 and M >= 16384 aligned members of the sweep
@@ -116,6 +116,20 @@ def kernel_work(conv, plan):
         f0, b0 = w.get(k, (0.0, 0.0))
         w[k] = (f0 + f, b0 + b)
 
+    if conv.is3d and plan["algo"] == "winograd" and plan["taps"] == 1:
+        # native 3D Winograd F(m^3, 3^3)
+        m = plan["winograd_m"]
+        a3 = (m + 2) ** 3
+        T = s.n * math.ceil(s.od / m) * math.ceil(s.oh / m) * math.ceil(s.ow / m)
+        st = 4 if plan["engine"] == "simt" else esz
+        in_b = s.n * s.d * s.h * s.w * s.c * esz
+        out_b = s.n * s.od * s.oh * s.ow * s.o * esz
+        add("wino3d_filter", 0.0, s.o * 27 * s.c * esz + a3 * s.o * s.c * st)
+        add("wino3d_input", 0.0, in_b + a3 * T * s.c * st)
+        gk = "wino3d_gemm_tc" if plan["engine"] == "tcgen05" else "wino3d_gemm_simt"
+        add(gk, 2.0 * a3 * T * s.c * s.o, a3 * T * (s.c * st + s.o * 4))
+        add("wino3d_output", 0.0, a3 * T * s.o * 4 + out_b)
+        return w
     if conv.is3d and plan["taps"] == 1 and plan["engine"] == "tcgen05":
         # native K-fused 3D implicit GEMM: one pass, output written once
         M = s.n * s.od * s.oh * s.ow
@@ -157,9 +171,9 @@ def kernel_work(conv, plan):
 
 
 def kernel_bound(name):
-    if name in ("tc_conv", "tc_conv3d", "wino_gemm_tc"):
+    if name in ("tc_conv", "tc_conv3d", "wino_gemm_tc", "wino3d_gemm_tc"):
         return "tensor"
-    if name in ("simt_conv", "wino_gemm_simt"):
+    if name in ("simt_conv", "wino_gemm_simt", "wino3d_gemm_simt"):
         return "alu"
     return "hbm"
 
@@ -168,9 +182,13 @@ KERNEL_SOURCES = {
     "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["wino_gemm_f32.cu"],
     "tc_conv": ["tc_conv.cu", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "common.cuh"],
     "tc_conv3d": ["tc_conv.cu", "common.cuh"],
-    "wino_input": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
-    "wino_output": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
-    "wino_filter": ["winograd.cu", "winograd_gen.cuh", "common.cuh"],
+    "wino_input": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino_output": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino_filter": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino3d_gemm_simt": ["wino_gemm_f32.cu"], "wino3d_gemm_tc": ["tc_conv.cu", "common.cuh"],
+    "wino3d_input": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino3d_output": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino3d_filter": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "accumulate": ["elementwise.cu", "common.cuh"], "channel_pad": ["elementwise.cu", "common.cuh"],
 }
 

@@ -77,9 +77,11 @@ long long out_extent(long long in, int k, int s, int p, int d) {
 // Opt-in: each kernel launch is bracketed by two events on its stream.
 
 enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_SPLITK_REDUCE, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
-            K_WINO_OUTPUT, K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
+            K_WINO_OUTPUT, K_WINO3D_FILTER, K_WINO3D_INPUT, K_WINO3D_GEMM_TC, K_WINO3D_GEMM_SIMT, K_WINO3D_OUTPUT,
+            K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
 const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "splitk_reduce", "wino_filter", "wino_input", "wino_gemm_tc",
-                                        "wino_gemm_simt", "wino_output", "accumulate", "channel_pad", "fill"};
+                                        "wino_gemm_simt", "wino_output", "wino3d_filter", "wino3d_input", "wino3d_gemm_tc",
+                                        "wino3d_gemm_simt", "wino3d_output", "accumulate", "channel_pad", "fill"};
 
 struct ProfRecord {
   int kind;
@@ -581,19 +583,108 @@ bool native3d_shape_ok(const Geom3& g, conv_dtype_t dt, const conv_device_props_
          (long long)g.dd * (g.kd - 1) <= 65535;
 }
 
+// Native 3D Winograd F(m^3, 3^3): 3x3x3 kernels, stride 1, dilation 1, any
+// padding.  fp32 takes F(4,3) along each axis (alpha^3 = 216); 16-bit takes
+// F(2,3) (alpha^3 = 64), whose transforms keep bf16 inside its tolerance.
+bool wino3d_shape(const conv3d_desc_t* d) {
+  for (int i = 0; i < 3; ++i)
+    if (d->stride[i] != 1 || d->dilation[i] != 1) return false;
+  return d->kd == 3 && d->kh == 3 && d->kw == 3;
+}
+int wino3d_m_for(conv_dtype_t dt) { return dt == CONV_F32 ? 4 : 2; }
+
+// Workspace of the 3D Winograd path for batch tiles of nu units, a unit being
+// one (image, depth tile) slab of tiles_hw tiles:
+//   tensor-core GEMM (16-bit operands): U [a3][O][C], V [a3][T][C], M [a3][T][O] fp32
+//   FFMA GEMM (fp32 operands):          U [a3][C][O4], V [a3][T][C], M [a3][T][O] fp32
+struct Wino3Layout {
+  size_t u_bytes = 0, v_bytes = 0, m_bytes = 0;
+  long long tiles_hw = 0, units = 0;
+  size_t per_unit = 0;   // V + M bytes per unit (the budget unit)
+};
+
+Wino3Layout wino3d_layout(const Geom3& g, conv_dtype_t store, bool ffma, int m, long long nu) {
+  Wino3Layout L;
+  const long long a3 = (long long)(m + 2) * (m + 2) * (m + 2);
+  L.tiles_hw = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+  L.units = (long long)g.n * ((g.od + m - 1) / m);
+  const int esz = dtype_size(store);
+  L.per_unit = (size_t)(a3 * L.tiles_hw) * ((size_t)g.c * esz + (size_t)g.o * 4);
+  const long long t = nu * L.tiles_hw;
+  L.u_bytes = align256((size_t)(a3 * g.c * (ffma ? round4(g.o) : g.o)) * esz);
+  L.v_bytes = align256((size_t)(a3 * t * g.c) * esz);
+  L.m_bytes = align256((size_t)(a3 * t * g.o) * 4);
+  return L;
+}
+
+// The Winograd selection of select2d with units in place of images.  Returns
+// true and fills s when the 3D Winograd runs.
+bool select_wino3d(const conv3d_desc_t* d, const Geom3& g, conv_dtype_t dt, const conv_device_props_t& p,
+                   const conv_options_t& o, Sel* s) {
+  if (!wino3d_shape(d) || g.n == 0 || g.c % 4 != 0) return false;
+  if (o.algo == CONV_ALGO_AUTO) {
+    if (dt != CONV_F32 || g.c % 32 != 0 || g.o % 32 != 0 || g.c + g.o < 256) return false;
+  } else if (o.algo != CONV_ALGO_WINOGRAD) {
+    return false;
+  }
+  const int m = wino3d_m_for(dt);
+  const bool tc_gemm = dt != CONV_F32 && p.cc_major == 10 && g.c % 8 == 0;
+  const conv_dtype_t store = tc_gemm ? dt : CONV_F32;
+  const Wino3Layout L1 = wino3d_layout(g, store, !tc_gemm, m, 1);
+  const int esz = dtype_size(dt);
+  long long budget;
+  if (o.winograd_budget_bytes >= 0) {
+    budget = o.winograd_budget_bytes;
+  } else {
+    const long long own = (long long)g.n * g.d * g.h * g.w * g.c * esz +
+                          (long long)g.n * g.od * g.oh * g.ow * g.o * esz + (long long)L1.u_bytes;
+    budget = std::min((long long)(p.total_global_mem / 4 * 3) - own, kWinogradCap);
+  }
+  long long nu = budget > 0 ? budget / (long long)L1.per_unit : 0;
+  nu = std::min<long long>(nu, L1.units);
+  const bool forced_tile = o.winograd_tile_batch > 0;
+  if (forced_tile) nu = std::min<long long>(nu, o.winograd_tile_batch);
+  const long long r_min = (long long)p.sm_count * 128;
+  if (nu <= 0 || (!forced_tile && nu < L1.units && nu * L1.tiles_hw < r_min)) return false;
+  s->algo = CONV_ALGO_WINOGRAD;
+  s->engine = tc_gemm ? CONV_ENGINE_TCGEN05 : CONV_ENGINE_SIMT;
+  s->wino_m = m;
+  s->wino_store = store;
+  s->nb = (int)nu;
+  s->ntiles = (int)((L1.units + nu - 1) / nu);
+  s->tile_m = 128;
+  s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
+  s->cpad = 0;
+  s->wpack = false;
+  s->ksplit = 1;
+  const Wino3Layout L = wino3d_layout(g, store, !tc_gemm, m, nu);
+  s->ws = L.u_bytes + L.v_bytes + L.m_bytes;
+  return true;
+}
+
+enum Path3d { P3_TAPS, P3_NATIVE, P3_WINO3D };
+
 conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_device_props_t& p,
                           const conv_options_t& o, Sel* s, Geom* g2, long long* od, size_t* ws_total,
-                          bool* native) {
+                          Path3d* path) {
   if (!valid_dtype(dt)) return CONV_ERR_INVALID;
   conv_status_t st = geom3d(d, od, g2);
   if (st != CONV_OK) return st;
   const Geom3 g3 = geom3_of(d, *od, *g2);
+  // fp32 3x3x3 stride-1 convs under the channel rule (or any dtype, forced):
+  // the native 3D Winograd, when its workspace budget allows a full wave.
+  if (select_wino3d(d, g3, dt, p, o, s)) {
+    *path = P3_WINO3D;
+    *ws_total = s->ws;
+    return CONV_OK;
+  }
   const bool can_native = native3d_shape_ok(g3, dt, p);
   // Auto: the page's guard keeps the depth taps; the cases it sends to a native
   // 3D kernel go to the K-fused tcgen05 implicit GEMM.  Forcing the implicit
   // GEMM asks for the native kernel whenever it can run the shape.
-  *native = can_native && ((o.algo == CONV_ALGO_AUTO && !depth_tap_guard(d)) || o.algo == CONV_ALGO_IMPLICIT_GEMM);
-  if (*native) {
+  const bool native = can_native && ((o.algo == CONV_ALGO_AUTO && !depth_tap_guard(d)) || o.algo == CONV_ALGO_IMPLICIT_GEMM);
+  *path = native ? P3_NATIVE : P3_TAPS;
+  if (native) {
     s->algo = CONV_ALGO_IMPLICIT_GEMM;
     s->engine = CONV_ENGINE_TCGEN05;
     s->tile_m = 128;
@@ -611,6 +702,52 @@ conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_de
   if (st != CONV_OK) return st;
   // Taps after the first add into out inside their own output stage: no tap scratch.
   *ws_total = s->ws;
+  return CONV_OK;
+}
+
+// Run the planned 3D Winograd: the filter transform once, then per batch tile
+// of s.nb units the input transform, the alpha^3 batched GEMMs and the output
+// transform, all through one reused workspace.
+conv_status_t run3d_winograd(const void* in, const void* w, void* out, const Geom3& g, conv_dtype_t dt, const Sel& s,
+                             void* ws, const DeviceState& d, cudaStream_t st) {
+  const int m = s.wino_m, a3 = (m + 2) * (m + 2) * (m + 2);
+  const bool ffma = s.engine == CONV_ENGINE_SIMT;
+  const Wino3Layout L = wino3d_layout(g, s.wino_store, ffma, m, s.nb);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* u = base;
+  void* v = base + L.u_bytes;
+  float* mb = reinterpret_cast<float*>(base + L.u_bytes + L.v_bytes);
+  cudaError_t e;
+  {
+    ProfScope ps(K_WINO3D_FILTER, st);
+    e = launch_wino3d_filter(w, g.o, g.c, m, dt, s.wino_store, ffma, round4(g.o), u, st);
+  }
+  if (e != cudaSuccess) return CONV_ERR_CUDA;
+  for (long long u0 = 0; u0 < L.units; u0 += s.nb) {
+    const long long nu = std::min<long long>(s.nb, L.units - u0);
+    const long long t = nu * L.tiles_hw;
+    if (t > 0x7fffffffLL) return CONV_ERR_UNSUPPORTED;
+    {
+      ProfScope ps(K_WINO3D_INPUT, st);
+      e = launch_wino3d_input(in, g, u0, nu, m, dt, s.wino_store, v, t, st);
+    }
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    if (ffma) {
+      ProfScope ps(K_WINO3D_GEMM_SIMT, st);
+      e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), mb, a3, (int)t, g.c, g.o,
+                               g.c, round4(g.o), true, st);
+    } else {
+      BatchedGemm bg{a3, (int)t, g.c, g.o, v, u, mb};
+      ProfScope ps(K_WINO3D_GEMM_TC, st);
+      e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
+    }
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    {
+      ProfScope ps(K_WINO3D_OUTPUT, st);
+      e = launch_wino3d_output(mb, g, u0, nu, m, t, dt, out, st);
+    }
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+  }
   return CONV_OK;
 }
 
@@ -732,10 +869,10 @@ conv_status_t conv3d_plan_for_props(const conv3d_desc_t* desc, conv_dtype_t dtyp
   Geom g2;
   long long od;
   size_t ws;
-  bool native = false;
-  conv_status_t st = plan3d_impl(desc, dtype, *props, effective_options(opts), &s, &g2, &od, &ws, &native);
+  Path3d path = P3_TAPS;
+  conv_status_t st = plan3d_impl(desc, dtype, *props, effective_options(opts), &s, &g2, &od, &ws, &path);
   if (st != CONV_OK) return st;
-  fill_plan(s, plan, native ? 1 : desc->kd, ws);
+  fill_plan(s, plan, path == P3_TAPS ? desc->kd : 1, ws);
   return CONV_OK;
 }
 
@@ -763,8 +900,8 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
   Geom g2;
   long long od;
   size_t ws;
-  bool native = false;
-  st = plan3d_impl(desc, dtype, d->props, effective_options(opts), &s, &g2, &od, &ws, &native);
+  Path3d path = P3_TAPS;
+  st = plan3d_impl(desc, dtype, d->props, effective_options(opts), &s, &g2, &od, &ws, &path);
   if (st != CONV_OK) return st;
   if (desc->n == 0) return CONV_OK;
   if (!in || !w || !out) return CONV_ERR_INVALID;
@@ -779,7 +916,8 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
     return CONV_ERR_INVALID;
 
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  if (native) {
+  if (path == P3_WINO3D) return run3d_winograd(in, w, out, geom3_of(desc, od, g2), dtype, s, workspace, *d, st_);
+  if (path == P3_NATIVE) {
     const Geom3 g3 = geom3_of(desc, od, g2);
     if (tc_conv3d_supported(g3, dtype, in, w)) {
       ProfScope ps(K_TC_CONV3D, st_);

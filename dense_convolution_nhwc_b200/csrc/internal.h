@@ -107,6 +107,19 @@ cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb,
                                long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
                                cudaStream_t s);
 
+// Native 3D Winograd F(m^3, 3^3) transforms, m in {2, 4}, for 3x3x3 stride-1
+// dilation-1 convs.  Tiles are numbered unit-major, a unit being one (image,
+// depth tile) slab of ceil(OH/m)*ceil(OW/m) tiles; a call covers units
+// [u0, u0 + nu).  U: [a3][C][o_pad] fp32 (cmajor) or [a3][O][C] in store_dt;
+// V: [a3][t_stride][C] in store_dt; M: [a3][t_stride][O] fp32.
+cudaError_t launch_wino3d_filter(const void* w, int o, int c, int m, conv_dtype_t in_dt, conv_dtype_t store_dt,
+                                 bool cmajor, long long o_pad, void* u, cudaStream_t s);
+cudaError_t launch_wino3d_input(const void* in, const Geom3& g, long long u0, long long nu, int m,
+                                conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_stride,
+                                cudaStream_t s);
+cudaError_t launch_wino3d_output(const float* mbuf, const Geom3& g, long long u0, long long nu, int m,
+                                 long long t_stride, conv_dtype_t out_dt, void* out, cudaStream_t s);
+
 // Elementwise helpers.
 cudaError_t launch_accumulate(void* out, const void* tap, size_t count, conv_dtype_t dt,
                               cudaStream_t s);

@@ -17,34 +17,12 @@
 // tile it was processed in (batch tiling stays bit-identical).
 #include <cuda_runtime.h>
 
-#include <type_traits>
-
 #include "common.cuh"
 #include "internal.h"
-#include "winograd_gen.cuh"
+#include "wino_1d.cuh"
 
 namespace b200conv {
 namespace {
-
-template <int M> struct Wino;
-template <> struct Wino<2> {
-  static constexpr int A = 4;
-  static __device__ __forceinline__ void bt(const float* x, float* y) { wino2_bt(x, y); }
-  static __device__ __forceinline__ void g(const float* x, float* y) { wino2_g(x, y); }
-  static __device__ __forceinline__ void at(const float* x, float* y) { wino2_at(x, y); }
-};
-template <> struct Wino<4> {
-  static constexpr int A = 6;
-  static __device__ __forceinline__ void bt(const float* x, float* y) { wino4_bt(x, y); }
-  static __device__ __forceinline__ void g(const float* x, float* y) { wino4_g(x, y); }
-  static __device__ __forceinline__ void at(const float* x, float* y) { wino4_at(x, y); }
-};
-template <> struct Wino<6> {
-  static constexpr int A = 8;
-  static __device__ __forceinline__ void bt(const float* x, float* y) { wino6_bt(x, y); }
-  static __device__ __forceinline__ void g(const float* x, float* y) { wino6_g(x, y); }
-  static __device__ __forceinline__ void at(const float* x, float* y) { wino6_at(x, y); }
-};
 
 // ---------------------------------------------------------------------------
 // Filter transform: one thread per (o, c).
@@ -349,26 +327,6 @@ wino_input_cmajor_kernel(const Tin* __restrict__ in, const WinoInCArgs a, float*
   }
 }
 
-template <typename F>
-cudaError_t by_m(int m, F&& f) {
-  switch (m) {
-    case 2: return f(std::integral_constant<int, 2>{});
-    case 4: return f(std::integral_constant<int, 4>{});
-    case 6: return f(std::integral_constant<int, 6>{});
-  }
-  return cudaErrorInvalidValue;
-}
-
-template <typename F>
-cudaError_t by_dt(conv_dtype_t dt, F&& f) {
-  switch (dt) {
-    case CONV_F32: return f(float{});
-    case CONV_F16: return f(__half{});
-    case CONV_BF16: return f(__nv_bfloat16{});
-  }
-  return cudaErrorInvalidValue;
-}
-
 }  // namespace
 
 cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int c, int m,
@@ -376,11 +334,11 @@ cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int
   long long n = (long long)o * c;
   if (n == 0) return cudaSuccess;
   unsigned blocks = (unsigned)((n + 255) / 256);
-  return by_m(m, [&](auto mc) {
+  return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
-    return by_dt(in_dt, [&](auto ti) {
+    return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
-      return by_dt(store_dt, [&](auto ts) {
+      return wino_by_dt(store_dt, [&](auto ts) {
         using Tst = decltype(ts);
         wino_filter_kernel<M, Tin, Tst><<<blocks, 256, 0, s>>>(
             static_cast<const Tin*>(w), w_row_stride, o, c, static_cast<Tst*>(u));
@@ -407,11 +365,11 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   const long long blocks = ((a.t_count + block.y - 1) / block.y) * ((g.c + bx - 1) / bx);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)blocks);
-  return by_m(m, [&](auto mc) {
+  return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
-    return by_dt(in_dt, [&](auto ti) {
+    return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
-      return by_dt(store_dt, [&](auto ts) {
+      return wino_by_dt(store_dt, [&](auto ts) {
         using Tst = decltype(ts);
         wino_input_kernel<M, Tin, Tst><<<grid, block, 0, s>>>(static_cast<const Tin*>(in), a,
                                                               static_cast<Tst*>(v));
@@ -426,9 +384,9 @@ cudaError_t launch_wino_filter_cmajor(const void* w, long long w_row_stride, int
   long long n = (long long)o * c;
   if (n == 0) return cudaSuccess;
   unsigned blocks = (unsigned)((n + 255) / 256);
-  return by_m(m, [&](auto mc) {
+  return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
-    return by_dt(in_dt, [&](auto ti) {
+    return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
       wino_filter_cmajor_kernel<M, Tin><<<blocks, 256, 0, s>>>(static_cast<const Tin*>(w), w_row_stride, o, c,
                                                                 o_pad, u);
@@ -451,9 +409,9 @@ cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int 
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)blocks);
-  return by_m(m, [&](auto mc) {
+  return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
-    return by_dt(in_dt, [&](auto ti) {
+    return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
       auto k = wino_input_cmajor_kernel<M, Tin>;
       cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Strip<M>::BYTES);
@@ -481,9 +439,9 @@ cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb,
   dim3 block(bx, 256 / bx);
   dim3 grid((unsigned)((a.t_count + block.y - 1) / block.y), (g.o + bx - 1) / bx);
   if (grid.y > 65535) return cudaErrorInvalidValue;
-  return by_m(m, [&](auto mc) {
+  return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
-    return by_dt(out_dt, [&](auto to) {
+    return wino_by_dt(out_dt, [&](auto to) {
       using Tout = decltype(to);
       wino_output_kernel<M, Tout><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
       return cudaGetLastError();

@@ -26,7 +26,9 @@
  *    the batch", Fix and Testing).
  * conv3d runs as KD depth-tap 2D convs over zero-copy frame views whose results
  * are accumulated in place ("Decompose small kernel-depth 3D convs into 2D
- * convs", Change).
+ * convs", Change), as a native 3D implicit GEMM, or, for 3x3x3 stride-1
+ * convs, as a native 3D Winograd F(m x m x m, 3 x 3 x 3) (that page's Open
+ * questions, item 3).
  *
  * Conventions shared by every entry point:
  *  - Pointers named in/w/out/workspace are DEVICE pointers owned by the caller;
@@ -128,8 +130,10 @@ typedef struct {
     conv_algo_t algo;          /* the algorithm that will run */
     conv_engine_t engine;      /* the GEMM engine under it */
     int tile_m, tile_n;        /* GEMM tile (rows x output channels) */
-    int winograd_m;            /* m of F(m x m, 3 x 3); 0 unless Winograd */
-    int batch_tile;            /* images per Winograd batch tile (= n when untiled) */
+    int winograd_m;            /* m of F(m x m, 3 x 3) (F(m^3, 3^3) for the 3D Winograd); 0 unless Winograd */
+    int batch_tile;            /* images per Winograd batch tile (= n when untiled); for the
+                                  3D Winograd, units per tile, a unit being one (image, depth
+                                  tile of m output frames) slab */
     int num_batch_tiles;       /* number of batch tiles */
     int channel_pad;           /* padded channel count of the pre-pass, 0 if none */
     int packed_taps;           /* 1 if the KW taps are folded into channel_pad channels (few-channel inputs) */
@@ -188,7 +192,7 @@ B200CONV_API conv_status_t conv1d_forward(const void *in, const void *w, void *o
                                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * conv3d, in[N,D,H,W,C], w[O,KD,KH,KW,C], out[N,OD,OH,OW,O].  Two algorithms:
+ * conv3d, in[N,D,H,W,C], w[O,KD,KH,KW,C], out[N,OD,OH,OW,O].  Three algorithms:
  *  - depth taps ("Decompose small kernel-depth 3D convs into 2D convs",
  *    Change): for each kd, a 2D conv over the zero-copy view of the input
  *    frames at depth offset kd*dd (frame stride sd*H*W*C) with the weight slice
@@ -199,13 +203,23 @@ B200CONV_API conv_status_t conv1d_forward(const void *in, const void *w, void *o
  *    exists.
  *  - a native 3D implicit GEMM (16-bit, tensor cores): K = KD*KH*KW*C in one
  *    main loop, A tiles gathered by a 5D TMA im2col map; output written once.
- * With CONV_ALGO_AUTO the page's guard (N == 1, KD <= 7, depth stride 1,
+ *  - a native 3D Winograd for KD = KH = KW = 3, all strides and dilations 1,
+ *    any padding, C % 4 == 0: the 1D F(m, 3) transforms applied along depth,
+ *    height and width around alpha^3 batched GEMMs (F(4,3), alpha^3 = 216, for
+ *    fp32; F(2,3), alpha^3 = 64, for 16-bit).  Its workspace is tiled over
+ *    units (image, depth tile of m output frames) under the conv2d Winograd
+ *    budget rule, tiled output bit-identical to untiled.
+ * With CONV_ALGO_AUTO, fp32 shapes of the 3D Winograd that meet the conv2d
+ * channel rule (C % 32 == 0, O % 32 == 0, C + O >= 256) take it when the
+ * budget allows (the same fallback rule as conv2d); otherwise the page's guard (N == 1, KD <= 7, depth stride 1,
  * kernel dilation 1, no depth padding, C and O multiples of 16) selects the
  * depth taps and the other shapes take the native GEMM when it can express them
  * (16-bit, C % 8 == 0, 5D box corners within [-16, 15]), else the depth taps.
  * CONV_ALGO_IMPLICIT_GEMM asks for the native GEMM whenever it can run;
- * CONV_ALGO_WINOGRAD / CONV_ALGO_DIRECT pick the depth taps' 2D algorithm.
- * plan->taps is KD for depth taps and 1 for the native GEMM.
+ * CONV_ALGO_WINOGRAD asks for the 3D Winograd on its shapes (any dtype, no
+ * channel rule) and otherwise for depth taps with the 2D Winograd;
+ * CONV_ALGO_DIRECT picks the depth taps' any-alignment 2D path.
+ * plan->taps is KD for depth taps and 1 for the native GEMM and the 3D Winograd.
  */
 B200CONV_API conv_status_t conv3d_plan(const conv3d_desc_t *desc, conv_dtype_t dtype, int device,
                           const conv_options_t *opts, conv_plan_t *plan);

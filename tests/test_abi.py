@@ -219,6 +219,73 @@ def test_conv3d_guard_selects_depth_taps_or_native_gemm():
     assert st == 0 and p["taps"] == 1
 
 
+def wino3d_ws(s, m, store_bytes, ffma, nu):
+    """U + V + M bytes of the 3D Winograd workspace for batch tiles of nu units."""
+    al = lambda x: (x + 255) // 256 * 256
+    a3 = (m + 2) ** 3
+    tiles_hw = -(-s.oh // m) * -(-s.ow // m)
+    t = nu * tiles_hw
+    o_u = (s.o + 3) // 4 * 4 if ffma else s.o
+    return al(a3 * s.c * o_u * store_bytes) + al(a3 * t * s.c * store_bytes) + al(a3 * t * s.o * 4)
+
+
+def test_conv3d_winograd_plan():
+    """fp32 3x3x3 stride-1 convs under the channel rule take the native 3D
+    Winograd F(4,3)^3 on the FFMA GEMM; 16-bit keeps the taps / native GEMM
+    unless Winograd is forced, which gives F(2,3)^3 on the tensor cores."""
+    s = synth.Conv3dShape(2, 17, 32, 32, 128, 128, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1))
+    units = 2 * -(-s.od // 4)
+    st, p = plan3d(s, "f32")
+    assert st == 0 and p["algo"] == "winograd" and p["winograd_m"] == 4 and p["taps"] == 1
+    assert p["engine"] == "simt" and p["batch_tile"] == units and p["num_batch_tiles"] == 1
+    assert p["workspace_bytes"] == wino3d_ws(s, 4, 4, True, units)
+    st, p = plan3d(s, "bf16")
+    assert st == 0 and p["algo"] != "winograd"
+    for dt in ("bf16", "f16"):
+        st, p = plan3d(s, dt, algo="winograd")
+        assert st == 0 and p["algo"] == "winograd" and p["winograd_m"] == 2 and p["engine"] == "tcgen05"
+        assert p["workspace_bytes"] == wino3d_ws(s, 2, 2, False, p["batch_tile"])
+    # channel rule (auto): C + O < 256 stays on depth taps; forcing ignores the rule
+    small = synth.Conv3dShape(1, 6, 8, 8, 32, 64, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    st, p = plan3d(small, "f32")
+    assert st == 0 and p["taps"] == 3
+    st, p = plan3d(small, "f32", algo="winograd")
+    assert st == 0 and p["algo"] == "winograd" and p["taps"] == 1 and p["winograd_m"] == 4
+    # not 3x3x3 / stride 1 / dilation 1: depth taps (forced Winograd: each tap's 2D Winograd)
+    for other in [synth.Conv3dShape(1, 9, 16, 16, 128, 128, 2, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),
+                  synth.Conv3dShape(1, 9, 16, 16, 128, 128, 3, 3, 3, (2, 1, 1), (0, 1, 1), (1, 1, 1)),
+                  synth.Conv3dShape(1, 9, 16, 16, 128, 128, 3, 3, 3, (1, 1, 1), (2, 1, 1), (2, 1, 1))]:
+        st, p = plan3d(other, "f32", algo="winograd")
+        assert st == 0 and p["taps"] == other.kd and p["winograd_m"] == 6, other
+    # C % 4 != 0: no 3D Winograd even when forced
+    odd = synth.Conv3dShape(1, 6, 8, 8, 6, 32, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    st, p = plan3d(odd, "f32", algo="winograd")
+    assert st == 0 and p["taps"] == 3
+
+
+def test_conv3d_winograd_budget_tiles_units():
+    """The budget bounds V + M per unit (one image's depth tile of m frames); a
+    forced tile is capped by it; tiles under one wave of 128-row GEMM tiles, or
+    a budget under one unit, fall back to the depth taps."""
+    s = synth.Conv3dShape(1, 42, 64, 64, 64, 256, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))   # OD = 40: 10 units
+    per_unit = 216 * (16 * 16) * (64 * 4 + 256 * 4)
+    st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit + 5, winograd_tile_batch=10)
+    assert st == 0 and p["algo"] == "winograd" and p["batch_tile"] == 3 and p["num_batch_tiles"] == 4
+    assert p["workspace_bytes"] == wino3d_ws(s, 4, 4, True, 3)
+    st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit, winograd_tile_batch=2)
+    assert st == 0 and p["batch_tile"] == 2 and p["num_batch_tiles"] == 5
+    st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit)      # 768 rows per tile < one wave
+    assert st == 0 and p["taps"] == 3
+    st, p = plan3d(s, "f32", winograd_budget_bytes=per_unit - 1, winograd_tile_batch=1)
+    assert st == 0 and p["taps"] == 3
+    big = synth.Conv3dShape(1, 42, 256, 256, 64, 256, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    per_unit = 216 * (64 * 64) * (64 * 4 + 256 * 4)
+    st, p = plan3d(big, "f32", winograd_budget_bytes=5 * per_unit)    # 5 * 4096 rows >= 148 * 128
+    assert st == 0 and p["algo"] == "winograd" and p["batch_tile"] == 5 and p["num_batch_tiles"] == 2
+    st, p = plan3d(big, "f32", winograd_budget_bytes=4 * per_unit)    # 4 * 4096 rows < 148 * 128
+    assert st == 0 and p["taps"] == 3 and p["winograd_m"] != 4        # depth taps (each a 2D Winograd)
+
+
 def test_split_k_for_small_m_long_k():
     """Under half a wave of tiles with a long K loop: the K range is split and
     the workspace holds the fp32 partials; large grids are never split."""

@@ -137,3 +137,73 @@ def test_native_and_taps_agree():
     ref = oracle.conv3d(x.cpu(), w.cpu(), "bf16", s.stride, s.pad, s.dilation)
     assert_close(as_f64(a), ref, "bf16", "native")
     assert_close(as_f64(b), ref, "bf16", "taps")
+
+
+# ---------------------------------------------------------------------------
+# Native 3D Winograd F(m^3, 3^3): the depth-tap page's open question on a
+# native 3D Winograd, built as the 2D method nested along depth.
+# ---------------------------------------------------------------------------
+
+WINO3D = [
+    synth.Conv3dShape(1, 10, 12, 12, 128, 128, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1)),   # whole 4^3 tiles
+    synth.Conv3dShape(2, 9, 13, 11, 64, 192, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # ragged in every dim, N = 2
+    synth.Conv3dShape(1, 7, 9, 10, 96, 160, 3, 3, 3, (1, 1, 1), (2, 0, 2), (1, 1, 1)),      # pads 2 / 0 / 2
+    synth.Conv3dShape(3, 5, 6, 7, 32, 224, 3, 3, 3, (1, 1, 1), (0, 2, 1), (1, 1, 1)),       # small volumes, OD = 3
+]
+
+
+def wino3d_plan(s, dtype, options=None):
+    desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+    return B.plan3d(desc, dtype, 0, options)
+
+
+@pytest.mark.parametrize("s", WINO3D, ids=lambda s: s.name())
+def test_winograd3d_f32_auto_against_oracle(s):
+    p = wino3d_plan(s, "f32")
+    assert p["algo"] == "winograd" and p["winograd_m"] == 4 and p["taps"] == 1
+    check3d(s, "f32")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("s", WINO3D[1:3], ids=lambda s: s.name())
+def test_winograd3d_16bit_forced_against_oracle(s, dtype):
+    opt = B.make_options("winograd")
+    p = wino3d_plan(s, dtype, opt)
+    assert p["algo"] == "winograd" and p["winograd_m"] == 2 and p["engine"] == "tcgen05"
+    check3d(s, dtype, options=opt)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_winograd3d_forced_unaligned_channels(dtype):
+    """C % 8 != 0 (16-bit operands then go through the FFMA GEMM in fp32) and an
+    O that is no multiple of 32 or of a GEMM tile."""
+    s = synth.Conv3dShape(2, 6, 7, 9, 36, 20, 3, 3, 3, (1, 1, 1), (1, 1, 0), (1, 1, 1))
+    opt = B.make_options("winograd")
+    p = wino3d_plan(s, dtype, opt)
+    assert p["algo"] == "winograd" and p["taps"] == 1 and p["engine"] == "simt"
+    check3d(s, dtype, options=opt)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_winograd3d_unit_tiling_is_bit_identical(dtype):
+    """Tiles of 1 and 2 units (the latter straddling images) equal the untiled
+    run bit for bit."""
+    s = synth.Conv3dShape(2, 11, 10, 9, 64, 192, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))   # OD = 9
+    units = 2 * (3 if dtype == "f32" else 5)          # depth tiles of 4 (fp32) or 2 (16-bit) frames
+    x, w = synth.conv3d_inputs(s, dtype, "normal", 3, device="cuda")
+    outs = []
+    for tb in (0, 1, 2):
+        opt = B.make_options("winograd", winograd_tile_batch=tb)
+        p = wino3d_plan(s, dtype, opt)
+        assert p["algo"] == "winograd" and p["batch_tile"] == (units if tb == 0 else tb)
+        outs.append(run3d(x, w, s, opt))
+    iv = torch.int32 if dtype == "f32" else torch.int16
+    assert torch.equal(outs[0].view(iv), outs[1].view(iv))
+    assert torch.equal(outs[0].view(iv), outs[2].view(iv))
+
+
+@pytest.mark.parametrize("s", synth.CONV3D_TAPS, ids=lambda s: s.name())
+def test_workload_shapes_f32_sampled(s):
+    """The conv3d workload in fp32: the 3D Winograd where its budget allows a
+    wave of GEMM rows, depth taps (each a 2D Winograd) otherwise."""
+    check3d(s, "f32", sample=1024)

@@ -4,6 +4,8 @@
   arithmetic, 1D and 2D: A^T[(G g) . (B^T d)] = sum_k g_k d_{i+k} and
   A^T[(G g G^T) . (B^T d B)]A = the 3x3 correlation of the tile (the method of
   "Fast Algorithms for Convolutional Neural Networks", Lavin and Gray).
+* The same matrices nested along three axes reproduce the 3x3x3 correlation
+  of an alpha^3 cube exactly (the native 3D Winograd's transforms).
 * The committed header is exactly what the generator writes.
 * The generated straight-line code (paired even/odd sums) computes those
   matrices: it is compiled with g++ as C++ and compared with the exact
@@ -53,6 +55,40 @@ def test_matrices_reproduce_2d_correlation_exactly(m):
     V = mm(mm(BT, d), tr(BT))
     Y = mm(mm(AT, [[U[i][j] * V[i][j] for j in range(a)] for i in range(a)]), tr(AT))
     want = [[sum(g[u][v] * d[i + u][j + v] for u in range(3) for v in range(3)) for j in range(m)] for i in range(m)]
+    assert Y == want
+
+
+@pytest.mark.parametrize("m", [2, 4])
+def test_matrices_reproduce_3d_correlation_exactly(m):
+    """(A^T (x) A^T (x) A^T)[(G (x) G (x) G) g . (B^T (x) B^T (x) B^T) d] is the
+    3x3x3 correlation of the alpha^3 cube d, each 1D matrix applied along one
+    axis in turn (depth, height, width)."""
+    AT, G, BT = gen_winograd.matrices(m)
+    a = m + 2
+    rng = random.Random(20 + m)
+
+    def along(M, X, axis):
+        """Apply the matrix M along one axis of the nested-list cube X."""
+        n0, n1, n2 = len(X), len(X[0]), len(X[0][0])
+        if axis == 0:
+            return [[[sum(M[i][k] * X[k][y][z] for k in range(n0)) for z in range(n2)] for y in range(n1)]
+                    for i in range(len(M))]
+        if axis == 1:
+            return [[[sum(M[i][k] * X[x][k][z] for k in range(n1)) for z in range(n2)] for i in range(len(M))]
+                    for x in range(n0)]
+        return [[[sum(M[i][k] * X[x][y][k] for k in range(n2)) for i in range(len(M))] for y in range(n1)]
+                for x in range(n0)]
+
+    def cube3(M, X):
+        return along(M, along(M, along(M, X, 0), 1), 2)
+
+    g = [[[Fr(rng.randint(-4, 4)) for _ in range(3)] for _ in range(3)] for _ in range(3)]
+    d = [[[Fr(rng.randint(-4, 4)) for _ in range(a)] for _ in range(a)] for _ in range(a)]
+    U, V = cube3(G, g), cube3(BT, d)
+    P = [[[U[i][j][k] * V[i][j][k] for k in range(a)] for j in range(a)] for i in range(a)]
+    Y = cube3(AT, P)
+    want = [[[sum(g[u][v][w] * d[i + u][j + v][k + w] for u in range(3) for v in range(3) for w in range(3))
+              for k in range(m)] for j in range(m)] for i in range(m)]
     assert Y == want
 
 
