@@ -71,6 +71,12 @@ def workload(name):
         n, h, w, c, o, k, st, pd, dl = (int(v) for v in dims.split(","))
         shape = synth.Conv2dShape(n, h, w, c, o, k, k, (st, st), (pd, pd), (dl, dl))
         return f"conv2d {dt} NHWC {shape.name()}", [Conv(shape, dt, "uniform" if dt == "f32" else "normal")], dt
+    if name.startswith("conv3d:"):
+        # conv3d:<n>,<d>,<h>,<w>,<c>,<o>,<k>,<stride>,<pad_d>,<pad_hw>:<dtype>  (a single conv, e.g. for ncu)
+        _, dims, dt = name.split(":")
+        n, d, h, w, c, o, k, st, pdd, phw = (int(v) for v in dims.split(","))
+        shape = synth.Conv3dShape(n, d, h, w, c, o, k, k, k, (st, st, st), (pdd, phw, phw), (1, 1, 1))
+        return f"conv3d {dt} NDHWC {shape.name()}", [Conv(shape, dt, "normal")], dt
     if name == "winograd_f32":
         return ("conv2d fp32 NHWC N=40 H=W=512 C=192->O=96 3x3 stride 1 pad 1 (Winograd, batch-tiled workspace)",
                 [Conv(synth.WINOGRAD_F32, "f32", "uniform")], "f32")

@@ -68,27 +68,52 @@ wino_gemm_f32_kernel(const WgArgs p) {
   float* __restrict__ D = p.d + bz * p.d_batch;
   const int ktiles = (p.c + BK - 1) / BK;
 
+  // Per-thread copy descriptors, fixed across k-tiles (only the k offset moves).
+  constexpr int A_PER = (A_CHUNKS + THREADS - 1) / THREADS;
+  constexpr int B_PER = (B_CHUNKS + THREADS - 1) / THREADS;
+  static_assert(!A_TMAJOR || A_CHUNKS % THREADS == 0, "A copies");
+  // A tile-major: copy i moves row (tid >> 2) + 32 i, chunk tid & 3.
+  const int a_chunk = tid & 3;
+  const int a_row0 = tid >> 2;
+  const float* a_src0 = A + (t0 + a_row0) * p.lda + a_chunk * 4;
+  const long long a_step = 32 * p.lda;
+  const uint32_t a_dst0 = (uint32_t)__cvta_generic_to_shared(As) +
+                          (uint32_t)(a_row0 * BK + ((a_chunk ^ ((a_row0 >> 2) & 3)) * 4)) * 4u;
+  unsigned a_valid = 0;
+#pragma unroll
+  for (int i = 0; i < A_PER; ++i)
+    if (t0 + a_row0 + 32 * i < p.t) a_valid |= 1u << i;
+  int b_off[B_PER], b_k[B_PER], b_bytes[B_PER];
+  uint32_t b_dst[B_PER];
+#pragma unroll
+  for (int i = 0; i < B_PER; ++i) {
+    const int q = tid + i * THREADS;
+    const int k = q / (BN / 4), col = (q % (BN / 4)) * 4;
+    const int oo = o0 + col;
+    b_k[i] = q < B_CHUNKS ? k : BK;          // BK: never copies
+    b_off[i] = (int)(k * p.ldb) + oo;
+    b_bytes[i] = oo < p.o ? min(16, (p.o - oo) * 4) : 0;
+    b_dst[i] = (uint32_t)__cvta_generic_to_shared(Bs) + (uint32_t)(k * BN + col) * 4u;
+  }
+
   auto load_stage = [&](int stage, int kt) {
     const int c0 = kt * BK;
-    float* as = As + stage * BK * BM;
-    float* bs = Bs + stage * BK * BN;
+    if (A_TMAJOR) {
+      const int cc = c0 + a_chunk * 4;
+      const int cbytes = cc < p.c ? min(16, (p.c - cc) * 4) : 0;
+      const uint32_t dst = a_dst0 + (uint32_t)(stage * BK * BM) * 4u;
 #pragma unroll
-    for (int i = 0; i < (A_CHUNKS + THREADS - 1) / THREADS; ++i) {
-      const int q = tid + i * THREADS;
-      if (q < A_CHUNKS) {
-        if (A_TMAJOR) {
-          const int row = q / (BK / 4), chunk = q % (BK / 4);
-          const long long tt = t0 + row;
-          const int cc = c0 + chunk * 4;
-          int bytes = 0;
-          const float* src = A;
-          if (tt < p.t && cc < p.c) {
-            bytes = min(16, (p.c - cc) * 4);
-            src = A + tt * p.lda + cc;
-          }
-          const int sw = chunk ^ ((row >> 2) & 3);
-          cp_async16((uint32_t)__cvta_generic_to_shared(as + row * BK + sw * 4), src, bytes);
-        } else {
+      for (int i = 0; i < A_PER; ++i) {
+        const int bytes = (a_valid >> i) & 1 ? cbytes : 0;
+        const float* src = bytes ? a_src0 + c0 + i * a_step : A;
+        cp_async16(dst + (uint32_t)(i * 32 * BK) * 4u, src, bytes);
+      }
+    } else {
+      float* as = As + stage * BK * BM;
+#pragma unroll
+      for (int i = 0; i < (A_CHUNKS + THREADS - 1) / THREADS; ++i) {
+        const int q = tid + i * THREADS;
+        if (q < A_CHUNKS) {
           const int k = q / (BM / 4), col = (q % (BM / 4)) * 4;
           const long long tt = t0 + col;
           int bytes = 0;
@@ -101,19 +126,13 @@ wino_gemm_f32_kernel(const WgArgs p) {
         }
       }
     }
+    const float* bbase = B + (long long)c0 * p.ldb;
+    const uint32_t bstage = (uint32_t)(stage * BK * BN) * 4u;
 #pragma unroll
-    for (int i = 0; i < (B_CHUNKS + THREADS - 1) / THREADS; ++i) {
-      const int q = tid + i * THREADS;
-      if (q < B_CHUNKS) {
-        const int k = q / (BN / 4), col = (q % (BN / 4)) * 4;
-        const int oo = o0 + col;
-        int bytes = 0;
-        const float* src = B;
-        if (c0 + k < p.c && oo < p.o) {
-          bytes = min(16, (p.o - oo) * 4);
-          src = B + (long long)(c0 + k) * p.ldb + oo;
-        }
-        cp_async16((uint32_t)__cvta_generic_to_shared(bs + k * BN + col), src, bytes);
+    for (int i = 0; i < B_PER; ++i) {
+      if (b_k[i] < BK) {
+        const int bytes = c0 + b_k[i] < p.c ? b_bytes[i] : 0;
+        cp_async16(b_dst[i] + bstage, bytes ? bbase + b_off[i] : B, bytes);
       }
     }
   };

@@ -172,15 +172,19 @@ wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __re
     Wino<M>::at(tt[i], res);
     const int y = ty * M + i;
     if (y >= a.oh) continue;
+    Tout* rp = op + (long long)y * a.ow * a.o;
+    if (a.accumulate) {
+      // the row's old values first, so the loads are not ordered behind the stores
+      float old[M];
+#pragma unroll
+      for (int j = 0; j < M; ++j) old[j] = tx * M + j < a.ow ? Store<Tout>::to_f32(rp[(long long)(tx * M + j) * a.o]) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < M; ++j) res[j] = old[j] + Store<Tout>::to_f32(Store<Tout>::from_f32(res[j]));
+    }
 #pragma unroll
     for (int j = 0; j < M; ++j) {
       const int xo = tx * M + j;
-      if (xo < a.ow) {
-        Tout* p = op + ((long long)y * a.ow + xo) * a.o;
-        float val = res[j];
-        if (a.accumulate) val = Store<Tout>::to_f32(*p) + Store<Tout>::to_f32(Store<Tout>::from_f32(val));
-        *p = Store<Tout>::from_f32(val);
-      }
+      if (xo < a.ow) rp[(long long)xo * a.o] = Store<Tout>::from_f32(res[j]);
     }
   }
 }
