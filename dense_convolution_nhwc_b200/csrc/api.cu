@@ -377,6 +377,9 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
 conv_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CONV_OK : CONV_ERR_CUDA; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+// The workspace's sub-buffers sit at 256-byte offsets from its base and are
+// read by TMA and 16-byte copies, so the base itself must be 256-byte aligned.
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
 
 // Run one planned 2D conv.  ws holds at least s.ws bytes.  accumulate: add the
 // result into out (out = round(out + round(result))), the depth-tap sum fused
@@ -828,6 +831,7 @@ conv_status_t conv2d_forward(const void* in, const void* w, void* out, const con
       overlaps(out, out_bytes, w, (size_t)g.o * g.w_row_stride * esz))
     return CONV_ERR_INVALID;
   if (workspace_bytes < s.ws || (s.ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
+  if (s.ws > 0 && !aligned256(workspace)) return CONV_ERR_ALIGNMENT;
   if (overlaps(out, out_bytes, workspace, s.ws)) return CONV_ERR_INVALID;
   return run2d(in, w, out, g, dtype, s, workspace, *d, static_cast<cudaStream_t>(stream));
 }
@@ -906,6 +910,7 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
   if (desc->n == 0) return CONV_OK;
   if (!in || !w || !out) return CONV_ERR_INVALID;
   if (workspace_bytes < ws || (ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
+  if (ws > 0 && !aligned256(workspace)) return CONV_ERR_ALIGNMENT;
   const int esz = dtype_size(dtype);
   const long long frame_in = (long long)desc->h * desc->w * desc->c;
   const long long frame_out = (long long)g2.oh * g2.ow * g2.o;

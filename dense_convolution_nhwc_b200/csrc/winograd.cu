@@ -71,7 +71,11 @@ struct WinoInArgs {
   long long t_stride;     // row count of V's planes (the workspace's tile capacity)
 };
 
-template <int M, typename Tin, typename Tst>
+// Idx is the type of the offsets inside one image and one V plane set: int
+// when the host has checked that they fit (fewer address instructions per
+// element), long long otherwise.  Tiles wholly inside the image skip the
+// bounds tests.
+template <int M, typename Tin, typename Tst, typename Idx>
 __global__ void __launch_bounds__(256)
 wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restrict__ v) {
   constexpr int A = Wino<M>::A;
@@ -89,17 +93,28 @@ wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restric
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
   const int y0 = ty * M - a.ph, x0 = tx * M - a.pw;
   const Tin* base = in + (long long)(a.n0 + nl) * a.in_img_stride + c;
+  const Idx cs = a.c, wc = (Idx)a.w * a.c;
 
   float d[A][A];
+  if (y0 >= 0 && x0 >= 0 && y0 + A <= a.h && x0 + A <= a.w) {
+    const Tin* p = base + ((Idx)y0 * wc + (Idx)x0 * cs);
 #pragma unroll
-  for (int i = 0; i < A; ++i) {
-    const int y = y0 + i;
-    const bool yok = y >= 0 && y < a.h;
+    for (int i = 0; i < A; ++i)
 #pragma unroll
-    for (int j = 0; j < A; ++j) {
-      const int x = x0 + j;
-      d[i][j] = (yok && x >= 0 && x < a.w)
-                    ? Store<Tin>::to_f32(base[((long long)y * a.w + x) * a.c]) : 0.0f;
+      for (int j = 0; j < A; ++j) d[i][j] = Store<Tin>::to_f32(p[(Idx)i * wc + (Idx)j * cs]);
+  } else {
+    unsigned xm = 0;
+#pragma unroll
+    for (int j = 0; j < A; ++j)
+      if (x0 + j >= 0 && x0 + j < a.w) xm |= 1u << j;
+#pragma unroll
+    for (int i = 0; i < A; ++i) {
+      const int y = y0 + i;
+      const bool yok = y >= 0 && y < a.h;
+      const Idx ro = yok ? (Idx)y * wc + (Idx)x0 * cs : (Idx)0;
+#pragma unroll
+      for (int j = 0; j < A; ++j)
+        d[i][j] = (yok && ((xm >> j) & 1u)) ? Store<Tin>::to_f32(base[ro + (Idx)j * cs]) : 0.0f;
     }
   }
   // columns: t = B^T d, then rows: V = t B
@@ -113,14 +128,14 @@ wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restric
 #pragma unroll
     for (int i = 0; i < A; ++i) tt[i][j] = res[i];
   }
-  const long long plane = a.t_stride * a.c;
+  const Idx plane = (Idx)(a.t_stride * a.c);
   Tst* vp = v + t * a.c + c;
 #pragma unroll
   for (int i = 0; i < A; ++i) {
     float res[A];
     Wino<M>::bt(tt[i], res);
 #pragma unroll
-    for (int j = 0; j < A; ++j) vp[(long long)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
+    for (int j = 0; j < A; ++j) vp[(Idx)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
   }
 }
 
@@ -135,7 +150,7 @@ struct WinoOutArgs {
   int accumulate;
 };
 
-template <int M, typename Tout>
+template <int M, typename Tout, typename Idx>
 __global__ void __launch_bounds__(256)
 wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
   constexpr int A = Wino<M>::A;
@@ -147,13 +162,13 @@ wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __re
   const int r = (int)(t - (long long)nl * per_img);
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
 
-  const long long plane = a.t_stride * a.o;
+  const Idx plane = (Idx)(a.t_stride * a.o);
   const float* mp = mb + t * a.o + o;
   float x[A][A];
 #pragma unroll
   for (int i = 0; i < A; ++i)
 #pragma unroll
-    for (int j = 0; j < A; ++j) x[i][j] = __ldg(mp + (long long)(i * A + j) * plane);
+    for (int j = 0; j < A; ++j) x[i][j] = __ldg(mp + (Idx)(i * A + j) * plane);
   // columns: t = A^T x (M x A), then rows: y = t A (M x M)
   float tt[M][A];
 #pragma unroll
@@ -166,26 +181,27 @@ wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __re
     for (int i = 0; i < M; ++i) tt[i][j] = res[i];
   }
   Tout* op = out + (long long)(a.n0 + nl) * a.out_img_stride + o;
+  const Idx os = a.o, wo = (Idx)a.ow * a.o;
+  const bool whole = ty * M + M <= a.oh && tx * M + M <= a.ow;
 #pragma unroll
   for (int i = 0; i < M; ++i) {
     float res[M];
     Wino<M>::at(tt[i], res);
     const int y = ty * M + i;
-    if (y >= a.oh) continue;
-    Tout* rp = op + (long long)y * a.ow * a.o;
+    if (!whole && y >= a.oh) continue;
+    Tout* rp = op + ((Idx)y * wo + (Idx)(tx * M) * os);
     if (a.accumulate) {
       // the row's old values first, so the loads are not ordered behind the stores
       float old[M];
 #pragma unroll
-      for (int j = 0; j < M; ++j) old[j] = tx * M + j < a.ow ? Store<Tout>::to_f32(rp[(long long)(tx * M + j) * a.o]) : 0.0f;
+      for (int j = 0; j < M; ++j)
+        old[j] = (whole || tx * M + j < a.ow) ? Store<Tout>::to_f32(rp[(Idx)j * os]) : 0.0f;
 #pragma unroll
       for (int j = 0; j < M; ++j) res[j] = old[j] + Store<Tout>::to_f32(Store<Tout>::from_f32(res[j]));
     }
 #pragma unroll
-    for (int j = 0; j < M; ++j) {
-      const int xo = tx * M + j;
-      if (xo < a.ow) rp[(long long)xo * a.o] = Store<Tout>::from_f32(res[j]);
-    }
+    for (int j = 0; j < M; ++j)
+      if (whole || tx * M + j < a.ow) rp[(Idx)j * os] = Store<Tout>::from_f32(res[j]);
   }
 }
 
@@ -369,14 +385,22 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   const long long blocks = ((a.t_count + block.y - 1) / block.y) * ((g.c + bx - 1) / bx);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)blocks);
+  // 32-bit offsets when one image (with a row of slack for the padding) and the
+  // whole V plane set stay below 2^31 elements
+  const int a2 = (m + 2) * (m + 2);
+  const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31) && (long long)a2 * t_tile * g.c < (1LL << 31);
   return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
       return wino_by_dt(store_dt, [&](auto ts) {
         using Tst = decltype(ts);
-        wino_input_kernel<M, Tin, Tst><<<grid, block, 0, s>>>(static_cast<const Tin*>(in), a,
-                                                              static_cast<Tst*>(v));
+        if (idx32)
+          wino_input_kernel<M, Tin, Tst, int><<<grid, block, 0, s>>>(static_cast<const Tin*>(in), a,
+                                                                     static_cast<Tst*>(v));
+        else
+          wino_input_kernel<M, Tin, Tst, long long><<<grid, block, 0, s>>>(static_cast<const Tin*>(in), a,
+                                                                           static_cast<Tst*>(v));
         return cudaGetLastError();
       });
     });
@@ -443,11 +467,16 @@ cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb,
   dim3 block(bx, 256 / bx);
   dim3 grid((unsigned)((a.t_count + block.y - 1) / block.y), (g.o + bx - 1) / bx);
   if (grid.y > 65535) return cudaErrorInvalidValue;
+  const int a2 = (m + 2) * (m + 2);
+  const bool idx32 = g.out_img_stride < (1LL << 31) && (long long)a2 * t_tile * g.o < (1LL << 31);
   return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(out_dt, [&](auto to) {
       using Tout = decltype(to);
-      wino_output_kernel<M, Tout><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
+      if (idx32)
+        wino_output_kernel<M, Tout, int><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
+      else
+        wino_output_kernel<M, Tout, long long><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
       return cudaGetLastError();
     });
   });

@@ -118,7 +118,9 @@ struct Wino3InArgs {
   long long t_stride;        // rows of each V plane
 };
 
-template <int M, typename Tin, typename Tst>
+// Idx: the offset type inside one image and one V plane set (int when the host
+// has checked that they fit, long long otherwise).
+template <int M, typename Tin, typename Tst, typename Idx>
 __global__ void __launch_bounds__(32 * (M + 2))
 wino3d_input_kernel(const Tin* __restrict__ in, const Wino3InArgs a, Tst* __restrict__ v) {
   constexpr int A = Wino<M>::A;
@@ -135,16 +137,27 @@ wino3d_input_kernel(const Tin* __restrict__ in, const Wino3InArgs a, Tst* __rest
   const Tin* base = in + (long long)ti.n * a.in_img_stride + (long long)x * a.c + c;
 
   // Slice x = j: depth then height transforms of its alpha x alpha values.
+  const Idx wc = (Idx)a.w * a.c, hwc = (Idx)a.h * wc;
   float d[A][A];
+  if (xok && z0 >= 0 && y0 >= 0 && z0 + A <= a.d && y0 + A <= a.h) {
+    const Tin* p = base + ((Idx)z0 * hwc + (Idx)y0 * wc);
 #pragma unroll
-  for (int zz = 0; zz < A; ++zz) {
-    const int z = z0 + zz;
-    const bool zok = xok && z >= 0 && z < a.d;
+    for (int zz = 0; zz < A; ++zz)
 #pragma unroll
-    for (int yy = 0; yy < A; ++yy) {
-      const int y = y0 + yy;
-      d[zz][yy] = (zok && y >= 0 && y < a.h)
-                      ? Store<Tin>::to_f32(base[((long long)z * a.h + y) * a.w * a.c]) : 0.0f;
+      for (int yy = 0; yy < A; ++yy) d[zz][yy] = Store<Tin>::to_f32(p[(Idx)zz * hwc + (Idx)yy * wc]);
+  } else {
+    unsigned ym = 0;
+#pragma unroll
+    for (int yy = 0; yy < A; ++yy)
+      if (y0 + yy >= 0 && y0 + yy < a.h) ym |= 1u << yy;
+#pragma unroll
+    for (int zz = 0; zz < A; ++zz) {
+      const int z = z0 + zz;
+      const bool zok = xok && z >= 0 && z < a.d;
+      const Idx ro = zok ? (Idx)z * hwc + (Idx)y0 * wc : (Idx)0;
+#pragma unroll
+      for (int yy = 0; yy < A; ++yy)
+        d[zz][yy] = (zok && ((ym >> yy) & 1u)) ? Store<Tin>::to_f32(base[ro + (Idx)yy * wc]) : 0.0f;
     }
   }
   float tz[A][A];     // [xi_z][y]
@@ -168,8 +181,8 @@ wino3d_input_kernel(const Tin* __restrict__ in, const Wino3InArgs a, Tst* __rest
 
   // Width transform of lines l = j, j + A, ... (all A*A (xi_z, xi_y) lines).
   if (!cok) return;
-  const long long plane = a.t_stride * a.c;
-  Tst* vp = v + t * a.c + c;
+  const Idx plane = (Idx)(a.t_stride * a.c);
+  Tst* vp = v + t * a.c + c + (long long)(j * A) * (a.t_stride * a.c);
 #pragma unroll
   for (int k = 0; k < A; ++k) {
     const int l = j + k * A;
@@ -178,7 +191,7 @@ wino3d_input_kernel(const Tin* __restrict__ in, const Wino3InArgs a, Tst* __rest
     for (int xx = 0; xx < A; ++xx) row[xx] = sm[l][xx][lane];
     Wino<M>::bt(row, r);
 #pragma unroll
-    for (int xx = 0; xx < A; ++xx) vp[(long long)(l * A + xx) * plane] = Store<Tst>::from_f32(r[xx]);
+    for (int xx = 0; xx < A; ++xx) vp[(Idx)(k * A * A + xx) * plane] = Store<Tst>::from_f32(r[xx]);
   }
 }
 
@@ -192,7 +205,7 @@ struct Wino3OutArgs {
   long long u0, t_count, t_stride;
 };
 
-template <int M, typename Tout>
+template <int M, typename Tout, typename Idx>
 __global__ void __launch_bounds__(32 * (M + 2))
 wino3d_output_kernel(const float* __restrict__ mb, const Wino3OutArgs a, Tout* __restrict__ out) {
   constexpr int A = Wino<M>::A;
@@ -205,13 +218,13 @@ wino3d_output_kernel(const float* __restrict__ mb, const Wino3OutArgs a, Tout* _
   const bool ook = o < a.o;
 
   // Slice xi_x = j: depth then height transforms.
-  const long long plane = a.t_stride * a.o;
-  const float* mp = mb + t * a.o + o;
+  const Idx plane = (Idx)(a.t_stride * a.o);
+  const float* mp = mb + t * a.o + o + (long long)j * (a.t_stride * a.o);
   float x[A][A];      // [xi_z][xi_y]
 #pragma unroll
   for (int zz = 0; zz < A; ++zz)
 #pragma unroll
-    for (int yy = 0; yy < A; ++yy) x[zz][yy] = ook ? __ldg(mp + (long long)((zz * A + yy) * A + j) * plane) : 0.0f;
+    for (int yy = 0; yy < A; ++yy) x[zz][yy] = ook ? __ldg(mp + (Idx)((zz * A + yy) * A) * plane) : 0.0f;
   float tz[M][A];     // [oz][xi_y]
 #pragma unroll
   for (int yy = 0; yy < A; ++yy) {
@@ -234,6 +247,8 @@ wino3d_output_kernel(const float* __restrict__ mb, const Wino3OutArgs a, Tout* _
   if (!ook) return;
   const TileIdx ti = tile_of(a.u0, t, a.tiles_d, a.tiles_h, a.tiles_w);
   Tout* op = out + (long long)ti.n * a.out_img_stride + o;
+  const Idx os = a.o, wo = (Idx)a.ow * a.o;
+  const bool xwhole = ti.tx * M + M <= a.ow;
   for (int l = j; l < M * M; l += A) {
     const int z = ti.tz * M + l / M, y = ti.ty * M + l % M;
     if (z >= a.od || y >= a.oh) continue;
@@ -241,12 +256,10 @@ wino3d_output_kernel(const float* __restrict__ mb, const Wino3OutArgs a, Tout* _
 #pragma unroll
     for (int xx = 0; xx < A; ++xx) row[xx] = sm[l][xx][lane];
     Wino<M>::at(row, r);
-    Tout* rp = op + ((long long)z * a.oh + y) * a.ow * a.o;
+    Tout* rp = op + (((Idx)z * a.oh + y) * wo + (Idx)(ti.tx * M) * os);
 #pragma unroll
-    for (int xx = 0; xx < M; ++xx) {
-      const int xo = ti.tx * M + xx;
-      if (xo < a.ow) rp[(long long)xo * a.o] = Store<Tout>::from_f32(r[xx]);
-    }
+    for (int xx = 0; xx < M; ++xx)
+      if (xwhole || ti.tx * M + xx < a.ow) rp[(Idx)xx * os] = Store<Tout>::from_f32(r[xx]);
   }
 }
 
@@ -302,14 +315,22 @@ cudaError_t launch_wino3d_input(const void* in, const Geom3& g, long long u0, lo
   if (a.t_count == 0) return cudaSuccess;
   const long long blocks = a.t_count * ((g.c + 31) / 32);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // 32-bit offsets when one image (with slack for the padding) and the whole V
+  // plane set stay below 2^31 elements
+  const long long a3 = (long long)(m + 2) * (m + 2) * (m + 2);
+  const bool idx32 = a.in_img_stride + 4LL * g.w * g.c < (1LL << 31) && a3 * t_stride * g.c < (1LL << 31);
   return by_m3(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(in_dt, [&](auto ti) {
       using Tin = decltype(ti);
       return wino_by_dt(store_dt, [&](auto ts) {
         using Tst = decltype(ts);
-        wino3d_input_kernel<M, Tin, Tst><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(static_cast<const Tin*>(in), a,
-                                                                                   static_cast<Tst*>(v));
+        if (idx32)
+          wino3d_input_kernel<M, Tin, Tst, int><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(
+              static_cast<const Tin*>(in), a, static_cast<Tst*>(v));
+        else
+          wino3d_input_kernel<M, Tin, Tst, long long><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(
+              static_cast<const Tin*>(in), a, static_cast<Tst*>(v));
         return cudaGetLastError();
       });
     });
@@ -330,11 +351,18 @@ cudaError_t launch_wino3d_output(const float* mbuf, const Geom3& g, long long u0
   if (a.t_count == 0) return cudaSuccess;
   const long long blocks = a.t_count * ((g.o + 31) / 32);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long a3 = (long long)(m + 2) * (m + 2) * (m + 2);
+  const bool idx32 = a.out_img_stride < (1LL << 31) && a3 * t_stride * g.o < (1LL << 31);
   return by_m3(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(out_dt, [&](auto to) {
       using Tout = decltype(to);
-      wino3d_output_kernel<M, Tout><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(mbuf, a, static_cast<Tout*>(out));
+      if (idx32)
+        wino3d_output_kernel<M, Tout, int><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(mbuf, a,
+                                                                                     static_cast<Tout*>(out));
+      else
+        wino3d_output_kernel<M, Tout, long long><<<(unsigned)blocks, 32 * (M + 2), 0, s>>>(mbuf, a,
+                                                                                           static_cast<Tout*>(out));
       return cudaGetLastError();
     });
   });

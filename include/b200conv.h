@@ -68,7 +68,8 @@ typedef enum {
     CONV_OK = 0,
     CONV_ERR_INVALID = 1,      /* bad shape, pointer, overlap or argument */
     CONV_ERR_UNSUPPORTED = 2,  /* forced algorithm cannot run this shape */
-    CONV_ERR_ALIGNMENT = 3,    /* reserved: misaligned pointers take the direct path instead */
+    CONV_ERR_ALIGNMENT = 3,    /* a workspace that is not 256-byte aligned; nothing was launched
+                                  (misaligned in / w / out take the any-alignment path instead) */
     CONV_ERR_WORKSPACE = 4,    /* workspace smaller than the plan needs; nothing was launched */
     CONV_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
     CONV_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out (reported by conv_check) */
@@ -168,6 +169,8 @@ B200CONV_API size_t conv2d_workspace_size(const conv2d_desc_t *desc, conv_dtype_
  * all of `dtype`, on the current CUDA device.  workspace may be NULL when the
  * plan needs 0 bytes; a workspace_bytes smaller than the plan's is
  * CONV_ERR_WORKSPACE and launches nothing (never a partial or zeroed result).
+ * A non-empty workspace must start on a 256-byte boundary (cudaMalloc and
+ * torch allocations do), else CONV_ERR_ALIGNMENT and nothing is launched.
  */
 B200CONV_API conv_status_t conv2d_forward(const void *in, const void *w, void *out,
                              const conv2d_desc_t *desc, conv_dtype_t dtype,

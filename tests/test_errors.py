@@ -45,6 +45,36 @@ def test_undersized_workspace_is_refused_and_nothing_runs():
     assert st == 4
 
 
+def test_misaligned_workspace_is_refused_and_nothing_runs():
+    """A workspace base off a 256-byte boundary is CONV_ERR_ALIGNMENT before any
+    launch, for conv2d (Winograd and split-K plans) and conv3d (3D Winograd)."""
+    x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
+    for opts in (B.make_options("winograd"), None):
+        shape = S if opts else synth.Conv2dShape(8, 14, 14, 512, 512, 3, 3, (2, 2), (1, 1), (1, 1))   # split-K
+        xx, ww = (x, w) if opts else synth.conv2d_inputs(shape, "f32", "normal", 0, device="cuda")
+        need = B.conv2d_workspace_size(desc(shape), 0, 0, opts)
+        assert need > 0
+        ws = torch.empty(need + 512, dtype=torch.uint8, device="cuda")
+        out = torch.full((shape.n, shape.oh, shape.ow, shape.o), float("nan"), device="cuda")
+        st = B.conv2d_forward(xx.data_ptr(), ww.data_ptr(), out.data_ptr(), desc(shape), 0, opts, ws.data_ptr() + 16,
+                              need, stream())
+        assert st == 3       # CONV_ERR_ALIGNMENT
+        torch.cuda.synchronize()
+        assert torch.isnan(out).all()
+    s3 = synth.Conv3dShape(1, 6, 8, 8, 128, 128, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    x3, w3 = synth.conv3d_inputs(s3, "f32", "normal", 0, device="cuda")
+    d3 = B.make_desc3d(s3.n, s3.d, s3.h, s3.w, s3.c, s3.o, s3.kd, s3.kh, s3.kw, s3.stride, s3.pad, s3.dilation)
+    need = B.conv3d_workspace_size(d3, 0, 0, None)
+    assert need > 0
+    ws = torch.empty(need + 512, dtype=torch.uint8, device="cuda")
+    out = torch.full((1, s3.od, s3.oh, s3.ow, s3.o), float("nan"), device="cuda")
+    st = B.conv3d_forward(x3.data_ptr(), w3.data_ptr(), out.data_ptr(), d3, 0, None, ws.data_ptr() + 128, need,
+                          stream())
+    assert st == 3
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all()
+
+
 def test_overlapping_output_is_refused():
     x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
     st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), x.data_ptr(), desc(S), 0, None, 0, 0, stream())
