@@ -186,12 +186,12 @@ def kernel_bound(name):
 
 KERNEL_SOURCES = {
     "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["wino_gemm_f32.cu"],
-    "tc_conv": ["tc_conv.cu", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "common.cuh"],
-    "tc_conv3d": ["tc_conv.cu", "common.cuh"],
+    "tc_conv": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
+    "tc_conv3d": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "wino_input": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino_output": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino_filter": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
-    "wino3d_gemm_simt": ["wino_gemm_f32.cu"], "wino3d_gemm_tc": ["tc_conv.cu", "common.cuh"],
+    "wino3d_gemm_simt": ["wino_gemm_f32.cu"], "wino3d_gemm_tc": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "wino3d_input": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino3d_output": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino3d_filter": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
