@@ -12,8 +12,9 @@
 //
 // Tiling: 128 x BN output tile per 256-thread block, 16-wide k chunks staged
 // through double-buffered shared memory (transposed, k-major), 8 x BN/16
-// outputs per thread.  k chunks never straddle a filter tap, so each A row
-// resolves its input pixel once per tap.
+// outputs per thread, multiplied as packed fp32 FMAs on column pairs (two
+// lanes per instruction, each exactly fmaf).  k chunks never straddle a
+// filter tap, so each A row resolves its input pixel once per tap.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -163,11 +164,12 @@ simt_conv_kernel(const SimtArgs a) {
     }
   };
 
-  float acc[8][TN];
+  // column pairs for the packed fp32 FMA (each lane exactly fmaf)
+  float2 acc[8][TN / 2];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < TN / 2; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
   if (steps > 0) load_tiles(0);
   else ra[0][0] = ra[0][1] = ra[0][2] = ra[0][3] = ra[1][0] = ra[1][1] = ra[1][2] = ra[1][3] = 0.0f;
@@ -183,21 +185,21 @@ simt_conv_kernel(const SimtArgs a) {
     if (step + 1 < steps) load_tiles(step + 1);
 #pragma unroll
     for (int k = 0; k < BK; ++k) {
-      float av[8], bv[TN];
+      float av[8];
+      float2 bv[TN / 2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float2 t = *reinterpret_cast<const float2*>(&As[buf][k][32 * i + ty * 2]);
         av[2 * i] = t.x; av[2 * i + 1] = t.y;
       }
 #pragma unroll
-      for (int j = 0; j < TN / 2; ++j) {
-        float2 t = *reinterpret_cast<const float2*>(&Bs[buf][k][32 * j + tx * 2]);
-        bv[2 * j] = t.x; bv[2 * j + 1] = t.y;
+      for (int j = 0; j < TN / 2; ++j) bv[j] = *reinterpret_cast<const float2*>(&Bs[buf][k][32 * j + tx * 2]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 a2 = make_float2(av[i], av[i]);
+#pragma unroll
+        for (int j = 0; j < TN / 2; ++j) acc[i][j] = __ffma2_rn(a2, bv[j], acc[i][j]);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
     if (step + 1 < steps) store_tiles(buf ^ 1);
     __syncthreads();
@@ -213,7 +215,7 @@ simt_conv_kernel(const SimtArgs a) {
 #pragma unroll
       for (int j = 0; j < TN; ++j) {
         int o = n0 + 32 * (j >> 1) + tx * 2 + (j & 1);
-        if (o < a.o) prow[o] = acc[i][j];
+        if (o < a.o) prow[o] = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
       }
       continue;
     }
@@ -222,7 +224,7 @@ simt_conv_kernel(const SimtArgs a) {
     for (int j = 0; j < TN; ++j) {
       int o = n0 + 32 * (j >> 1) + tx * 2 + (j & 1);
       if (o < a.o) {
-        float v = acc[i][j];
+        float v = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
         if (a.accumulate) v = Store<T>::to_f32(orow[o]) + Store<T>::to_f32(Store<T>::from_f32(v));
         orow[o] = Store<T>::from_f32(v);
       }

@@ -12,9 +12,11 @@
 // 16-byte cp.async (zero-filled past T, C and O) in a 3-stage ring, with no
 // register staging and no transposes.  Each of the 128 threads owns an
 // 8 x BN/8 block of D and reads its operand fragments with 128-bit shared
-// loads.  Every output's reduction runs over c in ascending order inside one
-// thread, so the result does not depend on T (batch-tiled Winograd stays
-// bit-identical to untiled).
+// loads.  The products run as packed fp32 FMAs on column pairs (sm_100's
+// two-lane FMA; each lane is exactly fmaf), which halves the FMA issue slots
+// of a kernel that is otherwise issue-bound.  Every output's reduction runs
+// over c in ascending order inside one thread, so the result does not depend
+// on T (batch-tiled Winograd stays bit-identical to untiled).
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -137,11 +139,13 @@ wino_gemm_f32_kernel(const WgArgs p) {
     }
   };
 
-  float acc[8][TN];
+  // accumulators in column pairs: the packed fp32 FMA (two lanes per
+  // instruction, each lane exactly fmaf) halves the FMA issue slots
+  float2 acc[8][TN / 2];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < TN / 2; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
 
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
@@ -171,24 +175,27 @@ wino_gemm_f32_kernel(const WgArgs p) {
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int k = 4 * k4 + kq;
-          float bv[TN];
+          float2 bv[TN / 2];
 #pragma unroll
           for (int j = 0; j < TN / 4; ++j) {
             const float4 b = *reinterpret_cast<const float4*>(bs + k * BN + 32 * j + tc * 4);
-            bv[4 * j] = b.x; bv[4 * j + 1] = b.y; bv[4 * j + 2] = b.z; bv[4 * j + 3] = b.w;
+            bv[2 * j] = make_float2(b.x, b.y);
+            bv[2 * j + 1] = make_float2(b.z, b.w);
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float av = kq == 0 ? a4[i].x : kq == 1 ? a4[i].y : kq == 2 ? a4[i].z : a4[i].w;
+            const float2 a2 = make_float2(av, av);
 #pragma unroll
-            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av, bv[j], acc[i][j]);
+            for (int j = 0; j < TN / 2; ++j) acc[i][j] = __ffma2_rn(a2, bv[j], acc[i][j]);
           }
         }
       }
     } else {
 #pragma unroll
       for (int k = 0; k < BK; ++k) {
-        float av[8], bv[TN];
+        float av[8];
+        float2 bv[TN / 2];
         const float4 a0 = *reinterpret_cast<const float4*>(as + k * BM + tr * 4);
         const float4 a1 = *reinterpret_cast<const float4*>(as + k * BM + 64 + tr * 4);
         av[0] = a0.x; av[1] = a0.y; av[2] = a0.z; av[3] = a0.w;
@@ -196,12 +203,15 @@ wino_gemm_f32_kernel(const WgArgs p) {
 #pragma unroll
         for (int j = 0; j < TN / 4; ++j) {
           const float4 b = *reinterpret_cast<const float4*>(bs + k * BN + 32 * j + tc * 4);
-          bv[4 * j] = b.x; bv[4 * j + 1] = b.y; bv[4 * j + 2] = b.z; bv[4 * j + 3] = b.w;
+          bv[2 * j] = make_float2(b.x, b.y);
+          bv[2 * j + 1] = make_float2(b.z, b.w);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+          const float2 a2 = make_float2(av[i], av[i]);
 #pragma unroll
-          for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+          for (int j = 0; j < TN / 2; ++j) acc[i][j] = __ffma2_rn(a2, bv[j], acc[i][j]);
+        }
       }
     }
   }
@@ -217,13 +227,14 @@ wino_gemm_f32_kernel(const WgArgs p) {
 #pragma unroll
     for (int j = 0; j < TN / 4; ++j) {
       const int o = o0 + 32 * j + tc * 4;
+      const float4 v4 = make_float4(acc[i][2 * j].x, acc[i][2 * j].y, acc[i][2 * j + 1].x, acc[i][2 * j + 1].y);
       if (vec && o + 3 < p.o) {
-        *reinterpret_cast<float4*>(drow + o) =
-            make_float4(acc[i][4 * j], acc[i][4 * j + 1], acc[i][4 * j + 2], acc[i][4 * j + 3]);
+        *reinterpret_cast<float4*>(drow + o) = v4;
       } else {
+        const float ve[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (o + e < p.o) drow[o + e] = acc[i][4 * j + e];
+          if (o + e < p.o) drow[o + e] = ve[e];
       }
     }
   }
