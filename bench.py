@@ -165,8 +165,9 @@ def kernel_work(conv, plan):
         add("wino_filter", 0.0, w_b + a2 * s.o * s.c * st)
         add("wino_input", 0.0, in_b + a2 * T * s.c * st)
         gk = "wino_gemm_tc" if plan["engine"] == "tcgen05" else "wino_gemm_simt"
-        add(gk, 2.0 * a2 * T * s.c * s.o, a2 * T * (s.c * st + s.o * 4))
-        add("wino_output", 0.0, a2 * T * s.o * 4 + out_b)
+        # M is fp32 on the FFMA path and in the 16-bit operand type on the tensor-core path
+        add(gk, 2.0 * a2 * T * s.c * s.o, a2 * T * (s.c * st + s.o * st))
+        add("wino_output", 0.0, a2 * T * s.o * st + out_b)
     else:
         k = "tc_conv" if plan["engine"] == "tcgen05" else "simt_conv"
         add(k, 2.0 * M * s.o * K, in_b + w_b + out_b)

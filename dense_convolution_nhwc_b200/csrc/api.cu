@@ -214,7 +214,8 @@ long long round4(long long x) { return (x + 3) & ~3LL; }
 constexpr bool kF32VTileMajor = B200CONV_F32_V_TILE_MAJOR != 0;
 
 // Workspace layout of the Winograd path for batch tiles of nb images.
-//   tensor-core GEMM (16-bit operands): U [a2][O][C], V [a2][T][C], M [a2][T][O] fp32
+//   tensor-core GEMM (16-bit operands): U [a2][O][C], V [a2][T][C], M [a2][T][O], all in the
+//                                       operand type (M accumulated in fp32, stored rounded)
 //   FFMA GEMM (fp32 operands):          U [a2][C][O4], V [a2][T][C] (tile-major) or
 //                                       [a2][C][T4] (channel-major), M [a2][T][O] fp32
 // (O4, T4 = O, T rounded up to 4 so rows start 16-byte aligned).
@@ -229,7 +230,7 @@ WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m
   const long long a2 = (long long)(m + 2) * (m + 2);
   L.tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
   const int esz = dtype_size(store);
-  L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * esz + (size_t)g.o * 4);
+  L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * esz + (size_t)g.o * (cmajor ? 4 : esz));
   const long long t = nb * L.tiles_per_img;
   if (cmajor) {
     L.u_bytes = align256((size_t)(a2 * g.c * round4(g.o)) * esz);
@@ -238,7 +239,7 @@ WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m
     L.u_bytes = align256((size_t)(a2 * g.o * g.c) * esz);
     L.v_bytes = align256((size_t)(a2 * t * g.c) * esz);
   }
-  L.m_bytes = align256((size_t)(a2 * t * g.o) * 4);
+  L.m_bytes = align256((size_t)(a2 * t * g.o) * (cmajor ? 4 : esz));
   return L;
 }
 
@@ -394,7 +395,8 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     uint8_t* base = static_cast<uint8_t*>(ws);
     void* u = base;
     void* v = base + L.u_bytes;
-    float* mb = reinterpret_cast<float*>(base + L.u_bytes + L.v_bytes);
+    void* mb = base + L.u_bytes + L.v_bytes;
+    const conv_dtype_t m_dt = cmajor ? CONV_F32 : s.wino_store;
     cudaError_t e;
     {
       ProfScope ps(K_WINO_FILTER, st);
@@ -416,17 +418,17 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
       if (cmajor) {
         ProfScope ps(K_WINO_GEMM_SIMT, st);
         const bool tmajor = kF32VTileMajor && g.c % 4 == 0;
-        e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), mb, a2, (int)t, g.c, g.o,
-                                 tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
+        e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), static_cast<float*>(mb),
+                                 a2, (int)t, g.c, g.o, tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
       } else {
-        BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb};
+        BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb, m_dt};
         ProfScope ps(K_WINO_GEMM_TC, st);
         e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
       }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
       {
         ProfScope ps(K_WINO_OUTPUT, st);
-        e = launch_wino_output(mb, g, n0, nbi, m, t, dt, out, accumulate, st);
+        e = launch_wino_output(mb, m_dt, g, n0, nbi, m, t, dt, out, accumulate, st);
       }
       if (e != cudaSuccess) return CONV_ERR_CUDA;
     }
@@ -740,7 +742,7 @@ conv_status_t run3d_winograd(const void* in, const void* w, void* out, const Geo
       e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), mb, a3, (int)t, g.c, g.o,
                                g.c, round4(g.o), true, st);
     } else {
-      BatchedGemm bg{a3, (int)t, g.c, g.o, v, u, mb};
+      BatchedGemm bg{a3, (int)t, g.c, g.o, v, u, mb, CONV_F32};
       ProfScope ps(K_WINO3D_GEMM_TC, st);
       e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
     }

@@ -44,11 +44,13 @@ struct Geom3 {
 
 // Batched GEMM view used by the Winograd path: for b < batches,
 //   D_b[t][o] = sum_c A_b[t][c] * B_b[o][c]   (A: [batches][T][C], B: [batches][O][C])
+// accumulated in fp32 and stored in d_dt (fp32, or the 16-bit operand type).
 struct BatchedGemm {
   int batches, t, c, o;
   const void* a;        // [batches][T][C] in the input dtype (fp32 for the SIMT engine)
   const void* b;        // [batches][O][C]
-  float* d;             // [batches][T][O] fp32
+  void* d;              // [batches][T][O] in d_dt
+  conv_dtype_t d_dt;
 };
 
 // ---- kernel launchers (return a CUDA error; never synchronise) ----
@@ -64,8 +66,6 @@ cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geo
 // out[i] = round(out[i] + round(sum)), for i < count.
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count, void* out, conv_dtype_t dt,
                                  bool accumulate, cudaStream_t s);
-// SIMT batched GEMM on fp32 operands (Winograd fp32 path).
-cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s);
 
 // tcgen05 implicit GEMM for 16-bit dtypes (TMA im2col staging, TMEM accumulators).
 // Returns cudaErrorNotSupported if the shape cannot be encoded as TMA maps.
@@ -103,7 +103,8 @@ cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int 
 cudaError_t launch_wino_gemm_f32(const float* a, const float* b, float* d, int batches, int t, int c, int o,
                                  long long lda, long long ldb, bool a_tmajor, cudaStream_t s);
 int wino_gemm_f32_tile_n(int o);
-cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb, int m,
+// M [a2][t_tile][O] in m_dt (fp32, or the 16-bit operand type of the tensor-core path).
+cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, int nb, int m,
                                long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
                                cudaStream_t s);
 

@@ -281,27 +281,5 @@ cudaError_t launch_simt_conv(const void* in, const void* w, void* out, const Geo
   return vec ? launch_dt<true>(a, dt, a.ksplit, s) : launch_dt<false>(a, dt, a.ksplit, s);
 }
 
-cudaError_t launch_simt_batched_gemm(const BatchedGemm& bg, cudaStream_t s) {
-  // Each batch is a 1x1 "convolution" of a 1 x T image with C channels.
-  SimtArgs a{};
-  a.in = bg.a; a.w = bg.b; a.out = bg.d;
-  a.h = 1; a.w_ = bg.t; a.c = bg.c; a.o = bg.o; a.kh = 1; a.kw = 1;
-  a.sh = a.sw = 1; a.ph = a.pw = 0; a.dh = a.dw = 1;
-  a.oh = 1; a.ow = bg.t;
-  a.m = bg.t;
-  a.in_img_stride = (long long)bg.t * bg.c;
-  a.w_row_stride = bg.c;
-  a.a_batch = (long long)bg.t * bg.c;
-  a.b_batch = (long long)bg.o * bg.c;
-  a.d_batch = (long long)bg.t * bg.o;
-  a.accumulate = 0;
-  a.ksplit = 1;
-  a.partial = nullptr;
-  if (a.m == 0 || bg.batches == 0) return cudaSuccess;
-  bool vec = (bg.c % 4 == 0) && ((reinterpret_cast<uintptr_t>(bg.a) & 15) == 0) &&
-             ((reinterpret_cast<uintptr_t>(bg.b) & 15) == 0);
-  return vec ? launch_typed<float, true>(a, bg.batches, s)
-             : launch_typed<float, false>(a, bg.batches, s);
-}
 
 }  // namespace b200conv

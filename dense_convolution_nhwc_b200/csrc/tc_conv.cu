@@ -56,12 +56,12 @@ template <int BN> struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
-  // fp32-output variants stage each epilogue warp's 32 x 32 chunk for a TMA
-  // store: 4 warps x 2 buffers x 4 KB, 128-byte swizzled
-  static constexpr int STORE_BYTES = 4 * 2 * 32 * 32 * 4;
+  // The epilogue stages each warp's output chunk for a TMA store: 32 rows of
+  // 128 bytes (32 fp32 or 64 16-bit columns), 4 warps x 2 buffers, 128-byte swizzled
+  static constexpr int STORE_BYTES = 4 * 2 * 32 * 128;
   template <typename TOut>
   static constexpr int smem() {
-    return 1024 + STAGES * STAGE_BYTES + (sizeof(TOut) == 4 ? STORE_BYTES : 0) + BAR_BYTES;
+    return 1024 + STAGES * STAGE_BYTES + STORE_BYTES + BAR_BYTES;
   }
 };
 
@@ -78,7 +78,7 @@ struct TcArgs {
   long long out_batch;         // elements between batches
   int accumulate;              // out = round(out + round(acc)) instead of out = round(acc)
   int ksplit;                  // conv modes: > 1 splits the K range, the split index in the batch slot
-  int tma_store;               // fp32 output: write 32 x 32 chunks with TMA stores through tmD
+  int tma_store;               // write 32-row x 128-byte chunks with TMA stores through tmD
   int* err;
 };
 
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const TcArgs a) {
   using C = Cfg<BN>;
-  constexpr int STORE_BYTES = sizeof(TOut) == 4 ? C::STORE_BYTES : 0;
+  constexpr int STORE_BYTES = C::STORE_BYTES;
   constexpr uint32_t IDESC = make_idesc<BN>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
 
   extern __shared__ uint8_t smem_raw[];
@@ -325,6 +325,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
             continue;
           }
+        } else {
+          if (a.tma_store) {
+            // 16-bit: stage row `lane` of a 32 x 64 chunk (two 32-column groups, 128 bytes
+            // per row, 16-byte chunks XOR-swizzled by lane % 8), then one lane stores it
+#pragma unroll
+            for (int h = 0; h < EPI / 32; h += 2) {
+              const int c0 = n0 + cg + 32 * h;
+              if (c0 >= a.ocols) continue;
+              uint4* sb = reinterpret_cast<uint4*>(sStore + (q * 2 + (store_count & 1)) * 4096);
+              if (store_count >= 2) {
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+              }
+              uint4* rowp = sb + lane * 8;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const uint32_t* r = rr[h + (k >> 2)] + (k & 3) * 8;
+                uint4 u;
+                u.x = pack2<TOut>(__uint_as_float(r[0]), __uint_as_float(r[1]));
+                u.y = pack2<TOut>(__uint_as_float(r[2]), __uint_as_float(r[3]));
+                u.z = pack2<TOut>(__uint_as_float(r[4]), __uint_as_float(r[5]));
+                u.w = pack2<TOut>(__uint_as_float(r[6]), __uint_as_float(r[7]));
+                rowp[k ^ (lane & 7)] = u;
+              }
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tmD, smem_u32(sb), c0, mt * BM + q * 32, b);
+                bulk_commit();
+              }
+              ++store_count;
+            }
+            continue;
+          }
         }
         if (!row_ok) continue;
 #pragma unroll
@@ -396,10 +430,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
-    if constexpr (sizeof(TOut) == 4) {
-      if (a.tma_store && lane == 0) bulk_wait_all();   // the last stores have landed
-      __syncwarp();
-    }
+    if (a.tma_store && lane == 0) bulk_wait_all();   // the last stores have landed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -448,15 +480,20 @@ cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcAr
   return cudaGetLastError();
 }
 
-// 3D fp32 map over D [batches][rows][cols] for the epilogue's TMA stores (box 32 x 32, 128-byte swizzle).
-bool encode_store_map(CUtensorMap* m, const float* d, long long cols, long long rows, long long batches) {
-  if (cols % 4 != 0 || (reinterpret_cast<uintptr_t>(d) & 15)) return false;
+// 3D map over D [batches][rows][cols] (fp32 or 16-bit) for the epilogue's TMA stores: boxes of
+// 32 rows x 128 bytes (32 fp32 or 64 16-bit columns), 128-byte swizzle.  Rows must be 16-byte
+// multiples and D 16-byte aligned; rows and columns past the ends are clipped by the map.
+bool encode_store_map(CUtensorMap* m, const void* d, conv_dtype_t dt, long long cols, long long rows,
+                      long long batches) {
+  const int esz = dtype_size(dt);
+  if ((cols * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(d) & 15)) return false;
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batches};
-  cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)rows * cols * 4};
-  cuuint32_t box[3] = {32, 32, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * esz, (cuuint64_t)rows * cols * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / esz), 32, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return g_encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(d), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+  const CUtensorMapDataType t = dt == CONV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tmap_dtype(dt);
+  return g_encode_tiled(m, t, 3, const_cast<void*>(d), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -533,18 +570,20 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
     a.out_batch = M * g.o;
     a.accumulate = 0;
     CUtensorMap tD;
-    a.tma_store = encode_store_map(&tD, partial, g.o, M, ksplit) ? 1 : 0;
+    a.tma_store = encode_store_map(&tD, partial, CONV_F32, g.o, M, ksplit) ? 1 : 0;
     if (dt == CONV_BF16)
       return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
                            : launch_kernel<128, 1, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
     return tile_n == 256 ? launch_kernel<256, 1, __half, float>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 1, __half, float>(tA, tB, a, sm_count, s, &tD);
   }
+  CUtensorMap tD;
+  a.tma_store = !accumulate && encode_store_map(&tD, out, dt, g.o, M, 1) ? 1 : 0;
   if (dt == CONV_BF16)
-    return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
-  return tile_n == 256 ? launch_kernel<256, 1, __half, __half>(tA, tB, a, sm_count, s)
-                       : launch_kernel<128, 1, __half, __half>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD)
+                         : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD);
+  return tile_n == 256 ? launch_kernel<256, 1, __half, __half>(tA, tB, a, sm_count, s, &tD)
+                       : launch_kernel<128, 1, __half, __half>(tA, tB, a, sm_count, s, &tD);
 }
 
 bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w) {
@@ -603,11 +642,13 @@ cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geo
   a.out_batch = 0;
   a.accumulate = 0;
   a.err = err_word;
+  CUtensorMap tD;
+  a.tma_store = encode_store_map(&tD, out, dt, g.o, M, 1) ? 1 : 0;
   if (dt == CONV_BF16)
-    return tile_n == 256 ? launch_kernel<256, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s)
-                         : launch_kernel<128, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s);
-  return tile_n == 256 ? launch_kernel<256, 2, __half, __half>(tA, tB, a, sm_count, s)
-                       : launch_kernel<128, 2, __half, __half>(tA, tB, a, sm_count, s);
+    return tile_n == 256 ? launch_kernel<256, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD)
+                         : launch_kernel<128, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD);
+  return tile_n == 256 ? launch_kernel<256, 2, __half, __half>(tA, tB, a, sm_count, s, &tD)
+                       : launch_kernel<128, 2, __half, __half>(tA, tB, a, sm_count, s, &tD);
 }
 
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n, int sm_count,
@@ -638,8 +679,19 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   a.out_batch = (long long)bg.t * bg.o;
   a.ksplit = 1;
   a.err = err_word;
+  if (bg.d_dt != CONV_F32) {
+    // D in the operand type: the vectorised 16-bit epilogue
+    if (bg.d_dt != dt) return cudaErrorInvalidValue;
+    CUtensorMap tD16;
+    a.tma_store = encode_store_map(&tD16, bg.d, dt, bg.o, bg.t, bg.batches) ? 1 : 0;
+    if (dt == CONV_BF16)
+      return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD16)
+                           : launch_kernel<128, 0, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD16);
+    return tile_n == 256 ? launch_kernel<256, 0, __half, __half>(tA, tB, a, sm_count, s, &tD16)
+                         : launch_kernel<128, 0, __half, __half>(tA, tB, a, sm_count, s, &tD16);
+  }
   CUtensorMap tD;
-  a.tma_store = encode_store_map(&tD, bg.d, bg.o, bg.t, bg.batches) ? 1 : 0;
+  a.tma_store = encode_store_map(&tD, bg.d, CONV_F32, bg.o, bg.t, bg.batches) ? 1 : 0;
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);

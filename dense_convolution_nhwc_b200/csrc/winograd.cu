@@ -150,9 +150,11 @@ struct WinoOutArgs {
   int accumulate;
 };
 
-template <int M, typename Tout, typename Idx>
+// TM: the element type of M (fp32, or the 16-bit operand type of the
+// tensor-core path).
+template <int M, typename TM, typename Tout, typename Idx>
 __global__ void __launch_bounds__(256)
-wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
+wino_output_kernel(const TM* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
   constexpr int A = Wino<M>::A;
   const int o = blockIdx.y * blockDim.x + threadIdx.x;
   const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
@@ -163,12 +165,12 @@ wino_output_kernel(const float* __restrict__ mb, const WinoOutArgs a, Tout* __re
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
 
   const Idx plane = (Idx)(a.t_stride * a.o);
-  const float* mp = mb + t * a.o + o;
+  const TM* mp = mb + t * a.o + o;
   float x[A][A];
 #pragma unroll
   for (int i = 0; i < A; ++i)
 #pragma unroll
-    for (int j = 0; j < A; ++j) x[i][j] = __ldg(mp + (Idx)(i * A + j) * plane);
+    for (int j = 0; j < A; ++j) x[i][j] = Store<TM>::to_f32(mp[(Idx)(i * A + j) * plane]);
   // columns: t = A^T x (M x A), then rows: y = t A (M x M)
   float tt[M][A];
 #pragma unroll
@@ -450,7 +452,7 @@ cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int 
   });
 }
 
-cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb, int m,
+cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, int nb, int m,
                                long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
                                cudaStream_t s) {
   WinoOutArgs a{};
@@ -473,11 +475,19 @@ cudaError_t launch_wino_output(const float* mbuf, const Geom& g, int n0, int nb,
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(out_dt, [&](auto to) {
       using Tout = decltype(to);
-      if (idx32)
-        wino_output_kernel<M, Tout, int><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
-      else
-        wino_output_kernel<M, Tout, long long><<<grid, block, 0, s>>>(mbuf, a, static_cast<Tout*>(out));
-      return cudaGetLastError();
+      auto go = [&](auto tm) {
+        using TM = decltype(tm);
+        const TM* mp = static_cast<const TM*>(mbuf);
+        if (idx32)
+          wino_output_kernel<M, TM, Tout, int><<<grid, block, 0, s>>>(mp, a, static_cast<Tout*>(out));
+        else
+          wino_output_kernel<M, TM, Tout, long long><<<grid, block, 0, s>>>(mp, a, static_cast<Tout*>(out));
+        return cudaGetLastError();
+      };
+      // M is fp32, or the output's own 16-bit type
+      if (m_dt == CONV_F32) return go(float{});
+      if (m_dt != out_dt) return cudaErrorInvalidValue;
+      return go(Tout{});
     });
   });
 }

@@ -124,8 +124,15 @@ def test_sixteen_bit_takes_tensor_cores():
 
 
 def test_sixteen_bit_forced_winograd_uses_f2x2():
-    st, p = plan2d(synth.Conv2dShape(2, 32, 32, 256, 256, 3, 3, (1, 1), (1, 1), (1, 1)), "bf16", algo="winograd")
-    assert st == 0 and p["algo"] == "winograd" and p["winograd_m"] == 2 and p["engine"] == "tcgen05"
+    """F(2x2,3x3) on the tensor cores, with U, V and M all in the 16-bit type:
+    workspace = 16 * (O*C + T*C + T*O) * 2 bytes (each buffer 256-aligned)."""
+    s = synth.Conv2dShape(2, 32, 32, 256, 192, 3, 3, (1, 1), (1, 1), (1, 1))
+    for dt in ("bf16", "f16"):
+        st, p = plan2d(s, dt, algo="winograd")
+        assert st == 0 and p["algo"] == "winograd" and p["winograd_m"] == 2 and p["engine"] == "tcgen05"
+        al = lambda x: (x + 255) // 256 * 256
+        T = 2 * 16 * 16
+        assert p["workspace_bytes"] == al(16 * 192 * 256 * 2) + al(16 * T * 256 * 2) + al(16 * T * 192 * 2)
 
 
 def test_forced_winograd_rejects_other_shapes():

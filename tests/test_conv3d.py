@@ -173,6 +173,19 @@ def test_winograd3d_16bit_forced_against_oracle(s, dtype):
     check3d(s, dtype, options=opt)
 
 
+def test_winograd3d_large_pads_and_empty_batch():
+    """Pads beyond the filter reach (whole tiles of padding) in every dimension,
+    and N = 0, which is a no-op that touches nothing."""
+    s = synth.Conv3dShape(1, 4, 5, 6, 32, 64, 3, 3, 3, (1, 1, 1), (3, 4, 2), (1, 1, 1))
+    opt = B.make_options("winograd")
+    assert wino3d_plan(s, "f32", opt)["algo"] == "winograd"
+    check3d(s, "f32", options=opt)
+    e = synth.Conv3dShape(0, 6, 8, 8, 32, 32, 3, 3, 3, (1, 1, 1), (1, 1, 1), (1, 1, 1))
+    d = B.make_desc3d(0, e.d, e.h, e.w, e.c, e.o, 3, 3, 3, e.stride, e.pad, e.dilation)
+    st = B.conv3d_forward(0, 0, 0, d, 0, opt, 0, 0, torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_winograd3d_forced_unaligned_channels(dtype):
     """C % 8 != 0 (16-bit operands then go through the FFMA GEMM in fp32) and an
