@@ -4,9 +4,9 @@
 // and Fix; maintainer review: dispatch never depends on current memory):
 //   * Winograd is considered for 3x3, stride 1, dilation 1 convs that meet
 //     the page's channel rule C % 32 == 0 && O % 32 == 0 && C + O >= 256, for
-//     fp32 inputs (16-bit inputs take the tensor-core implicit GEMM unless
-//     Winograd is forced: on B200 the unfused transforms' HBM traffic costs
-//     more than the tensor cores save).
+//     fp32 inputs, and for 16-bit inputs only with deep, wide GEMMs (C >= 1024
+//     and O >= 1024, or C >= 512 and O >= 2048): below that the transforms'
+//     HBM traffic costs more than the tensor cores save.
 //   * The batch is cut into tiles of nb images, nb = floor(budget /
 //     per-image scratch), budget = min(3/4 * total device memory - (input +
 //     output + transformed filter), 8 GiB).  nb = 0, or tiles carrying fewer
@@ -184,6 +184,13 @@ bool winograd_shape(const Geom& g) {
 bool winograd_channel_rule(const Geom& g) {
   return g.c % 32 == 0 && g.o % 32 == 0 && g.c + g.o >= 256;
 }
+// 16-bit inputs: F(2x2,3x3) on the tensor cores against the implicit GEMM.
+// Winograd saves 2.25x of the tensor work but moves V and M through HBM; on
+// B200 it is the faster of the two once the GEMMs are deep and wide enough
+// (measured on the wide 3x3 set: C >= 1024 with O >= 1024, C >= 512 with O >= 2048).
+bool winograd_16bit_wins(const Geom& g) {
+  return (g.c >= 1024 && g.o >= 1024) || (g.c >= 512 && g.o >= 2048);
+}
 int winograd_m_for(conv_dtype_t dt) { return dt == CONV_F32 ? 6 : 2; }
 
 // The tensor-core engine can express this shape (pointer alignment is checked at launch).
@@ -252,7 +259,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     if (!wshape) return CONV_ERR_UNSUPPORTED;
     want_wino = true;
   } else if (o.algo == CONV_ALGO_AUTO) {
-    want_wino = wshape && winograd_channel_rule(g) && dt == CONV_F32;
+    want_wino = wshape && winograd_channel_rule(g) && (dt == CONV_F32 || winograd_16bit_wins(g));
   } else if (o.algo != CONV_ALGO_IMPLICIT_GEMM && o.algo != CONV_ALGO_DIRECT) {
     return CONV_ERR_INVALID;
   }

@@ -23,6 +23,20 @@ template <> struct Store<__nv_bfloat16> {
   static __device__ __forceinline__ __nv_bfloat16 from_f32(float v) { return __float2bfloat16_rn(v); }
 };
 
+// Two adjacent 16-bit values as one 32-bit word, converted per component with
+// the same round-to-nearest-even as Store<T>.
+template <typename T> struct Pair;
+template <> struct Pair<__half> {
+  using type = __half2;
+  static __device__ __forceinline__ float2 to_f32(type v) { return __half22float2(v); }
+  static __device__ __forceinline__ type from_f32(float a, float b) { return __floats2half2_rn(a, b); }
+};
+template <> struct Pair<__nv_bfloat16> {
+  using type = __nv_bfloat162;
+  static __device__ __forceinline__ float2 to_f32(type v) { return __bfloat1622float2(v); }
+  static __device__ __forceinline__ type from_f32(float a, float b) { return __floats2bfloat162_rn(a, b); }
+};
+
 template <typename T>
 __device__ __forceinline__ float ld_f32(const T* p) { return Store<T>::to_f32(*p); }
 template <typename T>

@@ -208,6 +208,154 @@ wino_output_kernel(const TM* __restrict__ mb, const WinoOutArgs a, Tout* __restr
 }
 
 // ---------------------------------------------------------------------------
+// 16-bit transforms on channel pairs: a thread owns channels (2p, 2p+1) of one
+// tile, so each load and store moves 32 bits (the arithmetic per channel is
+// that of the kernels above, bit for bit).
+// ---------------------------------------------------------------------------
+template <int M, typename T, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_input_pair_kernel(const T* __restrict__ in, const WinoInArgs a, T* __restrict__ v) {
+  using P = Pair<T>;
+  using PT = typename P::type;
+  constexpr int A = Wino<M>::A;
+  const int cp = a.c >> 1;
+  const int cgroups = (cp + blockDim.x - 1) / blockDim.x;
+  const int cg = (int)(blockIdx.x % cgroups);
+  const long long tg = blockIdx.x / cgroups;
+  const int c2 = cg * blockDim.x + threadIdx.x;
+  const long long t = tg * blockDim.y + threadIdx.y;
+  if (c2 >= cp || t >= a.t_count) return;
+  const int per_img = a.tiles_h * a.tiles_w;
+  const int nl = (int)(t / per_img);
+  const int r = (int)(t - (long long)nl * per_img);
+  const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
+  const int y0 = ty * M - a.ph, x0 = tx * M - a.pw;
+  const PT* base = reinterpret_cast<const PT*>(in + (long long)(a.n0 + nl) * a.in_img_stride) + c2;
+  const Idx cs = cp, wc = (Idx)a.w * cp;
+
+  float d[2][A][A];
+  auto put = [&](int i, int j, PT pv) {
+    const float2 f = P::to_f32(pv);
+    d[0][i][j] = f.x;
+    d[1][i][j] = f.y;
+  };
+  if (y0 >= 0 && x0 >= 0 && y0 + A <= a.h && x0 + A <= a.w) {
+    const PT* p = base + ((Idx)y0 * wc + (Idx)x0 * cs);
+#pragma unroll
+    for (int i = 0; i < A; ++i)
+#pragma unroll
+      for (int j = 0; j < A; ++j) put(i, j, p[(Idx)i * wc + (Idx)j * cs]);
+  } else {
+    unsigned xm = 0;
+#pragma unroll
+    for (int j = 0; j < A; ++j)
+      if (x0 + j >= 0 && x0 + j < a.w) xm |= 1u << j;
+#pragma unroll
+    for (int i = 0; i < A; ++i) {
+      const int y = y0 + i;
+      const bool yok = y >= 0 && y < a.h;
+      const Idx ro = yok ? (Idx)y * wc + (Idx)x0 * cs : (Idx)0;
+#pragma unroll
+      for (int j = 0; j < A; ++j) {
+        if (yok && ((xm >> j) & 1u)) {
+          put(i, j, base[ro + (Idx)j * cs]);
+        } else {
+          d[0][i][j] = 0.0f;
+          d[1][i][j] = 0.0f;
+        }
+      }
+    }
+  }
+  float res[2][A][A];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float tt[A][A];
+#pragma unroll
+    for (int j = 0; j < A; ++j) {
+      float col[A], rr[A];
+#pragma unroll
+      for (int i = 0; i < A; ++i) col[i] = d[h][i][j];
+      Wino<M>::bt(col, rr);
+#pragma unroll
+      for (int i = 0; i < A; ++i) tt[i][j] = rr[i];
+    }
+#pragma unroll
+    for (int i = 0; i < A; ++i) Wino<M>::bt(tt[i], res[h][i]);
+  }
+  const Idx plane = (Idx)(a.t_stride * cp);
+  PT* vp = reinterpret_cast<PT*>(v + t * a.c) + c2;
+#pragma unroll
+  for (int i = 0; i < A; ++i)
+#pragma unroll
+    for (int j = 0; j < A; ++j) vp[(Idx)(i * A + j) * plane] = P::from_f32(res[0][i][j], res[1][i][j]);
+}
+
+template <int M, typename T, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_output_pair_kernel(const T* __restrict__ mb, const WinoOutArgs a, T* __restrict__ out) {
+  using P = Pair<T>;
+  using PT = typename P::type;
+  constexpr int A = Wino<M>::A;
+  const int op = a.o >> 1;
+  const int o2 = blockIdx.y * blockDim.x + threadIdx.x;
+  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  if (o2 >= op || t >= a.t_count) return;
+  const int per_img = a.tiles_h * a.tiles_w;
+  const int nl = (int)(t / per_img);
+  const int r = (int)(t - (long long)nl * per_img);
+  const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
+
+  const Idx plane = (Idx)(a.t_stride * op);
+  const PT* mp = reinterpret_cast<const PT*>(mb + t * a.o) + o2;
+  float x[2][A][A];
+#pragma unroll
+  for (int i = 0; i < A; ++i)
+#pragma unroll
+    for (int j = 0; j < A; ++j) {
+      const float2 f = P::to_f32(mp[(Idx)(i * A + j) * plane]);
+      x[0][i][j] = f.x;
+      x[1][i][j] = f.y;
+    }
+  float y[2][M][M];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float tt[M][A];
+#pragma unroll
+    for (int j = 0; j < A; ++j) {
+      float col[A], rr[M];
+#pragma unroll
+      for (int i = 0; i < A; ++i) col[i] = x[h][i][j];
+      Wino<M>::at(col, rr);
+#pragma unroll
+      for (int i = 0; i < M; ++i) tt[i][j] = rr[i];
+    }
+#pragma unroll
+    for (int i = 0; i < M; ++i) Wino<M>::at(tt[i], y[h][i]);
+  }
+  PT* opp = reinterpret_cast<PT*>(out + (long long)(a.n0 + nl) * a.out_img_stride) + o2;
+  const Idx os = op, wo = (Idx)a.ow * op;
+  const bool whole = ty * M + M <= a.oh && tx * M + M <= a.ow;
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+    const int yy = ty * M + i;
+    if (!whole && yy >= a.oh) continue;
+    PT* rp = opp + ((Idx)yy * wo + (Idx)(tx * M) * os);
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      if (!whole && tx * M + j >= a.ow) continue;
+      float v0 = y[0][i][j], v1 = y[1][i][j];
+      if (a.accumulate) {
+        const float2 old = P::to_f32(rp[(Idx)j * os]);
+        const float2 tap = P::to_f32(P::from_f32(v0, v1));
+        v0 = old.x + tap.x;
+        v1 = old.y + tap.y;
+      }
+      rp[(Idx)j * os] = P::from_f32(v0, v1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Channel-major variants for the FFMA GEMM: U[xi][c][o] (row stride O_pad) and
 // V[xi][c][t] (row stride T_pad), fp32.  Rows of both are contiguous in the
 // GEMM's m / n direction, so the GEMM stages them with 16-byte copies.
@@ -391,6 +539,26 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   // whole V plane set stay below 2^31 elements
   const int a2 = (m + 2) * (m + 2);
   const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31) && (long long)a2 * t_tile * g.c < (1LL << 31);
+  // 16-bit in and out, F(2,3): channel pairs
+  if (m == 2 && in_dt != CONV_F32 && store_dt == in_dt && g.c % 2 == 0 && g.in_img_stride % 2 == 0 &&
+      (reinterpret_cast<uintptr_t>(in) & 3) == 0 && (reinterpret_cast<uintptr_t>(v) & 3) == 0) {
+    const int cp = g.c / 2;
+    const int pbx = cp >= 64 ? 64 : 32;
+    dim3 pblock(pbx, 256 / pbx);
+    const long long pblocks = ((a.t_count + pblock.y - 1) / pblock.y) * ((cp + pbx - 1) / pbx);
+    if (pblocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    auto go = [&](auto tv) {
+      using T = decltype(tv);
+      if (idx32)
+        wino_input_pair_kernel<2, T, int><<<(unsigned)pblocks, pblock, 0, s>>>(static_cast<const T*>(in), a,
+                                                                              static_cast<T*>(v));
+      else
+        wino_input_pair_kernel<2, T, long long><<<(unsigned)pblocks, pblock, 0, s>>>(static_cast<const T*>(in), a,
+                                                                                    static_cast<T*>(v));
+      return cudaGetLastError();
+    };
+    return in_dt == CONV_BF16 ? go(__nv_bfloat16{}) : go(__half{});
+  }
   return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(in_dt, [&](auto ti) {
@@ -471,6 +639,26 @@ cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& 
   if (grid.y > 65535) return cudaErrorInvalidValue;
   const int a2 = (m + 2) * (m + 2);
   const bool idx32 = g.out_img_stride < (1LL << 31) && (long long)a2 * t_tile * g.o < (1LL << 31);
+  // 16-bit M and out, F(2,3): channel pairs
+  if (m == 2 && out_dt != CONV_F32 && m_dt == out_dt && g.o % 2 == 0 && g.out_img_stride % 2 == 0 &&
+      (reinterpret_cast<uintptr_t>(out) & 3) == 0 && (reinterpret_cast<uintptr_t>(mbuf) & 3) == 0) {
+    const int op = g.o / 2;
+    const int pbx = op >= 64 ? 64 : 32;
+    dim3 pblock(pbx, 256 / pbx);
+    dim3 pgrid((unsigned)((a.t_count + pblock.y - 1) / pblock.y), (op + pbx - 1) / pbx);
+    if (pgrid.y > 65535) return cudaErrorInvalidValue;
+    auto go = [&](auto tv) {
+      using T = decltype(tv);
+      if (idx32)
+        wino_output_pair_kernel<2, T, int><<<pgrid, pblock, 0, s>>>(static_cast<const T*>(mbuf), a,
+                                                                    static_cast<T*>(out));
+      else
+        wino_output_pair_kernel<2, T, long long><<<pgrid, pblock, 0, s>>>(static_cast<const T*>(mbuf), a,
+                                                                          static_cast<T*>(out));
+      return cudaGetLastError();
+    };
+    return out_dt == CONV_BF16 ? go(__nv_bfloat16{}) : go(__half{});
+  }
   return wino_by_m(m, [&](auto mc) {
     constexpr int M = decltype(mc)::value;
     return wino_by_dt(out_dt, [&](auto to) {

@@ -150,6 +150,10 @@ B200CONV_API conv_status_t conv_device_props(int device, conv_device_props_t *pr
  * Plan a conv2d: validate, compute the output shape, pick the algorithm, the
  * tile configuration and the Winograd batch tile, and size the workspace.
  * Pure: the same arguments give the same plan in any process at any time.
+ * Winograd (auto) needs 3x3, stride 1, dilation 1 and the page's channel rule
+ * (C % 32 == 0, O % 32 == 0, C + O >= 256); 16-bit inputs take it only for deep,
+ * wide GEMMs (C >= 1024 and O >= 1024, or C >= 512 and O >= 2048), else the
+ * tensor-core implicit GEMM.
  * The Winograd budget is 3/4 of the device's total memory minus the conv's own
  * tensors (input, output, transformed filter), capped at 8 GiB because the GPU
  * is shared ("Bound winograd conv2d working set by tiling the batch", Fix).

@@ -123,6 +123,25 @@ def test_sixteen_bit_takes_tensor_cores():
                 assert p["channel_pad"] == 0 and (p["workspace_bytes"] == 0) == (p["k_split"] == 1)
 
 
+def test_sixteen_bit_auto_winograd_only_for_deep_wide_gemms():
+    """16-bit auto takes F(2,3) on the tensor cores where it measured faster
+    than the implicit GEMM: C >= 1024 with O >= 1024, or C >= 512 with O >= 2048."""
+    for (c, o), want in [((1024, 1024), True), ((1024, 4096), True), ((512, 2048), True), ((1024, 512), False),
+                         ((512, 1024), False), ((256, 4096), False), ((2048, 2048), True)]:
+        s = synth.Conv2dShape(16, 64, 64, c, o, 3, 3, (1, 1), (1, 1), (1, 1))
+        for dt in ("bf16", "f16"):
+            st, p = plan2d(s, dt)
+            assert st == 0 and (p["algo"] == "winograd") == want, (c, o, dt, p["algo"])
+            assert p["engine"] == "tcgen05"
+            if want:
+                assert p["winograd_m"] == 2
+    # stride 2 or a 5x5 filter never takes it
+    for s in (synth.Conv2dShape(16, 64, 64, 1024, 1024, 3, 3, (2, 2), (1, 1), (1, 1)),
+              synth.Conv2dShape(16, 64, 64, 1024, 1024, 5, 5, (1, 1), (2, 2), (1, 1))):
+        st, p = plan2d(s, "bf16")
+        assert st == 0 and p["algo"] == "implicit"
+
+
 def test_sixteen_bit_forced_winograd_uses_f2x2():
     """F(2x2,3x3) on the tensor cores, with U, V and M all in the 16-bit type:
     workspace = 16 * (O*C + T*C + T*O) * 2 bytes (each buffer 256-aligned)."""

@@ -101,6 +101,29 @@ def test_taps_equal_manual_per_frame_loop(dtype):
     assert torch.equal(got[0], acc)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_winograd_taps_accumulate_equal_manual_loop(dtype):
+    """KD = 2 with forced Winograd: depth taps whose 2D Winograd output stage adds
+    into out equal conv2d (forced Winograd) per frame view + conv_accumulate, bit
+    for bit, and match the oracle."""
+    s = synth.Conv3dShape(1, 7, 10, 12, 64, 96, 2, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    opt = B.make_options("winograd")
+    x, w = synth.conv3d_inputs(s, dtype, "normal", 8, device="cuda")
+    got = run3d(x, w, s, opt)
+    acc = None
+    for kd in range(s.kd):
+        tap = B.conv2d(x[0, kd:kd + s.od], w[:, kd].contiguous(), s.stride[1:], s.pad[1:], s.dilation[1:], options=opt)
+        if acc is None:
+            acc = tap
+        else:
+            assert B.conv_accumulate(acc.data_ptr(), tap.data_ptr(), acc.numel(), B.DTYPE[dtype],
+                                     torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(got[0], acc)
+    ref = oracle.conv3d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
+    assert_close(as_f64(got), ref, dtype, s.name())
+
+
 @pytest.mark.parametrize("s", synth.CONV3D_TAPS, ids=lambda s: s.name())
 def test_workload_shapes_sampled(s):
     check3d(s, "bf16", sample=2048)
