@@ -10,7 +10,8 @@ _BINDING_NAMES = frozenset({
     # C-ABI entry points (same names as include/b200conv.h)
     "conv2d_forward", "conv3d_forward", "conv1d_forward", "conv1d_plan", "conv1d_workspace_size", "conv2d_forward_winograd_static", "conv2d_plan", "conv3d_plan",
     "conv2d_plan_for_props", "conv3d_plan_for_props",
-    "conv2d_workspace_size", "conv3d_workspace_size", "conv_check", "conv_selftest_timeout",
+    "conv2d_workspace_size", "conv3d_workspace_size", "conv_check", "conv_selftest_timeout", "conv_fp32_fma_rate",
+    "fp32_fma_rate",
     "conv_status_string", "conv_device_props", "conv_accumulate", "conv_profile_begin", "conv_profile_end",
     "profile_end", "KernelTime",
     # types and helpers

@@ -115,6 +115,7 @@ _conv2d_forward_winograd_static = _sig("conv2d_forward_winograd_static", _I, _P,
                                        ctypes.POINTER(Conv2dDesc), _I, _P)
 _conv_check = _sig("conv_check", _I, _P)
 _conv_selftest_timeout = _sig("conv_selftest_timeout", _I, ctypes.c_longlong, _P)
+_conv_fp32_fma_rate = _sig("conv_fp32_fma_rate", _I, _I, ctypes.POINTER(ctypes.c_double), _P)
 _conv_status_string = _sig("conv_status_string", ctypes.c_char_p, _I)
 
 
@@ -215,6 +216,20 @@ def conv_check(stream: int) -> int:
 
 def conv_selftest_timeout(limit_ns: int, stream: int) -> int:
     return _conv_selftest_timeout(limit_ns, stream or None)
+
+
+def conv_fp32_fma_rate(packed: int, tflops, stream: int) -> int:
+    """tflops: a ctypes.c_double filled with the measured fp32 FMA rate (TFLOP/s)."""
+    return _conv_fp32_fma_rate(packed, ctypes.byref(tflops), stream or None)
+
+
+def fp32_fma_rate(packed: bool = True, stream: int = 0) -> float:
+    """The measured CUDA-core fp32 FMA rate of the current device, TFLOP/s."""
+    v = ctypes.c_double(0.0)
+    st = _conv_fp32_fma_rate(1 if packed else 0, ctypes.byref(v), stream or None)
+    if st != 0:
+        raise ConvError(st, "conv_fp32_fma_rate")
+    return v.value
 
 
 def conv_profile_begin() -> int:

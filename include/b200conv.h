@@ -250,6 +250,15 @@ B200CONV_API conv_status_t conv_accumulate(void *out, const void *tap, size_t co
                               void *stream);
 
 /*
+ * Diagnostic: measure the CUDA-core fp32 FMA rate of the current device in
+ * TFLOP/s (2 FLOP per lane per FMA), scalar FFMA (packed = 0) or sm_100's
+ * packed two-lane FMA (packed = 1), the denominator of the fp32 kernels'
+ * roofline.  Runs a few short FMA-chain kernels on `stream` and synchronizes
+ * it; allocates no device memory.  CONV_ERR_CUDA if the device cannot run it.
+ */
+B200CONV_API conv_status_t conv_fp32_fma_rate(int packed, double *tflops, void *stream);
+
+/*
  * Synchronise `stream`, then read and clear the current device's error word.
  * Returns CONV_ERR_TIMEOUT if a kernel's bounded wait ran out since the last
  * check, CONV_ERR_CUDA if the synchronisation failed, else CONV_OK.

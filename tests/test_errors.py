@@ -75,6 +75,17 @@ def test_misaligned_workspace_is_refused_and_nothing_runs():
     assert torch.isnan(out).all()
 
 
+def test_fp32_fma_rate_probe():
+    """The FMA-chain probe reports a plausible CUDA-core fp32 rate for both forms
+    (a B200 at 1.9-2.0 GHz: ~70-80 TFLOP/s scalar), and refuses a null output."""
+    import ctypes
+    scalar = B.fp32_fma_rate(packed=False)
+    packed = B.fp32_fma_rate(packed=True)
+    print(f"fp32 FMA rate: scalar {scalar:.1f}, packed {packed:.1f} TFLOP/s")
+    assert 20.0 < scalar < 400.0 and 20.0 < packed < 400.0
+    assert B._conv_fp32_fma_rate(0, None, None) == 1
+
+
 def test_overlapping_output_is_refused():
     x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
     st = B.conv2d_forward(x.data_ptr(), w.data_ptr(), x.data_ptr(), desc(S), 0, None, 0, 0, stream())
