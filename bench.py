@@ -41,7 +41,7 @@ from dense_convolution_nhwc_b200 import synth  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
 FP32_LANES_PER_SM = 128
-BASELINE_CONTEXT = {
+PAGES_NUMBER = {
     # direct-equivalent TFLOP/s of the pages' own measurement of the same workload
     # (310 ms on an M2 Max: 2*40*512*512*96*192*9 / 0.310 s); context, another machine
     "winograd_f32": 11.2,
@@ -669,7 +669,7 @@ def main():
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": (value / BASELINE_CONTEXT[args.workload]) if args.workload in BASELINE_CONTEXT else None,
+            "vs_baseline": (value / PAGES_NUMBER[args.workload]) if args.workload in PAGES_NUMBER else None,
             "dtype": dtype, "data": "synthetic",
             "config": {"workload": desc, "plan": {k: plan0[k] for k in ("algo", "engine", "winograd_m", "batch_tile",
                                                                           "num_batch_tiles", "tile_n")},
@@ -682,7 +682,7 @@ def main():
             "gpu_launches_per_step": gpu_launches / args.steps,
             "e2e": e2e, "cpu_baseline": cpu,
         }
-        if args.workload in BASELINE_CONTEXT:
+        if args.workload in PAGES_NUMBER:
             line["vs_baseline_note"] = "pages' 310 ms on an M2 Max for the same workload (context, other hardware)"
         print(json.dumps(line))
         if args.per_conv:
