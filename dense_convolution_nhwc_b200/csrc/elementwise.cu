@@ -161,34 +161,16 @@ __global__ void splitk_reduce_scalar_kernel(const float* __restrict__ partial, i
   }
 }
 
-// dst[k][o] = w[o][k] (row strides w_row_stride, ldb), 32 x 32 tiles through shared memory.
-__global__ void transpose_weights_kernel(const float* __restrict__ w, int O, long long K, long long w_row_stride,
-                                         float* __restrict__ dst, long long ldb) {
-  __shared__ float tile[32][33];
-  const long long k0 = (long long)blockIdx.x * 32;
-  const int o0 = blockIdx.y * 32;
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const int o = o0 + r;
-    const long long k = k0 + threadIdx.x;
-    tile[r][threadIdx.x] = (o < O && k < K) ? w[(long long)o * w_row_stride + k] : 0.0f;
-  }
-  __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
-    const long long k = k0 + r;
-    const int o = o0 + threadIdx.x;
-    if (k < K && o < O) dst[k * ldb + o] = tile[threadIdx.x][r];
-  }
-}
-
 }  // namespace
 
-cudaError_t launch_transpose_weights(const float* w, int o, long long k, long long w_row_stride, float* dst,
-                                     long long ldb, cudaStream_t s) {
-  if (o == 0 || k == 0) return cudaSuccess;
-  dim3 grid((unsigned)((k + 31) / 32), (o + 31) / 32);
-  if (grid.y > 65535) return cudaErrorInvalidValue;
-  transpose_weights_kernel<<<grid, dim3(32, 8), 0, s>>>(w, o, k, w_row_stride, dst, ldb);
-  return cudaGetLastError();
+// The small kernels that run between tensor-core convs ask for the same
+// shared-memory carveout as those (the maximum), so the SM is not
+// reconfigured between a conv and its reduce or pre-pass.  A preference only;
+// set once per kernel (the attribute is per function).
+template <typename K>
+bool prefer_max_shared(K kernel) {
+  cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  return true;
 }
 
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count, void* out, conv_dtype_t dt,
@@ -200,6 +182,10 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count,
   unsigned blocks = (unsigned)((items + 255) / 256 < 148 * 16 ? (items + 255) / 256 : 148 * 16);
   auto run = [&](auto tag) {
     using T = decltype(tag);
+    static const bool pv = prefer_max_shared(splitk_reduce_kernel<T>);
+    static const bool ps = prefer_max_shared(splitk_reduce_scalar_kernel<T>);
+    (void)pv;
+    (void)ps;
     if (vec)
       splitk_reduce_kernel<T><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<T*>(out), acc);
     else
