@@ -1,10 +1,14 @@
-// common.cuh -- device helpers shared by the kernels: storage-type traits and
-// round-to-nearest-even conversions from the fp32 accumulators.
+// common.cuh -- helpers shared by the kernels: storage-type traits,
+// round-to-nearest-even conversions from the fp32 accumulators, and
+// programmatic dependent launch.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <utility>
+
+#include <cuda_runtime.h>
 
 namespace b200conv {
 
@@ -51,6 +55,34 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) 
 template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel in the
+// stream finishes; it runs its prologue (barriers, TMEM, tensor-map prefetch),
+// then waits here for the previous kernel's results before touching global
+// memory, and lets the next kernel start launching.  Both are no-ops for a
+// normal launch.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with programmatic stream serialization (the kernel calls
+// pdl_wait_then_release before its first global access).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, int smem, cudaStream_t s, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
 }  // namespace b200conv

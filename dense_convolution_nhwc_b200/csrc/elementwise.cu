@@ -127,6 +127,7 @@ __global__ void wpack_kernel(const T* __restrict__ src, long long pixels /* n*h*
 template <typename T>
 __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int ksplit, size_t count, T* __restrict__ out,
                                      int accumulate) {
+  pdl_wait_then_release();     // the partials come from the conv launched just before
   const size_t n4 = count / 4;
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -150,6 +151,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int kspl
 template <typename T>
 __global__ void splitk_reduce_scalar_kernel(const float* __restrict__ partial, int ksplit, size_t count,
                                             T* __restrict__ out, int accumulate) {
+  pdl_wait_then_release();
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (; i < count; i += stride) {
@@ -186,17 +188,16 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count,
     static const bool ps = prefer_max_shared(splitk_reduce_scalar_kernel<T>);
     (void)pv;
     (void)ps;
-    if (vec)
-      splitk_reduce_kernel<T><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<T*>(out), acc);
-    else
-      splitk_reduce_scalar_kernel<T><<<blocks, 256, 0, s>>>(partial, ksplit, count, static_cast<T*>(out), acc);
+    T* o = static_cast<T*>(out);
+    if (vec) return launch_pdl(splitk_reduce_kernel<T>, dim3(blocks), dim3(256), 0, s, partial, ksplit, count, o, acc);
+    return launch_pdl(splitk_reduce_scalar_kernel<T>, dim3(blocks), dim3(256), 0, s, partial, ksplit, count, o, acc);
   };
   switch (dt) {
-    case CONV_F32: run(float{}); break;
-    case CONV_F16: run(__half{}); break;
-    case CONV_BF16: run(__nv_bfloat16{}); break;
+    case CONV_F32: return run(float{});
+    case CONV_F16: return run(__half{});
+    case CONV_BF16: return run(__nv_bfloat16{});
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,

@@ -131,10 +131,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  if (threadIdx.x == 32) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (a.tma_store) prefetch_tensormap(&tmD);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_then_release();
 
   const long long total_tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
   const int ksteps = a.taps * a.kb_per_tap;
@@ -476,8 +482,7 @@ cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcAr
   int grid = (int)(tiles < sm_count ? tiles : sm_count);
   CUtensorMap none;
   memset(&none, 0, sizeof(none));
-  k<<<grid, THREADS, smem, s>>>(A, B, D ? *D : none, a);
-  return cudaGetLastError();
+  return launch_pdl(k, dim3(grid), dim3(THREADS), smem, s, A, B, D ? *D : none, a);
 }
 
 // 3D map over D [batches][rows][cols] (fp32 or 16-bit) for the epilogue's TMA stores: boxes of

@@ -15,6 +15,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace b200conv {
@@ -164,6 +165,10 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_fmt) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),             \
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])              \
       : "r"(taddr))
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
 
 // ------------------------------- host side ----------------------------------
 
