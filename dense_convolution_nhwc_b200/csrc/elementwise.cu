@@ -89,28 +89,38 @@ __global__ void wpack_kernel(const T* __restrict__ src, long long pixels /* n*h*
                              int pw, int dw, int ow, long long in_row_stride, long long in_img_stride, int h,
                              T* __restrict__ dst, int cp) {
   // one thread per output pixel (n, y, x); its cp packed channels are written in
-  // 8-element vectors (cp is a multiple of 8, rows 16-byte aligned)
+  // 8-element vectors (cp is a multiple of 8, rows 16-byte aligned).  Packed
+  // channel ch = k*c + cc is walked incrementally (no division per element).
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long stride = (long long)gridDim.x * blockDim.x;
+  const int kc = kw * c;
   for (; i < pixels; i += stride) {
-    const int x = (int)(i % ow);
-    const long long nh = i / ow;
+    long long nh;
+    int x;
+    if (pixels < (1LL << 31)) {        // 32-bit division when the pixel count allows it
+      const int ii = (int)i;
+      nh = ii / ow;
+      x = ii - (int)nh * ow;
+    } else {
+      nh = i / ow;
+      x = (int)(i - nh * ow);
+    }
     const long long n = nh / h, y = nh - n * h;
     const T* row = src + n * in_img_stride + y * in_row_stride;
-    const int x0 = x * sw - pw;
     T* out = dst + i * cp;
+    int ix = x * sw - pw, cc = 0, ch = 0;
     for (int ch0 = 0; ch0 < cp; ch0 += 8) {
       __align__(16) T v[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int ch = ch0 + e;
         float f = 0.0f;
-        if (ch < kw * c) {
-          const int k = ch / c, cc = ch - k * c;
-          const int ix = x0 + k * dw;
-          if (ix >= 0 && ix < w) f = Store<T>::to_f32(row[(long long)ix * c + cc]);
-        }
+        if (ch < kc && ix >= 0 && ix < w) f = Store<T>::to_f32(row[(long long)ix * c + cc]);
         v[e] = Store<T>::from_f32(f);
+        ++ch;
+        if (++cc == c) {
+          cc = 0;
+          ix += dw;
+        }
       }
       if constexpr (sizeof(T) == 2) {
         *reinterpret_cast<uint4*>(out + ch0) = *reinterpret_cast<const uint4*>(v);
