@@ -350,7 +350,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     if (s->engine == CONV_ENGINE_TCGEN05) {
       const long long ksteps = taps * ((c_eff + 63) / 64);
       const long long tiles = ((M + 127) / 128) * ((g.o + s->tile_n - 1) / s->tile_n);
-      if (tiles * 2 <= p.sm_count && ksteps >= 8) ks = std::min({(long long)p.sm_count / tiles, ksteps / 4, 16LL});
+      if (tiles * 2 <= p.sm_count && ksteps >= 16) ks = std::min({(long long)p.sm_count / tiles, ksteps / 4, 16LL});
     } else {
       const long long steps = taps * ((c_eff + 15) / 16);
       const long long blocks = ((M + 127) / 128) * ((g.o + s->tile_n - 1) / s->tile_n);
