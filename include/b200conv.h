@@ -218,10 +218,11 @@ B200CONV_API conv_status_t conv1d_forward(const void *in, const void *w, void *o
  *    budget rule, tiled output bit-identical to untiled.
  * With CONV_ALGO_AUTO, fp32 shapes of the 3D Winograd that meet the conv2d
  * channel rule (C % 32 == 0, O % 32 == 0, C + O >= 256) take it when the
- * budget allows (the same fallback rule as conv2d); otherwise the page's guard (N == 1, KD <= 7, depth stride 1,
- * kernel dilation 1, no depth padding, C and O multiples of 16) selects the
- * depth taps and the other shapes take the native GEMM when it can express them
- * (16-bit, C % 8 == 0, 5D box corners within [-16, 15]), else the depth taps.
+ * budget allows (the same fallback rule as conv2d).  Otherwise the page's
+ * guard (N == 1, KD <= 7, depth stride 1, kernel dilation 1, no depth padding,
+ * C and O multiples of 16) selects the depth taps, and the other shapes take
+ * the native GEMM when it can express them (16-bit, C % 8 == 0, 5D box corners
+ * within [-16, 15]), else the depth taps.
  * CONV_ALGO_IMPLICIT_GEMM asks for the native GEMM whenever it can run;
  * CONV_ALGO_WINOGRAD asks for the 3D Winograd on its shapes (any dtype, no
  * channel rule) and otherwise for depth taps with the 2D Winograd;
