@@ -412,175 +412,286 @@ def run_reference(args, wl_name):
 # our arm
 # ---------------------------------------------------------------------------
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="winograd_f32")
-    ap.add_argument("--algo", default="auto", choices=["auto", "implicit", "winograd", "direct"])
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--per-conv", action="store_true", help="also print one line per conv of the workload")
-    ap.add_argument("--graph", action="store_true",
-                    help="capture one step as a CUDA graph and time its replays (removes host launch gaps)")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
-    if args.impl == "reference":
-        run_reference(args, args.workload)
-        return
+# Per-config entries printed inside the headline's JSON line (same run, same
+# GPU): the small fp32 case, the ResNet-50 layer sets (fp16/bf16, batch 1/8),
+# the wide-channel implicit-GEMM members (auto and forced implicit GEMM), the
+# wide 3x3 members with Winograd forced (the Winograd GEMM core), and the
+# conv3d cases.  (key, workload, algo, time as a CUDA graph too)
+PER_CONFIG = [
+    ("config1_small_f32", "small_f32", "auto", False),
+    ("config3_resnet50_f16_b1", "resnet50_f16_b1", "auto", True),
+    ("config3_resnet50_bf16_b1", "resnet50_bf16_b1", "auto", True),
+    ("config3_resnet50_f16_b8", "resnet50_f16_b8", "auto", True),
+    ("config3_resnet50_bf16_b8", "resnet50_bf16_b8", "auto", True),
+    ("config4_wide_bf16_auto", "wide_bf16", "auto", False),
+    ("config4_wide_f16_auto", "wide_f16", "auto", False),
+    ("config4_wide_bf16_implicit", "wide_bf16", "implicit", False),
+    ("config4_wide_f16_implicit", "wide_f16", "implicit", False),
+    ("config4_wide3_bf16_winograd", "wide3_bf16", "winograd", False),
+    ("config4_wide3_f16_winograd", "wide3_f16", "winograd", False),
+    ("config5_conv3d_bf16", "conv3d_bf16", "auto", False),
+    ("config5_conv3d_f32", "conv3d_f32", "auto", False),
+]
 
-    import torch
-    from dense_convolution_nhwc_b200 import binding as B
 
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream(dev)
-    desc, convs, dtype = workload(args.workload)
-    opts = B.make_options(args.algo)
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return json.load(open(p)) if os.path.exists(p) else {}
+    except Exception:
+        return {}
 
-    # resident inputs, outputs and workspaces
-    items = []
-    ws_max = 0
-    for i, cv in enumerate(convs):
-        s = cv.shape
-        if cv.is3d:
-            x, w = synth.conv3d_inputs(s, cv.dtype, cv.dist, i, dev)
-            d = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
-            plan = B.plan3d(d, cv.dtype, local, opts)
-            out = torch.empty((s.n, s.od, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
-        else:
-            x, w = synth.conv2d_inputs(s, cv.dtype, cv.dist, i, dev)
-            d = B.make_desc2d(s.n, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
-            plan = B.plan2d(d, cv.dtype, local, opts)
-            out = torch.empty((s.n, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
-        ws_max = max(ws_max, plan["workspace_bytes"])
-        items.append((cv, x, w, d, plan, out))
-    ws = torch.empty(max(ws_max, 256), dtype=torch.uint8, device=dev)
-    dt_code = B.DTYPE[dtype]
-    fwd = B.conv3d_forward if convs[0].is3d else B.conv2d_forward
-    sptr = stream.cuda_stream
 
-    def step(xs=None, outs=None):
-        for j, (cv, x, w, d, plan, out) in enumerate(items):
-            xp = xs[j].data_ptr() if xs is not None else x.data_ptr()
-            op = outs[j].data_ptr() if outs is not None else out.data_ptr()
-            st = fwd(xp, w.data_ptr(), op, d, dt_code, opts, ws.data_ptr(), ws.numel(), sptr)
+class Bench:
+    """One workload made resident on the device: inputs, outputs, plans and a
+    shared workspace, and the step that runs every conv of it once."""
+
+    def __init__(self, wl_name, algo, dev, stream):
+        import torch
+        from dense_convolution_nhwc_b200 import binding as B
+        self.B, self.torch = B, torch
+        self.desc, convs, self.dtype = workload(wl_name)
+        self.opts = B.make_options(algo)
+        self.dev, self.stream = dev, stream
+        self.sptr = stream.cuda_stream
+        self.items = []
+        ws_max = 0
+        local = dev.index or 0
+        for i, cv in enumerate(convs):
+            s = cv.shape
+            if cv.is3d:
+                x, w = synth.conv3d_inputs(s, cv.dtype, cv.dist, i, dev)
+                d = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+                plan = B.plan3d(d, cv.dtype, local, self.opts)
+                out = torch.empty((s.n, s.od, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
+            else:
+                x, w = synth.conv2d_inputs(s, cv.dtype, cv.dist, i, dev)
+                d = B.make_desc2d(s.n, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
+                plan = B.plan2d(d, cv.dtype, local, self.opts)
+                out = torch.empty((s.n, s.oh, s.ow, s.o), dtype=x.dtype, device=dev)
+            ws_max = max(ws_max, plan["workspace_bytes"])
+            self.items.append((cv, x, w, d, plan, out))
+        self.ws = torch.empty(max(ws_max, 256), dtype=torch.uint8, device=dev)
+        self.dt_code = B.DTYPE[self.dtype]
+        self.fwd = B.conv3d_forward if convs[0].is3d else B.conv2d_forward
+        self.total_flops = sum(cv.flops for cv, *_ in self.items)
+        self.in_bytes = sum(x.numel() * x.element_size() for _, x, _, _, _, _ in self.items)
+        self.flush = (torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+                      if self.in_bytes < 2 * L2_BYTES else None)
+        self.graph = None
+
+    def step(self, sptr=None):
+        sptr = sptr or self.sptr
+        for cv, x, w, d, plan, out in self.items:
+            st = self.fwd(x.data_ptr(), w.data_ptr(), out.data_ptr(), d, self.dt_code, self.opts,
+                          self.ws.data_ptr(), self.ws.numel(), sptr)
             if st != 0:
-                raise B.ConvError(st, cv.name)
+                raise self.B.ConvError(st, cv.name)
 
-    in_bytes = sum(x.numel() * x.element_size() for _, x, _, _, _, _ in items)
-    flush_needed = in_bytes < 2 * L2_BYTES
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush_needed else None
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert B.conv_check(sptr) == 0
-
-    run_step = step
-    graph = None
-    if args.graph:
-        g_stream = torch.cuda.Stream(dev)
-        g_stream.wait_stream(stream)
+    def capture(self):
+        """One step captured as a CUDA graph (removes host launch gaps)."""
+        torch = self.torch
+        g_stream = torch.cuda.Stream(self.dev)
+        g_stream.wait_stream(self.stream)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.stream(g_stream):
-            sptr_saved = sptr
-            sptr = g_stream.cuda_stream
             with torch.cuda.graph(graph, stream=g_stream):
-                step()
-            sptr = sptr_saved
-        stream.wait_stream(g_stream)
+                self.step(g_stream.cuda_stream)
+        self.stream.wait_stream(g_stream)
         torch.cuda.synchronize()
-        run_step = graph.replay
+        self.graph = graph
 
-    # timed region (device time of the steps; an L2 flush between steps is outside the events)
-    total_flops = sum(cv.flops for cv, *_ in items)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        B.conv_profile_begin()
-        for k in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            ev[k][0].record(stream)
-            run_step()
-            ev[k][1].record(stream)
+    def timed(self, steps, use_graph=False):
+        """Device time of `steps` steps, ms each (CUDA events on the launching
+        stream; an L2 flush between steps when the inputs fit in L2, outside
+        the events).  No profiling hook is active."""
+        torch = self.torch
+        run = self.graph.replay if use_graph else self.step
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for k in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            ev[k][0].record(self.stream)
+            run()
+            ev[k][1].record(self.stream)
         torch.cuda.synchronize()
-        prof = B.profile_end()
-    if graph is not None:
-        # graph replays record no per-kernel events: take the kernel breakdown from plain steps
-        B.conv_profile_begin()
-        for k in range(args.steps):
-            step()
-        torch.cuda.synchronize()
-        prof = B.profile_end()
-    barrier(world)
-    assert B.conv_check(sptr) == 0
-    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
-    ms = reduce_max(ms, world, dev)
-    value = world * total_flops / (ms * 1e-3) / 1e12
-    clocks = clk.summary()
+        return [a.elapsed_time(b) for a, b in ev]
 
-    # roofline of the dominant kernel (the one with the largest event time)
-    work = {}
-    for cv, x, w, d, plan, out in items:
-        for k, (f, b) in kernel_work(cv, plan).items():
-            f0, b0 = work.get(k, (0.0, 0.0))
-            work[k] = (f0 + f, b0 + b)
-    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
-        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    def kernel_split(self, steps):
+        """Per-kernel launches and event time from separate, profiled steps."""
+        B = self.B
+        B.conv_profile_begin()
+        for _ in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            self.step()
+        self.torch.cuda.synchronize()
+        return B.profile_end()
+
+    def work(self):
+        w = {}
+        for cv, x, wt, d, plan, out in self.items:
+            for k, (f, b) in kernel_work(cv, plan).items():
+                f0, b0 = w.get(k, (0.0, 0.0))
+                w[k] = (f0 + f, b0 + b)
+        return w
+
+    def per_conv_work(self, kernel):
+        return [kernel_work(cv, plan).get(kernel, (0.0, 0.0)) for cv, _, _, _, plan, _ in self.items]
+
+
+def fp32_peak(B, torch, peaks):
+    smax = peaks.get("sm_max_mhz", 1965.0)
+    derived = 148 * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
+    # measured: the library's FMA-chain probe (scalar FFMA and the packed two-lane FMA);
+    # the higher of the two is the CUDA cores' fp32 peak
+    rates = {}
+    for packed in (0, 1):
+        v = ctypes.c_double(0.0)
+        if B.conv_fp32_fma_rate(packed, v, torch.cuda.current_stream().cuda_stream) == 0:
+            rates["packed" if packed else "scalar"] = v.value
+    if rates:
+        return max(rates.values()), ("measured: fp32 FMA-chain probe in this run (scalar %.1f, packed %.1f TFLOP/s; "
+                                     "derived 148 SMs x 128 lanes x 2 x %.0f MHz = %.1f)" %
+                                     (rates.get("scalar", 0.0), rates.get("packed", 0.0), smax, derived))
+    return derived, f"derived: 148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"
+
+
+def kernels_and_roofline(bench, prof, steps, peaks, fp32_pk, wl_name=None):
+    """Per-kernel shares and the roofline of the dominant kernel."""
+    work = bench.work()
     kernels = {}
+    tot_all = max(1e-9, sum(t for _, t in prof.values()))
     for name, (launches, tot) in prof.items():
-        per_launch_ms = tot / max(launches, 1)
         f, b = work.get(name, (0.0, 0.0))
-        kernels[name] = {"launches_per_step": launches / args.steps, "ms_per_step": tot / args.steps,
-                         "share": tot / max(1e-9, sum(t for _, t in prof.values())),
-                         "flops_per_step": f, "bytes_per_step": b, "per_launch_ms": per_launch_ms}
+        kernels[name] = {"launches_per_step": launches / steps, "ms_per_step": tot / steps, "share": tot / tot_all,
+                         "flops_per_step": f, "bytes_per_step": b, "per_launch_ms": tot / max(launches, 1)}
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     kd = kernels[dom]
     bound = kernel_bound(dom)
-    launches_step = kd["launches_per_step"]
+    lps = kd["launches_per_step"]
+    hbm = peaks.get("hbm_gbs")
+    bf16 = peaks.get("bf16_tflops")
+    bf16_sus = peaks.get("bf16_tflops_sustained")
+    src_note = "measured (MEASURED_PEAKS.json)" if peaks else "fallback (profiling recipe: 6.65 TB/s, 1.59 PFLOP/s)"
+    extra = {}
     if bound == "hbm":
-        achieved = kd["bytes_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e9
-        peak = peaks.get("hbm_gbs", 6650.0)
-        unit, peak_src = "GB/s", "measured (MEASURED_PEAKS.json hbm_gbs)" if peaks else "fallback"
+        achieved = kd["bytes_per_step"] / lps / (kd["per_launch_ms"] * 1e-3) / 1e9
+        peak, unit, peak_src = hbm or 6650.0, "GB/s", f"HBM copy bandwidth, {src_note}"
     elif bound == "tensor":
-        achieved = kd["flops_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e12
-        peak = peaks.get("bf16_tflops", 1590.0)
-        unit, peak_src = "TFLOP/s", "measured burst bf16 (MEASURED_PEAKS.json); fp16 same nominal rate"
+        achieved = kd["flops_per_step"] / lps / (kd["per_launch_ms"] * 1e-3) / 1e12
+        peak, unit = bf16 or 1590.0, "TFLOP/s"
+        peak_src = f"dense bf16 burst, {src_note}; fp16 taken at the same nominal rate"
+        sus = bf16_sus or 1400.0
+        extra["frac_of_sustained"] = achieved / sus
+        extra["sustained_peak"] = sus
+        # the shape-bound: per conv, the kernel cannot beat max(flops / tensor peak, bytes / HBM)
+        ideal = sum(max(f / (peak * 1e12), b / ((hbm or 6650.0) * 1e9)) for f, b in bench.per_conv_work(dom))
+        if ideal > 0:
+            attainable = kd["flops_per_step"] / ideal / 1e12
+            extra["attainable"] = attainable
+            extra["frac_of_attainable"] = achieved / attainable
+            extra["attainable_note"] = "sum over convs of max(FLOPs / tensor peak, algorithmic bytes / HBM peak)"
     else:
-        achieved = kd["flops_per_step"] / launches_step / (kd["per_launch_ms"] * 1e-3) / 1e12
-        smax = peaks.get("sm_max_mhz", 1965.0)
-        derived = 148 * FP32_LANES_PER_SM * 2 * smax * 1e6 / 1e12
-        # measured: the library's FMA-chain probe (scalar FFMA and the packed two-lane FMA),
-        # after the timed region; the higher of the two is the CUDA cores' fp32 peak
-        rates = {}
-        for packed in (0, 1):
-            v = ctypes.c_double(0.0)
-            if B.conv_fp32_fma_rate(packed, v, torch.cuda.current_stream().cuda_stream) == 0:
-                rates["packed" if packed else "scalar"] = v.value
-        if rates:
-            peak = max(rates.values())
-            unit, peak_src = "TFLOP/s", ("measured: fp32 FMA-chain probe in this run (scalar %.1f, packed %.1f TFLOP/s; "
-                                         "derived 148 SMs x 128 lanes x 2 x %.0f MHz = %.1f)" %
-                                         (rates.get("scalar", 0.0), rates.get("packed", 0.0), smax, derived))
-        else:
-            peak = derived
-            unit, peak_src = "TFLOP/s", f"derived: 148 SMs x 128 FP32 lanes x 2 x {smax:.0f} MHz"
-    traffic_db = load_traffic()
-    tr = traffic_db.get(f"{args.workload}:{dom}")
+        achieved = kd["flops_per_step"] / lps / (kd["per_launch_ms"] * 1e-3) / 1e12
+        peak, peak_src = fp32_pk
+        unit = "TFLOP/s"
     traffic = None
-    if tr and tr.get("source_hash") == source_hash(dom):
-        traffic = tr.get("bytes_per_launch")
-    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-            "algorithmic_per_launch": (kd["bytes_per_step"] if bound == "hbm" else kd["flops_per_step"]) / launches_step}
-    gpu_launches = int(round(sum(l for l, _ in prof.values())))
+    if wl_name is not None:
+        tr = load_traffic().get(f"{wl_name}:{dom}")
+        if tr and tr.get("source_hash") == source_hash(dom):
+            traffic = tr.get("bytes_per_launch")
+    roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic, "peak_source": peak_src,
+            "algorithmic_per_launch": (kd["bytes_per_step"] if bound == "hbm" else kd["flops_per_step"]) / lps}
+    roof.update(extra)
+    return kernels, roof
+
+
+def per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, fp32_pk, min_steps):
+    import torch
+    bench = Bench(wl_name, algo, dev, stream)
+    for _ in range(3):
+        bench.step()
+    torch.cuda.synchronize()
+    one = statistics.median(bench.timed(3))
+    # enough steps that the clock record covers the timed region (>= ~0.4 s)
+    steps = int(min(2000, max(min_steps, math.ceil(400.0 / max(one, 1e-3)))))
+    entry = {"workload": bench.desc, "algo": algo, "dtype": bench.dtype, "convs": len(bench.items),
+             "flops_per_step": bench.total_flops}
+    barrier(world)
+    with ClockSampler(dev.index or 0) as clk:
+        ms_eager = statistics.median(bench.timed(steps))
+    entry["clocks"] = clk.summary()
+    ms_eager = reduce_max(ms_eager, world, dev)
+    entry["ms_issued"] = ms_eager
+    ms = ms_eager
+    if use_graph:
+        bench.capture()
+        for _ in range(3):
+            bench.graph.replay()
+        ms_graph = reduce_max(statistics.median(bench.timed(steps, use_graph=True)), world, dev)
+        entry["ms_graph"] = ms_graph
+        ms = ms_graph
+        entry["timing"] = "CUDA graph replay of one step (host launch gaps removed); ms_issued is call by call"
+    entry["ms"] = ms
+    entry["value"] = world * bench.total_flops / (ms * 1e-3) / 1e12
+    entry["unit"] = "TFLOP/s"
+    entry["steps"] = steps
+    prof = bench.kernel_split(min(steps, 20))
+    kernels, roof = kernels_and_roofline(bench, prof, min(steps, 20), peaks, fp32_pk)
+    entry["kernels"] = {k: {"share": v["share"], "ms_per_step": v["ms_per_step"],
+                            "launches_per_step": v["launches_per_step"]} for k, v in kernels.items()}
+    entry["roofline"] = roof
+    if bench.dtype != "f32":
+        entry["frac_of_bf16_peak"] = entry["value"] / (peaks.get("bf16_tflops") or 1590.0)
+    plans = {}
+    for cv, *_, plan, _ in bench.items:
+        k = f'{plan["algo"]}/{plan["engine"]}'
+        plans[k] = plans.get(k, 0) + 1
+    entry["plans"] = plans
+    entry["l2"] = ("L2 flushed between steps (outside the events)" if bench.flush is not None
+                   else f"inputs larger than L2 ({bench.in_bytes / 1e9:.2f} GB per step)")
+    del bench
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_headline(args, B, torch, dev, stream, world, rank, local, peaks):
+    """The headline workload: timed steps, kernel split, e2e and the CPU
+    baseline.  Returns the pieces of the JSON line; every device buffer of the
+    workload is released when it returns."""
+    bench = Bench(args.workload, args.algo, dev, stream)
+    desc, dtype, items = bench.desc, bench.dtype, bench.items
+    sptr = bench.sptr
+    for _ in range(args.warmup):
+        bench.step()
+    torch.cuda.synchronize()
+    assert B.conv_check(sptr) == 0
+    if args.graph:
+        bench.capture()
+
+    # timed region: no profiling hook, only the events around each step
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = bench.timed(args.steps, use_graph=args.graph)
+    barrier(world)
+    assert B.conv_check(sptr) == 0
+    ms = sum(times) / args.steps
+    ms = reduce_max(ms, world, dev)
+    value = world * bench.total_flops / (ms * 1e-3) / 1e12
+    clocks = clk.summary()
+
+    # per-kernel split from separate, profiled steps (outside the timed region)
+    prof_steps = min(args.steps, 10)
+    prof = bench.kernel_split(prof_steps)
+    fp32_pk = fp32_peak(B, torch, peaks)
+    kernels, roof = kernels_and_roofline(bench, prof, prof_steps, peaks, fp32_pk, args.workload)
+    launches_per_step = sum(l for l, _ in prof.values()) / prof_steps
+    gpu_launches = int(round(launches_per_step * args.steps))
+    fwd, opts, dt_code, ws = bench.fwd, bench.opts, bench.dt_code, bench.ws
+    total_flops = bench.total_flops
 
     # e2e through the C ABI with host buffers.  Images are independent, so each
     # conv's batch is cut into chunks that flow through three streams: the
@@ -663,72 +774,143 @@ def main():
         r, cores, sample, _ = oracle_sample_rate(cv, xh, w.cpu(), 15.0)
         cpu = {"value": r, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
 
+    plan0 = items[0][4]
+    per_conv_lines = []
+    if args.per_conv and rank == 0:
+        per_conv_lines = per_conv_report(bench, peaks)
+    config = {"workload": desc, "plan": {k: plan0[k] for k in ("algo", "engine", "winograd_m", "batch_tile",
+                                                               "num_batch_tiles", "tile_n")},
+              "convs_per_step": len(items), "flops_per_step": total_flops,
+              "l2": "L2 flushed between steps (outside the events)" if bench.flush is not None
+              else f"inputs larger than L2 ({bench.in_bytes / 1e9:.2f} GB per step)",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+              "cuda_graph": bool(args.graph)}
+
+    return {"value": value, "ms": ms, "dtype": dtype, "desc": desc, "config": config, "roof": roof,
+            "kernels": kernels, "clocks": clocks, "gpu_launches": gpu_launches,
+            "launches_per_step": launches_per_step, "e2e": e2e, "cpu": cpu, "fp32_pk": fp32_pk,
+            "per_conv_lines": per_conv_lines, "sptr": sptr}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="winograd_f32")
+    ap.add_argument("--algo", default="auto", choices=["auto", "implicit", "winograd", "direct"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-config block")
+    ap.add_argument("--per-config-only", default="", help="comma-separated per-config keys to run (default: all)")
+    ap.add_argument("--per-conv", action="store_true", help="also print one line per conv of the workload")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step as a CUDA graph and time its replays (removes host launch gaps)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, args.workload)
+        return
+
+    import torch
+    from dense_convolution_nhwc_b200 import binding as B
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+
+    h = run_headline(args, B, torch, dev, stream, world, rank, local, peaks)
+    torch.cuda.empty_cache()
+    value, ms, dtype, config, roof, kernels, clocks = (h["value"], h["ms"], h["dtype"], h["config"], h["roof"],
+                                                       h["kernels"], h["clocks"])
+    gpu_launches, launches_per_step, e2e, cpu, fp32_pk = (h["gpu_launches"], h["launches_per_step"], h["e2e"],
+                                                          h["cpu"], h["fp32_pk"])
+    per_conv_lines, sptr = h["per_conv_lines"], h["sptr"]
+
+    per_config = None
+    if not args.no_per_config:
+        only = {k for k in args.per_config_only.split(",") if k}
+        per_config = {}
+        for key, wl, algo, use_graph in PER_CONFIG:
+            if only and key not in only:
+                continue
+            try:
+                per_config[key] = per_config_entry(key, wl, algo, use_graph, dev, stream, world, peaks, fp32_pk,
+                                                   min_steps=10)
+            except Exception as exc:      # report, never hide, a failed entry
+                per_config[key] = {"error": f"{type(exc).__name__}: {exc}"}
+        assert B.conv_check(sptr) == 0
+
     if rank == 0:
-        plan0 = items[0][4]
         line = {
             "metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": (value / PAGES_NUMBER[args.workload]) if args.workload in PAGES_NUMBER else None,
-            "dtype": dtype, "data": "synthetic",
-            "config": {"workload": desc, "plan": {k: plan0[k] for k in ("algo", "engine", "winograd_m", "batch_tile",
-                                                                          "num_batch_tiles", "tile_n")},
-                       "convs_per_step": len(items), "flops_per_step": total_flops,
-                       "l2": "L2 flushed between steps (outside the events)" if flush_needed
-                       else f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB per step)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "cuda_graph": bool(args.graph)},
-            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": gpu_launches * 1,
-            "gpu_launches_per_step": gpu_launches / args.steps,
+            "dtype": dtype, "data": "synthetic", "config": config,
+            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": gpu_launches,
+            "gpu_launches_per_step": launches_per_step,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         if args.workload in PAGES_NUMBER:
             line["vs_baseline_note"] = "pages' 310 ms on an M2 Max for the same workload (context, other hardware)"
+        if per_config is not None:
+            line["per_config"] = per_config
         print(json.dumps(line))
-        if args.per_conv:
-            for cv, x, w, d, plan, out in items:
-                evs = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                fwd_one = lambda: fwd(x.data_ptr(), w.data_ptr(), out.data_ptr(), d, dt_code, opts,
-                                      ws.data_ptr(), ws.numel(), sptr)
-                for _ in range(3):
-                    fwd_one()
-                reps = 10
-                if flush is not None:
-                    times = []
-                    for _ in range(reps):
-                        flush.zero_()
-                        evs[0].record(stream)
-                        fwd_one()
-                        evs[1].record(stream)
-                        torch.cuda.synchronize()
-                        times.append(evs[0].elapsed_time(evs[1]))
-                    t = statistics.median(times)
-                else:
-                    evs[0].record(stream)
-                    for _ in range(reps):
-                        fwd_one()
-                    evs[1].record(stream)
-                    torch.cuda.synchronize()
-                    t = evs[0].elapsed_time(evs[1]) / reps
-                B.conv_profile_begin()
-                for _ in range(reps):
-                    fwd_one()
-                torch.cuda.synchronize()
-                kp = B.profile_end()
-                kw = kernel_work(cv, plan)
-                ker = {}
-                for kn, (nl, tot) in kp.items():
-                    kms = tot / reps
-                    f, b = kw.get(kn, (0.0, 0.0))
-                    ker[kn] = {"ms": kms, "tflops": f / (kms * 1e-3) / 1e12 if f else None,
-                               "gbs": b / (kms * 1e-3) / 1e9 if b else None}
-                print(json.dumps({"conv": cv.name, "dtype": cv.dtype, "algo": plan["algo"], "engine": plan["engine"],
-                                  "tile_n": plan["tile_n"], "ms": t, "tflops": cv.flops / (t * 1e-3) / 1e12,
-                                  "frac_of_bf16_peak": cv.flops / (t * 1e-3) / 1e12 / peaks.get("bf16_tflops", 1590.0),
-                                  "kernels": ker}))
+        for l in per_conv_lines:
+            print(json.dumps(l))
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def per_conv_report(bench, peaks):
+    """One line per conv of the workload: its own event time and kernel split."""
+    import torch
+    B = bench.B
+    lines = []
+    evs = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    for cv, x, w, d, plan, out in bench.items:
+        def fwd_one():
+            st = bench.fwd(x.data_ptr(), w.data_ptr(), out.data_ptr(), d, bench.dt_code, bench.opts,
+                           bench.ws.data_ptr(), bench.ws.numel(), bench.sptr)
+            if st != 0:
+                raise B.ConvError(st, cv.name)
+        for _ in range(3):
+            fwd_one()
+        reps = 10
+        times = []
+        for _ in range(reps):
+            if bench.flush is not None:
+                bench.flush.zero_()
+            evs[0].record(bench.stream)
+            fwd_one()
+            evs[1].record(bench.stream)
+            torch.cuda.synchronize()
+            times.append(evs[0].elapsed_time(evs[1]))
+        t = statistics.median(times)
+        B.conv_profile_begin()
+        for _ in range(reps):
+            fwd_one()
+        torch.cuda.synchronize()
+        kp = B.profile_end()
+        kw = kernel_work(cv, plan)
+        ker = {}
+        for kn, (nl, tot) in kp.items():
+            kms = tot / reps
+            f, b = kw.get(kn, (0.0, 0.0))
+            ker[kn] = {"ms": kms, "tflops": f / (kms * 1e-3) / 1e12 if f else None,
+                       "gbs": b / (kms * 1e-3) / 1e9 if b else None}
+        lines.append({"conv": cv.name, "dtype": cv.dtype, "algo": plan["algo"], "engine": plan["engine"],
+                      "tile_n": plan["tile_n"], "k_split": plan["k_split"], "ms": t,
+                      "tflops": cv.flops / (t * 1e-3) / 1e12,
+                      "frac_of_bf16_peak": cv.flops / (t * 1e-3) / 1e12 / (peaks.get("bf16_tflops") or 1590.0),
+                      "kernels": ker})
+    return lines
 
 
 if __name__ == "__main__":

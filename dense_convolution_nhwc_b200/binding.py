@@ -307,6 +307,47 @@ def _check(x, name):
         raise ValueError(f"{name} must be contiguous (NHWC / OHWI)")
 
 
+def _check_out(out, shape, like):
+    """A caller's out= must be exactly the tensor the library will write: the C
+    ABI sees only a pointer, so a wrong shape, dtype, device or stride here
+    would become an out-of-bounds device write.  Raises before any launch."""
+    torch = _torch()
+    if not isinstance(out, torch.Tensor):
+        raise ValueError(f"out must be a torch tensor, got {type(out).__name__}")
+    if not out.is_cuda or out.device != like.device:
+        raise ValueError(f"out is on {out.device}, the input on {like.device}")
+    if out.dtype != like.dtype:
+        raise ValueError(f"out has dtype {out.dtype}, the input {like.dtype}")
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out has shape {tuple(out.shape)}, the conv writes {tuple(shape)}")
+    if not out.is_contiguous():
+        raise ValueError("out must be contiguous (NHWC)")
+
+
+def _check_workspace(ws, need, like):
+    """A caller's workspace= must sit on the input's device, be contiguous and
+    hold at least the bytes the plan asks for.  Raises before any launch."""
+    torch = _torch()
+    if not isinstance(ws, torch.Tensor):
+        raise ValueError(f"workspace must be a torch tensor, got {type(ws).__name__}")
+    if not ws.is_cuda or ws.device != like.device:
+        raise ValueError(f"workspace is on {ws.device}, the input on {like.device}")
+    if not ws.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    have = ws.numel() * ws.element_size()
+    if have < need:
+        raise ValueError(f"workspace holds {have} bytes, the plan needs {need}")
+
+
+def _check_pair(x, w):
+    _check(x, "x")
+    _check(w, "w")
+    if x.dtype != w.dtype:
+        raise TypeError("x and w must share a dtype")
+    if x.device != w.device:
+        raise ValueError(f"x is on {x.device}, w on {w.device}")
+
+
 def plan2d(desc: Conv2dDesc, dtype: str, device: int = 0, options: Optional[ConvOptions] = None) -> dict:
     p = ConvPlan()
     st = conv2d_plan(desc, DTYPE[dtype], device, options, p)
@@ -327,10 +368,7 @@ def conv2d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
            workspace=None):
     """NHWC conv2d: x [N,H,W,C], w [O,KH,KW,C] -> [N,OH,OW,O] on x's device."""
     torch = _torch()
-    _check(x, "x")
-    _check(w, "w")
-    if x.dtype != w.dtype:
-        raise TypeError("x and w must share a dtype")
+    _check_pair(x, w)
     N, H, W, C = x.shape
     O, KH, KW, C2 = w.shape
     if C2 != C:
@@ -348,9 +386,13 @@ def conv2d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
         OW = (W + 2 * p[1] - d[1] * (KW - 1) - 1) // s[1] + 1
         if out is None:
             out = torch.empty((N, OH, OW, O), dtype=x.dtype, device=x.device)
+        else:
+            _check_out(out, (N, OH, OW, O), x)
         ws_bytes = int(plan.workspace_bytes)
         if workspace is None and ws_bytes:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        elif workspace is not None:
+            _check_workspace(workspace, ws_bytes, x)
         ws_ptr = workspace.data_ptr() if workspace is not None else 0
         ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
         stream = torch.cuda.current_stream(x.device).cuda_stream
@@ -364,10 +406,7 @@ def conv1d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
            workspace=None):
     """NLC conv1d: x [N,L,C], w [O,K,C] -> [N,OL,O] on x's device (through conv1d_forward)."""
     torch = _torch()
-    _check(x, "x")
-    _check(w, "w")
-    if x.dtype != w.dtype:
-        raise TypeError("x and w must share a dtype")
+    _check_pair(x, w)
     N, L, C = x.shape
     O, K, C2 = w.shape
     if C2 != C:
@@ -383,9 +422,13 @@ def conv1d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
         OL = (L + 2 * padding - dilation * (K - 1) - 1) // stride + 1
         if out is None:
             out = torch.empty((N, OL, O), dtype=x.dtype, device=x.device)
+        else:
+            _check_out(out, (N, OL, O), x)
         ws_bytes = int(plan.workspace_bytes)
         if workspace is None and ws_bytes:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        elif workspace is not None:
+            _check_workspace(workspace, ws_bytes, x)
         ws_ptr = workspace.data_ptr() if workspace is not None else 0
         ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
         stream = torch.cuda.current_stream(x.device).cuda_stream
@@ -399,10 +442,7 @@ def conv3d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
            workspace=None):
     """NDHWC conv3d: x [N,D,H,W,C], w [O,KD,KH,KW,C] -> [N,OD,OH,OW,O]."""
     torch = _torch()
-    _check(x, "x")
-    _check(w, "w")
-    if x.dtype != w.dtype:
-        raise TypeError("x and w must share a dtype")
+    _check_pair(x, w)
     N, D, H, W, C = x.shape
     O, KD, KH, KW, C2 = w.shape
     if C2 != C:
@@ -420,9 +460,13 @@ def conv3d(x, w, stride=1, padding=0, dilation=1, options: Optional[ConvOptions]
         OD, OH, OW = [(i + 2 * p[a] - d[a] * (k - 1) - 1) // s[a] + 1 for a, (i, k) in enumerate(dims)]
         if out is None:
             out = torch.empty((N, OD, OH, OW, O), dtype=x.dtype, device=x.device)
+        else:
+            _check_out(out, (N, OD, OH, OW, O), x)
         ws_bytes = int(plan.workspace_bytes)
         if workspace is None and ws_bytes:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+        elif workspace is not None:
+            _check_workspace(workspace, ws_bytes, x)
         ws_ptr = workspace.data_ptr() if workspace is not None else 0
         ws_n = workspace.numel() * workspace.element_size() if workspace is not None else 0
         stream = torch.cuda.current_stream(x.device).cuda_stream

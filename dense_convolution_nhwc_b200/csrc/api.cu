@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -41,27 +42,34 @@ struct DeviceState {
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
+// Constant properties are cached per device.  The error word's device address
+// is looked up again on every call made with that device current: a context
+// torn down and re-created (cudaDeviceReset) gives the word a new address, and
+// a cached one would then point at memory the device no longer maps.  The
+// lookup allocates nothing.
 conv_status_t device_state(int dev, DeviceState** out) {
   if (dev < 0 || dev >= kMaxDevices) return CONV_ERR_INVALID;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DeviceState& d = g_dev[dev];
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return CONV_ERR_CUDA;
   if (!d.ready) {
-    int cur = -1;
-    if (cudaGetDevice(&cur) != cudaSuccess) return CONV_ERR_CUDA;
     cudaDeviceProp p;
     if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return CONV_ERR_CUDA;
     d.props.sm_count = p.multiProcessorCount;
     d.props.cc_major = p.major;
     d.props.cc_minor = p.minor;
     d.props.total_global_mem = (unsigned long long)p.totalGlobalMem;
+    d.ready = true;
+  }
+  if (cur == dev || !d.err_word) {
     if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return CONV_ERR_CUDA;
     void* addr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&addr, g_error_word);
-    if (e == cudaSuccess) e = cudaMemset(addr, 0, sizeof(int));
+    if (e == cudaSuccess && addr != d.err_word) e = cudaMemset(addr, 0, sizeof(int));   // a new context
     if (cur != dev) cudaSetDevice(cur);
     if (e != cudaSuccess) return CONV_ERR_CUDA;
     d.err_word = static_cast<int*>(addr);
-    d.ready = true;
   }
   *out = &d;
   return CONV_OK;
@@ -378,6 +386,31 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->k_split = s.ksplit;
   plan->taps = taps;
   plan->workspace_bytes = ws;
+}
+
+// B200CONV_LOG=1: one line per forward call on stderr with the plan that runs
+// (read on every call, like the other environment hooks).
+bool log_enabled() {
+  const char* v = std::getenv("B200CONV_LOG");
+  return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+const char* dtype_name(conv_dtype_t t) { return t == CONV_F32 ? "f32" : (t == CONV_F16 ? "f16" : "bf16"); }
+const char* algo_name(conv_algo_t a) {
+  switch (a) {
+    case CONV_ALGO_IMPLICIT_GEMM: return "implicit";
+    case CONV_ALGO_WINOGRAD: return "winograd";
+    case CONV_ALGO_DIRECT: return "direct";
+    default: return "auto";
+  }
+}
+
+void log_plan(const char* op, const char* shape, conv_dtype_t dt, const Sel& s, const char* path, size_t ws) {
+  std::fprintf(stderr,
+               "b200conv: %s %s %s -> algo=%s engine=%s path=%s tile=%dx%d winograd_m=%d batch_tile=%d "
+               "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d workspace=%zu\n",
+               op, shape, dtype_name(dt), algo_name(s.algo), s.engine == CONV_ENGINE_TCGEN05 ? "tcgen05" : "simt",
+               path, s.tile_m, s.tile_n, s.wino_m, s.nb, s.ntiles, s.cpad, s.wpack ? 1 : 0, s.ksplit, ws);
 }
 
 // ------------------------------- execution -----------------------------------
@@ -842,6 +875,12 @@ conv_status_t conv2d_forward(const void* in, const void* w, void* out, const con
   if (workspace_bytes < s.ws || (s.ws > 0 && !workspace)) return CONV_ERR_WORKSPACE;
   if (s.ws > 0 && !aligned256(workspace)) return CONV_ERR_ALIGNMENT;
   if (overlaps(out, out_bytes, workspace, s.ws)) return CONV_ERR_INVALID;
+  if (log_enabled()) {
+    char shape[192];
+    std::snprintf(shape, sizeof shape, "n%d %dx%d %d->%d k%dx%d s%d,%d p%d,%d d%d,%d", g.n, g.h, g.w, g.c, g.o, g.kh,
+                  g.kw, g.sh, g.sw, g.ph, g.pw, g.dh, g.dw);
+    log_plan("conv2d", shape, dtype, s, "2d", s.ws);
+  }
   return run2d(in, w, out, g, dtype, s, workspace, *d, static_cast<cudaStream_t>(stream));
 }
 
@@ -930,18 +969,32 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
     return CONV_ERR_INVALID;
 
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
-  if (path == P3_WINO3D) return run3d_winograd(in, w, out, geom3_of(desc, od, g2), dtype, s, workspace, *d, st_);
+  const Geom3 g3 = geom3_of(desc, od, g2);
+  const char* path_name = path == P3_WINO3D ? "winograd3d" : "depth_taps";
   if (path == P3_NATIVE) {
-    const Geom3 g3 = geom3_of(desc, od, g2);
     if (tc_conv3d_supported(g3, dtype, in, w)) {
-      ProfScope ps(K_TC_CONV3D, st_);
-      return cuda_status(launch_tc_conv3d(in, w, out, g3, dtype, s.tile_n, d->props.sm_count, d->err_word, st_));
+      path_name = "native3d";
+    } else {
+      // misaligned pointers: depth taps on the any-alignment path
+      conv_options_t o2 = effective_options(opts);
+      o2.algo = CONV_ALGO_DIRECT;
+      st = select2d(g2, dtype, d->props, o2, &s);
+      if (st != CONV_OK) return st;
+      path = P3_TAPS;
     }
-    // misaligned pointers: depth taps on the any-alignment path
-    conv_options_t o2 = effective_options(opts);
-    o2.algo = CONV_ALGO_DIRECT;
-    st = select2d(g2, dtype, d->props, o2, &s);
-    if (st != CONV_OK) return st;
+  }
+  if (log_enabled()) {
+    char shape[224];
+    std::snprintf(shape, sizeof shape, "n%d %dx%dx%d %d->%d k%dx%dx%d s%d,%d,%d p%d,%d,%d d%d,%d,%d", desc->n, desc->d,
+                  desc->h, desc->w, desc->c, desc->o, desc->kd, desc->kh, desc->kw, desc->stride[0], desc->stride[1],
+                  desc->stride[2], desc->pad[0], desc->pad[1], desc->pad[2], desc->dilation[0], desc->dilation[1],
+                  desc->dilation[2]);
+    log_plan("conv3d", shape, dtype, s, path_name, ws);
+  }
+  if (path == P3_WINO3D) return run3d_winograd(in, w, out, g3, dtype, s, workspace, *d, st_);
+  if (path == P3_NATIVE) {
+    ProfScope ps(K_TC_CONV3D, st_);
+    return cuda_status(launch_tc_conv3d(in, w, out, g3, dtype, s.tile_n, d->props.sm_count, d->err_word, st_));
   }
   Tap taps[1024];
   if (desc->kd > 1024) return CONV_ERR_UNSUPPORTED;

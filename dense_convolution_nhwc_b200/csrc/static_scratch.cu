@@ -22,33 +22,25 @@
 // CONV_ERR_WORKSPACE before anything is launched.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "internal.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;
 
 // Host code must never use this name as a device address: it is a host-side
 // stand-in.  The device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-void* g_scratch_addr[kMaxDevices];
-std::mutex g_scratch_mu;
-
-// Once per device, with that device current: look up the array's device
-// address.  This is the first call's set-up; it makes no allocation.
-conv_status_t scratch_address(int dev, void** out) {
-  if (dev < 0 || dev >= kMaxDevices) return CONV_ERR_INVALID;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return CONV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+// The array's device address in the current device's context.  It is looked
+// up on every call rather than cached: a context torn down and re-created
+// (cudaDeviceReset) places the array at a new address, and a cached one would
+// hand the kernels memory the device no longer maps.  The lookup allocates
+// nothing; the first one on a device loads the library's device code there.
+conv_status_t scratch_address(void** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return CONV_ERR_CUDA;
+  *out = p;
   return CONV_OK;
 }
 
@@ -61,7 +53,7 @@ extern "C" conv_status_t conv2d_forward_winograd_static(const void* in, const vo
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return CONV_ERR_CUDA;
   void* scratch = nullptr;
-  conv_status_t st = scratch_address(dev, &scratch);
+  conv_status_t st = scratch_address(&scratch);
   if (st != CONV_OK) return st;
 
   // Is the shape one the Winograd path runs at all (3x3, stride 1, dilation 1)?
@@ -71,23 +63,24 @@ extern "C" conv_status_t conv2d_forward_winograd_static(const void* in, const vo
   if (st != CONV_OK) return st;
   if (desc->n == 0) return CONV_OK;
 
-  // Largest batch tile whose scratch (filter + tile buffers) fits the array:
-  // start from the tile the array's size allows for the transform buffers and
-  // shrink it until the filter fits beside it.  Forcing the tile size keeps
-  // small tiles on the Winograd path.
+  // The largest batch tile whose scratch (transformed filter + the tile's
+  // transform buffers) fits the array, by bisection over the forced tile size
+  // (the scratch grows with the tile).  Forcing the tile keeps small tiles on
+  // the Winograd path.
   o.winograd_budget_bytes = (long long)kStaticScratchBytes;
-  o.winograd_tile_batch = desc->n;
-  for (int i = 0; i <= desc->n + 1; ++i) {
-    st = conv2d_plan(desc, dtype, dev, &o, &plan);
-    if (st == CONV_ERR_UNSUPPORTED) return CONV_ERR_WORKSPACE;   // not even one image fits
-    if (st != CONV_OK) return st;
-    if (plan.workspace_bytes <= kStaticScratchBytes) break;
-    if (plan.batch_tile <= 1) return CONV_ERR_WORKSPACE;
-    // drop at least one image; per-image share estimated from the plan
-    const double per_img = (double)plan.workspace_bytes / plan.batch_tile;
-    int drop = (int)((double)(plan.workspace_bytes - kStaticScratchBytes) / per_img) + 1;
-    o.winograd_tile_batch = plan.batch_tile - drop > 1 ? plan.batch_tile - drop : 1;
+  auto fits = [&](int tile, conv_plan_t* p) {
+    o.winograd_tile_batch = tile;
+    return conv2d_plan(desc, dtype, dev, &o, p) == CONV_OK && p->algo == CONV_ALGO_WINOGRAD &&
+           p->workspace_bytes <= kStaticScratchBytes;
+  };
+  if (!fits(1, &plan)) return CONV_ERR_WORKSPACE;   // not even one image fits
+  int lo = 1, hi = desc->n;                          // fits(lo) holds
+  while (lo < hi) {
+    const int mid = lo + (hi - lo + 1) / 2;
+    conv_plan_t p{};
+    if (fits(mid, &p)) lo = mid;
+    else hi = mid - 1;
   }
-  if (plan.algo != CONV_ALGO_WINOGRAD || plan.workspace_bytes > kStaticScratchBytes) return CONV_ERR_WORKSPACE;
+  if (!fits(lo, &plan)) return CONV_ERR_WORKSPACE;
   return conv2d_forward(in, w, out, desc, dtype, &o, scratch, kStaticScratchBytes, stream);
 }

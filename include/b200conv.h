@@ -119,7 +119,10 @@ typedef struct {
  *   B200CONV_ALGO=auto|implicit|winograd|direct
  *   B200CONV_WINOGRAD_WORKSPACE_BYTES=<bytes>   replaces the Winograd scratch budget
  *   B200CONV_WINOGRAD_TILE_BATCH=<images>       forces the batch-tile size (capped by the budget)
- * A non-NULL options struct ignores the environment.
+ * A non-NULL options struct ignores the environment.  Independently of the
+ * options, B200CONV_LOG=1 makes every conv*_forward call print the plan it
+ * runs (algorithm, engine, path, tile, Winograd m and batch tile, channel pad,
+ * K split, workspace bytes) as one line on stderr.
  */
 typedef struct {
     conv_algo_t algo;                     /* CONV_ALGO_AUTO: let the selector choose */
@@ -280,8 +283,11 @@ B200CONV_API conv_status_t conv_check(void *stream);
  * image's transform buffers exceed 64 MiB is rejected with CONV_ERR_WORKSPACE
  * and nothing is launched.  Output equals conv2d_forward with
  * CONV_ALGO_WINOGRAD at the same tile size.  No cudaMalloc or cudaFree is
- * called.  The first call on each device looks up the array's address; make
- * that first call before any stream capture.  All calls share the array and
+ * called.  Every call looks up the array's address in the current device's
+ * context (a lookup, not an allocation), so a context re-created after
+ * cudaDeviceReset is followed; the first call on a device also loads the
+ * library's device code there, so make that first call before any stream
+ * capture.  All calls share the array and
  * it keeps the last call's contents (nothing needs clearing); calls whose work
  * overlaps on the GPU race on it.
  */

@@ -37,12 +37,66 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     return e
 
 
-def run_conv2d(x, w, shape: synth.Conv2dShape, options=None, poison=True):
-    out = torch.full((shape.n, shape.oh, shape.ow, shape.o), float("nan"), dtype=x.dtype, device=x.device) \
-        if poison else None
-    out = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation, options=options, out=out)
+GUARD_BYTES = 4096          # canary band on each side of out and of the workspace
+GUARD_VALUE = 0x5B          # a byte pattern no kernel writes by accident (not 0, not a NaN half)
+
+
+class Guarded:
+    """A device buffer of `nbytes` between two canary bands.  The inner
+    region starts 4096 bytes into a fresh allocation (so it keeps the
+    allocator's 256-byte alignment) and the upper band starts right at its
+    last byte, so any write past either end lands in a band."""
+
+    def __init__(self, nbytes: int, device):
+        self.nbytes = int(nbytes)
+        self.buf = torch.full((GUARD_BYTES + self.nbytes + GUARD_BYTES,), GUARD_VALUE, dtype=torch.uint8,
+                              device=device)
+
+    def inner(self) -> torch.Tensor:
+        return self.buf[GUARD_BYTES:GUARD_BYTES + self.nbytes]
+
+    def tensor(self, shape, dtype) -> torch.Tensor:
+        return self.inner().view(dtype).view(shape)
+
+    def assert_intact(self, what: str):
+        lo = self.buf[:GUARD_BYTES]
+        hi = self.buf[GUARD_BYTES + self.nbytes:]
+        bad_lo = int((lo != GUARD_VALUE).sum())
+        bad_hi = int((hi != GUARD_VALUE).sum())
+        assert bad_lo == 0 and bad_hi == 0, \
+            f"{what}: write outside the buffer ({bad_lo} bytes below, {bad_hi} bytes above)"
+
+
+def guarded_output(shape, dtype, device):
+    """A NaN-poisoned output tensor inside canary bands."""
+    esz = torch.empty((), dtype=dtype).element_size()
+    g = Guarded(int(np.prod(shape)) * esz, device)
+    out = g.tensor(shape, dtype)
+    out.fill_(float("nan"))
+    return g, out
+
+
+def guarded_workspace(nbytes: int, device):
+    """The plan's workspace, exactly its size, inside canary bands (None if the plan needs none)."""
+    return Guarded(nbytes, device) if nbytes else None
+
+
+def run_conv2d(x, w, shape: synth.Conv2dShape, options=None):
+    """Run through the C ABI with a NaN-poisoned output and the exact workspace
+    the plan asks for, both inside canary bands checked after the call."""
+    desc = B.make_desc2d(shape.n, shape.h, shape.w, shape.c, shape.o, shape.kh, shape.kw, shape.stride, shape.pad,
+                         shape.dilation)
+    dt = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[x.dtype]
+    plan = B.plan2d(desc, dt, x.device.index or 0, options)
+    g_out, out = guarded_output((shape.n, shape.oh, shape.ow, shape.o), x.dtype, x.device)
+    g_ws = guarded_workspace(plan["workspace_bytes"], x.device)
+    out = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation, options=options, out=out,
+                   workspace=g_ws.inner() if g_ws else None)
     torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    g_out.assert_intact(f"{shape.name()} out")
+    if g_ws:
+        g_ws.assert_intact(f"{shape.name()} workspace")
     return out
 
 

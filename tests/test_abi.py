@@ -328,3 +328,21 @@ def test_split_k_for_small_m_long_k():
     # Winograd plans never split (bit identity of batch tiling)
     st, p = plan2d(synth.WINOGRAD_F32)
     assert p["algo"] == "winograd" and p["k_split"] == 1
+
+
+def test_binding_out_checks_need_no_gpu():
+    """The out= / workspace= checks of the torch conveniences reject host
+    tensors and non-tensors without touching a device."""
+    import torch
+    x = torch.zeros(2, 3)
+    for bad in (None, 3, "out"):
+        if bad is None:
+            continue
+        with pytest.raises(ValueError):
+            B._check_out(bad, (2, 3), x)
+        with pytest.raises(ValueError):
+            B._check_workspace(bad, 16, x)
+    with pytest.raises(ValueError):
+        B._check_out(torch.zeros(2, 3), (2, 3), x)        # host memory is never a valid out
+    with pytest.raises(ValueError):
+        B._check_workspace(torch.zeros(64, dtype=torch.uint8), 16, x)

@@ -87,3 +87,23 @@ def test_conv3d_depth_taps_count_every_tap():
     out_b = s.od * s.oh * s.ow * s.o * 2
     tap_b = (s.od * s.h * s.w * s.c + s.o * 9 * s.c + s.od * s.oh * s.ow * s.o) * 2   # frames in, slice, out
     assert w["tc_conv"][1] == 3 * tap_b + 2 * out_b     # taps 2 and 3 also read the output they add into
+
+
+def test_per_config_block_covers_every_config():
+    """The bench's per-config block measures configs 1, 3, 4 and 5 beside the
+    config-2 headline, every dtype the configs name, and every workload it
+    names resolves (no device needed)."""
+    keys = [k for k, *_ in bench.PER_CONFIG]
+    for cfg in ("config1_", "config3_", "config4_", "config5_"):
+        assert any(k.startswith(cfg) for k in keys), cfg
+    seen = set()
+    for key, wl, algo, _ in bench.PER_CONFIG:
+        desc, convs, dt = bench.workload(wl)
+        assert convs and algo in ("auto", "implicit", "winograd", "direct")
+        seen.add((key.split("_")[0], dt))
+    assert {("config3", "f16"), ("config3", "bf16"), ("config4", "f16"), ("config4", "bf16"),
+            ("config5", "bf16"), ("config1", "f32")} <= seen
+    # the wide-channel members: C_out >= 512 and M >= 16384, stride 1, dilation 1
+    _, convs, _ = bench.workload("wide_bf16")
+    assert all(c.shape.o >= 512 and c.shape.n * c.shape.oh * c.shape.ow >= 16384 for c in convs)
+    assert all(c.shape.stride == (1, 1) and c.shape.dilation == (1, 1) for c in convs)

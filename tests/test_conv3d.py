@@ -20,16 +20,26 @@ import torch
 import oracle
 from dense_convolution_nhwc_b200 import binding as B
 from dense_convolution_nhwc_b200 import synth
-from tests.gpu_util import TOL, as_f64, assert_close
+from tests.gpu_util import TOL, as_f64, assert_close, guarded_output, guarded_workspace
 
 pytestmark = pytest.mark.gpu
 
 
 def run3d(x, w, s, options=None):
-    out = torch.full((s.n, s.od, s.oh, s.ow, s.o), float("nan"), dtype=x.dtype, device=x.device)
-    out = B.conv3d(x, w, s.stride, s.pad, s.dilation, options=options, out=out)
+    """Through the C ABI with a NaN-poisoned output and the plan's exact
+    workspace, both inside canary bands that must stay untouched."""
+    desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
+    dt = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[x.dtype]
+    plan = B.plan3d(desc, dt, x.device.index or 0, options)
+    g_out, out = guarded_output((s.n, s.od, s.oh, s.ow, s.o), x.dtype, x.device)
+    g_ws = guarded_workspace(plan["workspace_bytes"], x.device)
+    out = B.conv3d(x, w, s.stride, s.pad, s.dilation, options=options, out=out,
+                   workspace=g_ws.inner() if g_ws else None)
     torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    g_out.assert_intact(f"{s.name()} out")
+    if g_ws:
+        g_ws.assert_intact(f"{s.name()} workspace")
     return out
 
 
@@ -73,7 +83,7 @@ FALLBACK_CASES = [
 ]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("s", FALLBACK_CASES, ids=lambda s: s.name())
 def test_generalised_taps(s, dtype):
     check3d(s, dtype)
@@ -126,7 +136,7 @@ def test_winograd_taps_accumulate_equal_manual_loop(dtype):
 
 @pytest.mark.parametrize("s", synth.CONV3D_TAPS, ids=lambda s: s.name())
 def test_workload_shapes_sampled(s):
-    check3d(s, "bf16", sample=2048)
+    check3d(s, "bf16", sample=4096)
 
 
 def test_accumulate_rounds_once_per_add():
@@ -242,4 +252,4 @@ def test_winograd3d_unit_tiling_is_bit_identical(dtype):
 def test_workload_shapes_f32_sampled(s):
     """The conv3d workload in fp32: the 3D Winograd where its budget allows a
     wave of GEMM rows, depth taps (each a 2D Winograd) otherwise."""
-    check3d(s, "f32", sample=1024)
+    check3d(s, "f32", sample=4096)

@@ -184,3 +184,44 @@ def test_bounded_wait_reports_timeout_instead_of_hanging():
     B.conv2d(x, w, S.stride, S.pad, S.dilation)
     assert B.conv_check(s) == 0
     assert B.conv_selftest_timeout(10, s) == 1     # limit out of range
+
+
+def test_bad_out_tensor_is_refused_before_any_launch():
+    """The torch conveniences check a caller's out= (shape, dtype, device,
+    contiguity) and workspace= (device, size) before a pointer reaches the
+    library: each raises ValueError and the poisoned buffers stay untouched
+    (no kernel ran)."""
+    x, w = synth.conv2d_inputs(S, "f32", "normal", 0, device="cuda")
+    good = (S.n, S.oh, S.ow, S.o)
+    bad_outs = [
+        torch.full((S.n, S.oh, S.ow - 1, S.o), float("nan"), device="cuda"),                # too small
+        torch.full((S.n, S.oh, S.ow, S.o + 1), float("nan"), device="cuda"),                # wrong shape
+        torch.full(good, float("nan"), dtype=torch.float16, device="cuda"),                 # wrong dtype
+        torch.full(good, float("nan")),                                                     # host memory
+        torch.full((S.n, S.oh, S.o, S.ow), float("nan"), device="cuda").transpose(2, 3),    # not contiguous
+    ]
+    for out in bad_outs:
+        with pytest.raises(ValueError):
+            B.conv2d(x, w, 1, 1, 1, out=out)
+    torch.cuda.synchronize()
+    for out in bad_outs:
+        assert torch.isnan(out.float()).all()
+    # conv3d and conv1d take the same checks
+    s3 = synth.Conv3dShape(1, 5, 6, 6, 16, 16, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    x3, w3 = synth.conv3d_inputs(s3, "bf16", "normal", 0, device="cuda")
+    o3 = torch.full((1, s3.od + 1, s3.oh, s3.ow, s3.o), float("nan"), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        B.conv3d(x3, w3, 1, (0, 1, 1), 1, out=o3)
+    x1, w1 = synth.make_inputs((2, 50, 16), (24, 3, 16), "f32", "normal", 0, device="cuda")
+    o1 = torch.full((2, 47, 24), float("nan"), device="cuda")
+    with pytest.raises(ValueError):
+        B.conv1d(x1, w1, 1, 0, 1, out=o1)
+    # a workspace smaller than the plan's, or on the host
+    opts = B.make_options("winograd")
+    need = B.conv2d_workspace_size(desc(S), 0, 0, opts)
+    out = torch.full(good, float("nan"), device="cuda")
+    for ws in (torch.empty(need - 1, dtype=torch.uint8, device="cuda"), torch.empty(need, dtype=torch.uint8)):
+        with pytest.raises(ValueError):
+            B.conv2d(x, w, 1, 1, 1, options=opts, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all() and torch.isnan(o3.float()).all() and torch.isnan(o1).all()

@@ -344,6 +344,27 @@ def test_sampled_pixels_match_full_tensor():
         assert np.array_equal(samp[i], full[n, y, xx])
 
 
+def test_sampled_pixels_match_full_tensor_3d():
+    """The 3D sampled mode reads (n, od, oh, ow) quadruples: each sampled row
+    equals the full tensor at that position, with N > 1, OD > 1 and stride,
+    padding and dilation that differ per axis (depth padding included), on
+    pixels that include the first and last output frame of both images."""
+    s = synth.Conv3dShape(2, 9, 8, 10, 3, 5, 3, 2, 3, (2, 1, 2), (2, 1, 1), (2, 1, 1))
+    x, w = synth.conv3d_inputs(s, "f16", "normal", 4)
+    full = oracle.conv3d(x, w, "f16", s.stride, s.pad, s.dilation)
+    assert full.shape == (2, s.od, s.oh, s.ow, 5) and s.od > 2
+    pix = synth.sample_pixels(2, s.oh, s.ow, count=40, seed=5, od=s.od)
+    quads = {tuple(p) for p in pix.tolist()}
+    for n in (0, 1):
+        for f in (0, s.od - 1):
+            assert (n, f, 0, 0) in quads and (n, f, s.oh - 1, s.ow - 1) in quads
+    assert {p[1] for p in quads} >= {0, s.od - 1} and len({p[1] for p in quads}) > 2
+    samp = oracle.conv3d(x, w, "f16", s.stride, s.pad, s.dilation, pixels=pix.numpy())
+    assert samp.shape == (pix.shape[0], 5)
+    for i, (n, f, y, xx) in enumerate(pix.tolist()):
+        assert np.array_equal(samp[i], full[n, f, y, xx]), (n, f, y, xx)
+
+
 def test_empty_batch_is_empty():
     x = np.zeros((0, 5, 5, 2), np.float32)
     w = np.ones((3, 3, 3, 2), np.float32)

@@ -36,7 +36,7 @@ def test_grid_auto(dtype):
     print(f"{dtype}: worst rel err over {len(GRID)} shapes = {worst:.3e}")
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("algo", ["implicit", "direct"])
 def test_grid_forced(dtype, algo):
     for shape in GRID[::5]:
@@ -103,23 +103,39 @@ def test_tf32_is_never_used():
 def test_resnet50_layers(batch, dtype):
     worst = 0.0
     for name, shape, _ in synth.resnet50_layers(batch):
-        worst = max(worst, check_conv2d(shape, dtype, dist="he", sample=1024))
+        worst = max(worst, check_conv2d(shape, dtype, dist="he", sample=4096))
     print(f"resnet50 b{batch} {dtype}: worst {worst:.3e}")
 
 
-SWEEP_SUBSET = [s for i, s in enumerate(synth.wide_sweep(True)) if i % 37 == 0]
+# Config-4 coverage: every (filter, C_in) x C_out x (stride, dilation)
+# combination of the wide-channel sweep once per dtype, at the sweep's largest
+# M (N = 16, 64x64 outputs), on >= 4096 seeded output pixels; and the whole
+# unaligned subset.  Grouped by (k, C_in) so a failure names its group.
+SWEEP_M_MAX = [s for s in synth.wide_sweep(True) if s.n == 16]
+SWEEP_GROUPS = sorted({(s.kh, s.c) for s in SWEEP_M_MAX})
+
+
+def test_sweep_coverage_is_complete():
+    combos = {(s.kh, s.c, s.o, s.stride, s.dilation) for s in SWEEP_M_MAX}
+    assert len(combos) == len(SWEEP_M_MAX) == 7 * 6 * 4
+    assert all(s.n * s.oh * s.ow == 65536 for s in SWEEP_M_MAX)
+    assert len(synth.wide_sweep(False)) == 48
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_wide_sweep_subset(dtype):
-    for shape in SWEEP_SUBSET:
-        check_conv2d(shape, dtype, sample=512)
+@pytest.mark.parametrize("group", SWEEP_GROUPS, ids=lambda g: f"k{g[0]}_c{g[1]}")
+def test_wide_sweep_every_combination(group, dtype):
+    worst = 0.0
+    for shape in SWEEP_M_MAX:
+        if (shape.kh, shape.c) == group:
+            worst = max(worst, check_conv2d(shape, dtype, sample=4096))
+    print(f"k{group[0]} C={group[1]} {dtype}: worst {worst:.3e}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 def test_wide_sweep_unaligned(dtype):
-    for shape in synth.wide_sweep(False)[::3]:
-        check_conv2d(shape, dtype, sample=512)
+    for shape in synth.wide_sweep(False):
+        check_conv2d(shape, dtype, sample=4096)
 
 
 CONV1D = [

@@ -5,8 +5,10 @@ It exists for callers that cannot allocate device memory or pass a workspace
 running, callers with only borrowed pointers): its scratch is a fixed 64 MiB
 device array inside the library.  These tests call it through the C ABI and
 compare it with the existing conv2d_forward entry point, on two calls in a
-row (the array keeps the previous call's contents, which must not matter),
-and check that a conv too large for the array is refused before any launch.
+row (the array keeps the previous call's contents, which must not matter):
+bit for bit against conv2d_forward forced to Winograd at the same batch tile,
+and within the parity tolerance against the CPU oracle and the auto path.  A
+conv too large for the array is refused before any launch.
 
 This file is named to be collected last, and it sets up nothing that depends
 on the other test files, so it passes alone in a fresh process too.
@@ -35,11 +37,36 @@ def _desc(s):
     return B.make_desc2d(s.n, s.h, s.w, s.c, s.o, s.kh, s.kw, s.stride, s.pad, s.dilation)
 
 
+STATIC_BYTES = 64 << 20
+
+
+def _static_tile(shape, dtype):
+    """The batch tile the static entry point settles on: the largest tile whose
+    transformed filter plus transform buffers fit the 64 MiB array (the same
+    search, done here through conv2d_plan)."""
+    desc = _desc(shape)
+    tile = shape.n
+    while True:
+        p = B.plan2d(desc, dtype, 0, B.make_options("winograd", STATIC_BYTES, tile))
+        if p["workspace_bytes"] <= STATIC_BYTES:
+            return p
+        assert p["batch_tile"] > 1, "not even one image fits"
+        tile = p["batch_tile"] - 1
+
+
 @pytest.mark.parametrize("shape,dtype", CASES, ids=lambda v: v.name() if hasattr(v, "name") else v)
 def test_static_scratch_matches_conv2d_forward(shape, dtype):
+    import oracle
     x, w = synth.conv2d_inputs(shape, dtype, "normal", 3, device="cuda")
-    ref = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation)      # existing entry point
-    ref_win = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation, options=B.make_options("winograd"))
+    plan = _static_tile(shape, dtype)
+    assert plan["algo"] == "winograd"
+    if shape == CASES[0][0]:
+        assert plan["num_batch_tiles"] > 1, plan      # the first case really runs batch-tiled
+    # the existing entry point, forced to Winograd at the static entry's tile size
+    ref_win = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation,
+                       options=B.make_options("winograd", winograd_tile_batch=plan["batch_tile"]))
+    ref_auto = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation)
+    want = oracle.conv2d(x.cpu(), w.cpu(), dtype, shape.stride, shape.pad, shape.dilation)
     stream = torch.cuda.current_stream().cuda_stream
     desc = _desc(shape)
     for call in range(2):
@@ -51,10 +78,13 @@ def test_static_scratch_matches_conv2d_forward(shape, dtype):
         assert B.conv_check(stream) == 0
         got = as_f64(out)
         assert np.isfinite(got).all(), f"call {call}: unwritten output"
-        e = rel_err(got, as_f64(ref))
-        assert e <= TOL[dtype], f"call {call}: {e:.3e}"
-        e2 = rel_err(got, as_f64(ref_win))
-        assert e2 <= TOL[dtype], f"call {call} vs forced Winograd: {e2:.3e}"
+        # bit for bit what conv2d_forward's Winograd path gives at the same tile size
+        assert torch.equal(out.view(torch.int32 if dtype == "f32" else torch.int16),
+                           ref_win.view(torch.int32 if dtype == "f32" else torch.int16)), f"call {call}"
+        e = rel_err(got, want)
+        assert e <= TOL[dtype], f"call {call} vs the oracle: {e:.3e}"
+        e2 = rel_err(got, as_f64(ref_auto))
+        assert e2 <= TOL[dtype], f"call {call} vs conv2d_forward (auto): {e2:.3e}"
 
 
 def test_static_scratch_refuses_what_does_not_fit():
