@@ -86,10 +86,11 @@ long long out_extent(long long in, int k, int s, int p, int d) {
 
 enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_SPLITK_REDUCE, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
             K_WINO_OUTPUT, K_WINO3D_FILTER, K_WINO3D_INPUT, K_WINO3D_GEMM_TC, K_WINO3D_GEMM_SIMT, K_WINO3D_OUTPUT,
-            K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_COUNT };
+            K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_WINO_PASS, K_COUNT };
 const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "splitk_reduce", "wino_filter", "wino_input", "wino_gemm_tc",
                                         "wino_gemm_simt", "wino_output", "wino3d_filter", "wino3d_input", "wino3d_gemm_tc",
-                                        "wino3d_gemm_simt", "wino3d_output", "accumulate", "channel_pad", "fill"};
+                                        "wino3d_gemm_simt", "wino3d_output", "accumulate", "channel_pad", "fill",
+                                        "wino_pass"};
 
 struct ProfRecord {
   int kind;
@@ -183,6 +184,7 @@ struct Sel {
   int ksplit = 1;          // implicit GEMM: K range split over ksplit CTAs, fp32 partials reduced after
   size_t split_off = 0;    // workspace offset of the partials
   conv_dtype_t wino_store = CONV_F32;
+  long long chunk = 0;     // Winograd: tiles per transform -> GEMM -> transform pass (0: the whole batch tile)
   size_t ws = 0;
 };
 
@@ -220,6 +222,17 @@ int tc_tile_n(const Geom& g, const conv_device_props_t& p) {
 
 long long round4(long long x) { return (x + 3) & ~3LL; }
 
+// CTA pairs (tile_m = 256, two SMs per tile sharing the weight tile) for
+// 256-wide column tiles when there are enough 256-row tiles to give every SM
+// pair one.  B200CONV_TC_PAIR=0 (a test hook, read on every call) keeps 128-row tiles.
+bool tc_pair_tiles(long long rows, long long batches, int o, int tile_n, const conv_device_props_t& p) {
+  if (tile_n != 256) return false;
+  if (const char* e = std::getenv("B200CONV_TC_PAIR"))
+    if (std::strcmp(e, "0") == 0) return false;
+  const long long tiles = batches * ((rows + 255) / 256) * ((o + 255) / 256);
+  return tiles >= p.sm_count / 2;
+}
+
 // V layout of the fp32 (FFMA) Winograd path: tile-major [a2][T][C] lets the
 // input transform write whole pixels' channels contiguously; the GEMM stages
 // it through swizzled shared rows.
@@ -240,22 +253,34 @@ struct WinoLayout {
   size_t per_img = 0;   // V + M bytes per image (the budget unit)
 };
 
-WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb) {
+// chunk > 0: the batch tile's tiles pass through V and M in chunks of at most
+// `chunk` tiles, so V and M hold one chunk.
+WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb, long long chunk = 0) {
   WinoLayout L;
   const long long a2 = (long long)(m + 2) * (m + 2);
   L.tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
   const int esz = dtype_size(store);
   L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * esz + (size_t)g.o * (cmajor ? 4 : esz));
-  const long long t = nb * L.tiles_per_img;
+  const long long t = chunk > 0 ? std::min(nb * L.tiles_per_img, chunk) : nb * L.tiles_per_img;
   if (cmajor) {
     L.u_bytes = align256((size_t)(a2 * g.c * round4(g.o)) * esz);
     L.v_bytes = align256((size_t)(a2 * g.c * ((kF32VTileMajor && g.c % 4 == 0) ? t : round4(t))) * esz);
+    if (chunk > 0) L.v_bytes *= 2;   // two V buffers: chunk i+1 is transformed while chunk i's GEMM drains
   } else {
     L.u_bytes = align256((size_t)(a2 * g.o * g.c) * esz);
     L.v_bytes = align256((size_t)(a2 * t * g.c) * esz);
   }
   L.m_bytes = align256((size_t)(a2 * t * g.o) * (cmajor ? 4 : esz));
   return L;
+}
+
+// Tiles per chunk of the fp32 Winograd pass (FFMA GEMM, tile-major V).  0
+// keeps the whole batch tile in one pass.  B200CONV_WINOGRAD_CHUNK_TILES
+// overrides it (a test hook, read on every call).
+long long winograd_chunk_tiles(const Geom& g, int m, const conv_device_props_t& p) {
+  (void)g; (void)m; (void)p;
+  if (const char* e = std::getenv("B200CONV_WINOGRAD_CHUNK_TILES")) return std::max(0LL, std::atoll(e));
+  return 0;
 }
 
 conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t& p,
@@ -303,9 +328,10 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->wino_store = store;
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
-      s->tile_m = 128;
       s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
-      const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb);
+      s->tile_m = tc_gemm && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o, s->tile_n, p) ? 256 : 128;
+      s->chunk = (!tc_gemm && kF32VTileMajor && g.c % 4 == 0) ? winograd_chunk_tiles(g, m, p) : 0;
+      const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb, s->chunk);
       s->ws = L.u_bytes + L.v_bytes + L.m_bytes;
       s->cpad = 0;
       return CONV_OK;
@@ -369,6 +395,8 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->split_off = s->ws;
       s->ws += align256((size_t)ks * M * g.o * 4);
     }
+    if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack && tc_pair_tiles(M, 1, g.o, s->tile_n, p))
+      s->tile_m = 256;
   }
   return CONV_OK;
 }
@@ -431,7 +459,7 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
   if (s.algo == CONV_ALGO_WINOGRAD) {
     const int m = s.wino_m, a2 = (m + 2) * (m + 2);
     const bool cmajor = s.engine == CONV_ENGINE_SIMT;
-    const WinoLayout L = winograd_layout(g, s.wino_store, cmajor, m, s.nb);
+    const WinoLayout L = winograd_layout(g, s.wino_store, cmajor, m, s.nb, s.chunk);
     uint8_t* base = static_cast<uint8_t*>(ws);
     void* u = base;
     void* v = base + L.u_bytes;
@@ -444,33 +472,69 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
                  : launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
     }
     if (e != cudaSuccess) return CONV_ERR_CUDA;
+    const bool tmajor = kF32VTileMajor && g.c % 4 == 0;
+    if (s.chunk > 0) {
+      // Chunked pipeline: per batch tile, chunks of at most s.chunk tiles, so V
+      // and M stay in L2 between the kernels.  Pass k transforms the output of
+      // chunk k-1 and the input of chunk k in one launch; the GEMM of chunk k
+      // sits between passes k and k+1.  V alternates between two buffers.
+      struct Chunk { long long t0, t; };
+      std::vector<Chunk> chunks;
+      for (int n0 = 0; n0 < g.n; n0 += s.nb) {
+        const long long t_all = (long long)std::min(s.nb, g.n - n0) * L.tiles_per_img;
+        for (long long tb = 0; tb < t_all; tb += s.chunk)
+          chunks.push_back({(long long)n0 * L.tiles_per_img + tb, std::min(s.chunk, t_all - tb)});
+      }
+      float* vbuf[2] = {static_cast<float*>(v), static_cast<float*>(v) + L.v_bytes / 2 / sizeof(float)};
+      const size_t nc = chunks.size();
+      for (size_t k = 0; k <= nc; ++k) {
+        const Chunk in_c = k < nc ? chunks[k] : Chunk{0, 0};
+        const Chunk out_c = k > 0 ? chunks[k - 1] : Chunk{0, 0};
+        {
+          ProfScope ps(K_WINO_PASS, st);
+          // the first pass waits for everything before it in the stream
+          e = launch_wino_pass(in, g, m, dt, 0, in_c.t0, in_c.t, vbuf[k & 1], out_c.t0, out_c.t,
+                               static_cast<const float*>(mb), out, accumulate, k > 0, st);
+        }
+        if (e != cudaSuccess) return CONV_ERR_CUDA;
+        if (k < nc) {
+          ProfScope ps(K_WINO_GEMM_SIMT, st);
+          e = launch_wino_gemm_f32(vbuf[k & 1], static_cast<const float*>(u), static_cast<float*>(mb), a2,
+                                   (int)in_c.t, g.c, g.o, g.c, round4(g.o), true, st);
+          if (e != cudaSuccess) return CONV_ERR_CUDA;
+        }
+      }
+      return CONV_OK;
+    }
     for (int n0 = 0; n0 < g.n; n0 += s.nb) {
       const int nbi = std::min(s.nb, g.n - n0);
-      const long long t = (long long)nbi * L.tiles_per_img;
+      const long long t_all = (long long)nbi * L.tiles_per_img;
       {
-        ProfScope ps(K_WINO_INPUT, st);
-        if (cmajor && !(kF32VTileMajor && g.c % 4 == 0))
-          e = launch_wino_input_cmajor(in, g, n0, nbi, m, dt, static_cast<float*>(v), round4(t), st);
-        else
-          e = launch_wino_input(in, g, n0, nbi, m, dt, s.wino_store, v, t, st);
+        const long long tb = 0, t = t_all;
+        {
+          ProfScope ps(K_WINO_INPUT, st);
+          if (cmajor && !tmajor)
+            e = launch_wino_input_cmajor(in, g, n0, nbi, m, dt, static_cast<float*>(v), round4(t), st);
+          else
+            e = launch_wino_input(in, g, n0, tb, t, m, dt, s.wino_store, v, t, st);
+        }
+        if (e != cudaSuccess) return CONV_ERR_CUDA;
+        if (cmajor) {
+          ProfScope ps(K_WINO_GEMM_SIMT, st);
+          e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), static_cast<float*>(mb),
+                                   a2, (int)t, g.c, g.o, tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
+        } else {
+          BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb, m_dt};
+          ProfScope ps(K_WINO_GEMM_TC, st);
+          e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st, s.tile_m);
+        }
+        if (e != cudaSuccess) return CONV_ERR_CUDA;
+        {
+          ProfScope ps(K_WINO_OUTPUT, st);
+          e = launch_wino_output(mb, m_dt, g, n0, tb, t, m, t, dt, out, accumulate, st);
+        }
+        if (e != cudaSuccess) return CONV_ERR_CUDA;
       }
-      if (e != cudaSuccess) return CONV_ERR_CUDA;
-      if (cmajor) {
-        ProfScope ps(K_WINO_GEMM_SIMT, st);
-        const bool tmajor = kF32VTileMajor && g.c % 4 == 0;
-        e = launch_wino_gemm_f32(static_cast<const float*>(v), static_cast<const float*>(u), static_cast<float*>(mb),
-                                 a2, (int)t, g.c, g.o, tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
-      } else {
-        BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb, m_dt};
-        ProfScope ps(K_WINO_GEMM_TC, st);
-        e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st);
-      }
-      if (e != cudaSuccess) return CONV_ERR_CUDA;
-      {
-        ProfScope ps(K_WINO_OUTPUT, st);
-        e = launch_wino_output(mb, m_dt, g, n0, nbi, m, t, dt, out, accumulate, st);
-      }
-      if (e != cudaSuccess) return CONV_ERR_CUDA;
     }
     return CONV_OK;
   }
@@ -525,11 +589,15 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     gg.w_row_stride = (long long)g.kh * g.kw * s.cpad;
   }
   float* partial = s.ksplit > 1 ? reinterpret_cast<float*>(base + s.split_off) : nullptr;
-  bool done = false;
+  bool done = false, reduced = false;
   if (s.engine == CONV_ENGINE_TCGEN05 && tc_conv_supported(gg, dt, cin, cw)) {
+    // split-K sums inside the kernel (a cluster per tile) unless the test hook
+    // B200CONV_SPLITK_CLUSTER=0 asks for the partials-and-reduce route
+    const char* sc = std::getenv("B200CONV_SPLITK_CLUSTER");
+    const bool cluster_ok = !(sc && std::strcmp(sc, "0") == 0);
     ProfScope ps(K_TC_CONV, st);
     if (launch_tc_conv(cin, cw, out, gg, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st, s.ksplit,
-                       partial) != cudaSuccess)
+                       partial, cluster_ok ? &reduced : nullptr, s.tile_m) != cudaSuccess)
       return CONV_ERR_CUDA;
     done = true;
   }
@@ -541,7 +609,7 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     if (launch_simt_conv(cin, cw, out, gg, dt, vec, accumulate, st, s.ksplit, partial) != cudaSuccess)
       return CONV_ERR_CUDA;
   }
-  if (s.ksplit > 1) {
+  if (s.ksplit > 1 && !reduced) {
     ProfScope ps(K_SPLITK_REDUCE, st);
     if (launch_splitk_reduce(partial, s.ksplit, (size_t)g.n * g.oh * g.ow * g.o, out, dt, accumulate, st) !=
         cudaSuccess)
@@ -735,6 +803,7 @@ conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_de
     s->tile_m = 128;
     const long long m_tiles = ((long long)d->n * *od * g2->oh * g2->ow + 127) / 128;
     s->tile_n = d->o <= 128 || m_tiles * ((d->o + 255) / 256) < p.sm_count ? 128 : 256;
+    s->tile_m = tc_pair_tiles((long long)d->n * *od * g2->oh * g2->ow, 1, d->o, s->tile_n, p) ? 256 : 128;
     s->wino_m = 0;
     s->nb = d->n;
     s->ntiles = 1;
@@ -994,7 +1063,7 @@ conv_status_t conv3d_forward(const void* in, const void* w, void* out, const con
   if (path == P3_WINO3D) return run3d_winograd(in, w, out, g3, dtype, s, workspace, *d, st_);
   if (path == P3_NATIVE) {
     ProfScope ps(K_TC_CONV3D, st_);
-    return cuda_status(launch_tc_conv3d(in, w, out, g3, dtype, s.tile_n, d->props.sm_count, d->err_word, st_));
+    return cuda_status(launch_tc_conv3d(in, w, out, g3, dtype, s.tile_n, d->props.sm_count, d->err_word, st_, s.tile_m));
   }
   Tap taps[1024];
   if (desc->kd > 1024) return CONV_ERR_UNSUPPORTED;

@@ -71,18 +71,24 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count,
 // Returns cudaErrorNotSupported if the shape cannot be encoded as TMA maps.
 bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w);
 // accumulate: out = round(out + round(result)), the unfused depth-tap add's arithmetic.
-// ksplit > 1: fp32 partials [ksplit][M][O] to `partial` (then launch_splitk_reduce).
+// ksplit > 1: the K range is split over ksplit CTAs per tile.  With `reduced`
+// given, the splits of a tile run as one thread-block cluster that sums the
+// partials in split order inside the kernel and sets *reduced; otherwise (or
+// when the device cannot hold the cluster) fp32 partials [ksplit][M][O] go to
+// `partial` and the caller runs launch_splitk_reduce (same sums, same order).
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
                            conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
-                           bool accumulate, cudaStream_t s, int ksplit = 1, float* partial = nullptr);
+                           bool accumulate, cudaStream_t s, int ksplit = 1, float* partial = nullptr,
+                           bool* reduced = nullptr, int tile_m = 128);
 // Native 3D implicit GEMM on tcgen05: K = KD*KH*KW*C in one main loop, the A
 // tiles gathered by a 5D TMA im2col map (corners limited to [-16, 15]).
 bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w);
+// tile_m == 256 (with tile_n == 256): CTA pairs on 256-row tiles where the device can hold them.
 cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geom3& g, conv_dtype_t dt, int tile_n,
-                             int sm_count, int* err_word, cudaStream_t s);
+                             int sm_count, int* err_word, cudaStream_t s, int tile_m = 128);
 // tcgen05 batched GEMM for 16-bit operands with fp32 D (Winograd 16-bit path).
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n,
-                                   int sm_count, int* err_word, cudaStream_t s);
+                                   int sm_count, int* err_word, cudaStream_t s, int tile_m = 128);
 
 // Watchdog self-test: one bounded wait on a barrier nothing arrives on.
 cudaError_t launch_wait_selftest(int* err_word, long long limit_ns, cudaStream_t s);
@@ -90,9 +96,23 @@ cudaError_t launch_wait_selftest(int* err_word, long long limit_ns, cudaStream_t
 // Winograd transforms (fp32 arithmetic; V/U stored in `store_dt`).
 cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int c, int m,
                                conv_dtype_t in_dt, conv_dtype_t store_dt, void* u, cudaStream_t s);
-cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int m,
+// A call covers tiles [t_base, t_base + t_count) counted from image n0's first
+// tile (tile t of an image at t / (tiles_h*tiles_w) images past n0); V and M
+// rows are numbered from 0 within the call, t_tile rows per plane.
+cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, long long t_base, long long t_count, int m,
                               conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_tile,
                               cudaStream_t s);
+// One pass of the chunked fp32-store Winograd pipeline: the input transform of
+// tiles [in_t_base, +in_t_count) into V (fp32, rows packed: in_t_count per
+// plane) and the output transform of tiles [out_t_base, +out_t_count) from M
+// (fp32, out_t_count rows per plane), tiles counted from image n0's first
+// tile, in one launch.  Either count may be 0.  pdl: launched with
+// programmatic stream serialization, the output part waiting for the previous
+// kernel (the GEMM that wrote M) and the input part not waiting, which is
+// correct only when V was last read by the kernel before that one.
+cudaError_t launch_wino_pass(const void* in, const Geom& g, int m, conv_dtype_t dt, int n0, long long in_t_base,
+                             long long in_t_count, float* v, long long out_t_base, long long out_t_count,
+                             const float* mb, void* out, bool accumulate, bool pdl, cudaStream_t s);
 // Channel-major fp32 variants for the FFMA GEMM: U[xi][c][o_pad], V[xi][c][t_stride].
 cudaError_t launch_wino_filter_cmajor(const void* w, long long w_row_stride, int o, int c, int m,
                                       conv_dtype_t in_dt, long long o_pad, float* u, cudaStream_t s);
@@ -104,9 +124,9 @@ cudaError_t launch_wino_gemm_f32(const float* a, const float* b, float* d, int b
                                  long long lda, long long ldb, bool a_tmajor, cudaStream_t s);
 int wino_gemm_f32_tile_n(int o);
 // M [a2][t_tile][O] in m_dt (fp32, or the 16-bit operand type of the tensor-core path).
-cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, int nb, int m,
-                               long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
-                               cudaStream_t s);
+cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, long long t_base,
+                               long long t_count, int m, long long t_tile, conv_dtype_t out_dt, void* out,
+                               bool accumulate, cudaStream_t s);
 
 // Native 3D Winograd F(m^3, 3^3) transforms, m in {2, 4}, for 3x3x3 stride-1
 // dilation-1 convs.  Tiles are numbered unit-major, a unit being one (image,

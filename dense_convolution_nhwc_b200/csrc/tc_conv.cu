@@ -49,10 +49,12 @@ constexpr int THREADS = 192;
 #define TC_EPI_COLS 128        // accumulator columns an epilogue thread reads per TMEM wait
 #endif
 
-template <int BN> struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+// CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a CTA pair computes a
+// 256 x BN tile, each CTA holding 128 rows of A and BN/2 rows of B per stage.
+template <int BN, int CG = 1> struct Cfg {
+  static constexpr int STAGES = CG == 2 ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = (BN / CG) * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators
   static constexpr int BAR_BYTES = 256;
@@ -79,19 +81,23 @@ struct TcArgs {
   int accumulate;              // out = round(out + round(acc)) instead of out = round(acc)
   int ksplit;                  // conv modes: > 1 splits the K range, the split index in the batch slot
   int tma_store;               // write 32-row x 128-byte chunks with TMA stores through tmD
+  int cluster_reduce;          // split-K whose ksplit CTAs of a tile form a cluster: rank 0 sums the
+                               // others' fp32 partials from their shared memory and writes out
   int* err;
 };
 
 // --------------------------------- kernel -----------------------------------
 
 // MODE 0: batched GEMM (tiled A); 1: conv2d (4D im2col A); 2: conv3d (5D im2col A).
-template <int BN, int MODE, typename TIn, typename TOut>
+// CG = 2: CTA pairs (clusters of 2) on 256-row tiles, a.m_tiles counting 256-row tiles.
+template <int BN, int MODE, typename TIn, typename TOut, int CG = 1>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const TcArgs a) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, CG>;
   constexpr int STORE_BYTES = C::STORE_BYTES;
-  constexpr uint32_t IDESC = make_idesc<BN>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
+  constexpr uint32_t IDESC = make_idesc<BN, BM * CG>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
+  static_assert(CG == 1 || CG == 2, "CTA group");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,6 +117,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   auto tfull_bar = [&](int i) { return bar0 + 8u * (2 * C::STAGES + i); };
   auto tempty_bar = [&](int i) { return bar0 + 8u * (2 * C::STAGES + 2 + i); };
   const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+  static_assert(BM * BN * 4 <= C::STAGES * C::STAGE_BYTES, "split partial fits the stage ring");
+  const bool cl = CG == 1 && MODE == 1 && a.cluster_reduce;
+  const uint32_t crank = cl ? cluster_rank() : 0u;
+  // CTA pair: rank 0 issues the MMAs; both load and drain their own halves.
+  const uint32_t prank = CG == 2 ? cluster_rank() : 0u;
+  const long long tile0 = CG == 2 ? (long long)(blockIdx.x >> 1) : (long long)blockIdx.x;
+  const long long tile_step = CG == 2 ? (long long)(gridDim.x >> 1) : (long long)gridDim.x;
+  // In cluster mode the grid holds one CTA per (tile, split), the splits of a
+  // tile adjacent (the cluster); map to the tile order of the other modes.
+  auto tile_of = [&](long long lt) {
+    if (!cl) return lt;
+    return (lt % a.ksplit) * ((long long)a.m_tiles * a.n_tiles) + lt / a.ksplit;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -119,17 +138,25 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull_bar(i), 1);
-      mbar_init(tempty_bar(i), 128);
+      mbar_init(tempty_bar(i), 128 * CG);     // CTA pair: both CTAs' epilogue threads, on rank 0's barrier
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)C::TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (CG == 2) {
+      // the same warp of both CTAs allocates, with the same destination offset
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"((uint32_t)C::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"((uint32_t)C::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   if (threadIdx.x == 32) {
     prefetch_tensormap(&tmA);
@@ -137,7 +164,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (a.tma_store) prefetch_tensormap(&tmD);
   }
   tc_fence_before();
-  __syncthreads();
+  if (cl || CG == 2)
+    cluster_sync_all();     // every CTA's barriers are initialised before any remote arrive
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait_then_release();
@@ -152,15 +182,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (long long tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      for (long long lt = tile0; lt < total_tiles && ok; lt += tile_step) {
+        const long long tile = tile_of(lt);
         const int nt = (int)(tile % a.n_tiles);
         const long long rest = tile / a.n_tiles;
         const int mt = (int)(rest % a.m_tiles);
         const int b = (int)(rest / a.m_tiles);
+        // this CTA's 128 rows of the tile (the second half of a pair's 256)
+        const long long row0 = (long long)mt * (BM * CG) + (long long)prank * BM;
         int img = 0, wx = 0, hy = 0, dz = 0;
         if (MODE != 0) {
           // first output pixel of the tile -> its window's corner in the input
-          const long long m0 = (long long)mt * BM;
+          const long long m0 = row0;
           const long long ohw = (long long)a.oh * a.ow;
           long long fr = m0 / ohw;                   // image (2D) or image*OD + od (3D)
           const int rem = (int)(m0 - fr * ohw);
@@ -186,10 +219,38 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           const int tap = ks / a.kb_per_tap;
           const int kb = ks - tap * a.kb_per_tap;
-          const uint32_t fb = full_bar(stage);
-          mbar_expect_tx(fb, C::STAGE_BYTES);
           const uint32_t dA = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t dB = smem_u32(sB + stage * C::B_BYTES);
+          if constexpr (CG == 2) {
+            // both CTAs' loads complete on rank 0's full barrier, which expects both halves
+            if (prank == 0) mbar_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+            const uint32_t fb0 = mapa_shared(full_bar(stage), 0);
+            const int ncol = nt * BN + (int)prank * (BN / 2);
+            if (MODE == 1) {
+              const int ky = tap / a.kw, kx = tap - (tap / a.kw) * a.kw;
+              tma_load_im2col_4d_pair(dA, &tmA, fb0, kb * BK, wx, hy, img, (uint16_t)(kx * a.dw),
+                                      (uint16_t)(ky * a.dh));
+              tma_load_3d_pair(dB, &tmB, fb0, kb * BK, tap, ncol);
+            } else if (MODE == 2) {
+              const int khw = a.kh * a.kw;
+              const int kz = tap / khw, r2 = tap - kz * khw;
+              const int ky = r2 / a.kw, kx = r2 - (r2 / a.kw) * a.kw;
+              tma_load_im2col_5d_pair(dA, &tmA, fb0, kb * BK, wx, hy, dz, img, (uint16_t)(kx * a.dw),
+                                      (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
+              tma_load_3d_pair(dB, &tmB, fb0, kb * BK, tap, ncol);
+            } else {
+              tma_load_3d_pair(dA, &tmA, fb0, kb * BK, (int)row0, b);
+              tma_load_3d_pair(dB, &tmB, fb0, kb * BK, ncol, b);
+            }
+            ++issued;
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
+          const uint32_t fb = full_bar(stage);
+          mbar_expect_tx(fb, C::STAGE_BYTES);
           if (MODE == 1) {
             const int ky = tap / a.kw, kx = tap - (tap / a.kw) * a.kw;
             tma_load_im2col_4d(dA, &tmA, fb, kb * BK, wx, hy, img, (uint16_t)(kx * a.dw),
@@ -203,7 +264,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
             tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
           } else {
-            tma_load_3d(dA, &tmA, fb, kb * BK, mt * BM, b);
+            tma_load_3d(dA, &tmA, fb, kb * BK, (int)row0, b);
             tma_load_3d(dB, &tmB, fb, kb * BK, nt * BN, b);
           }
           ++issued;
@@ -213,8 +274,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
       }
-      // Drain: wait (bounded) until the last loads in flight have landed.
-      const int pending = issued < C::STAGES ? (int)issued : C::STAGES;
+      // Drain: wait (bounded) until the last loads in flight have landed.  A pair's
+      // loads land on rank 0's barriers, so rank 0 drains for both.
+      const int pending = (CG == 2 && prank != 0) ? 0 : (issued < C::STAGES ? (int)issued : C::STAGES);
       int s = stage;
       uint32_t ph = phase;
       for (int i = 0; i < pending; ++i) {
@@ -228,12 +290,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0) {
+    // (a CTA pair's MMAs are issued by rank 0 alone, for both CTAs)
+    if (lane == 0 && (CG == 1 || prank == 0)) {
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (long long tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
+      for (long long lt = tile0; lt < total_tiles && ok; lt += tile_step, ++it) {
+        const long long tile = tile_of(lt);
         const int acc = it & 1;
         const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, a.err, DEVERR_TIMEOUT_MMA_TMEM)) {
@@ -255,19 +319,34 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tc_fence_after();
           const uint32_t aa = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t bb = smem_u32(sB + stage * C::B_BYTES);
+          if constexpr (CG == 2) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            tc_mma(d_tmem, sdesc(aa + 32u * k), sdesc(bb + 32u * k), IDESC, (ks | k) != 0 ? 1u : 0u);
-          tc_commit(empty_bar(stage));
+            for (int k = 0; k < BK / 16; ++k)
+              tc_mma_pair(d_tmem, sdesc(aa + 32u * k), sdesc(bb + 32u * k), IDESC, (ks | k) != 0 ? 1u : 0u);
+            tc_commit_pair_both(empty_bar(stage));      // frees the stage in both CTAs
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              tc_mma(d_tmem, sdesc(aa + 32u * k), sdesc(bb + 32u * k), IDESC, (ks | k) != 0 ? 1u : 0u);
+            tc_commit(empty_bar(stage));
+          }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) tc_commit(tfull_bar(acc));
+        if (ok) {
+          if constexpr (CG == 2)
+            tc_commit_pair_both(tfull_bar(acc));       // both CTAs' accumulator halves are ready
+          else
+            tc_commit(tfull_bar(acc));
+        }
       }
       // Drain: all MMAs this thread issued have completed once this arrives.
-      tc_commit(drain_bar);
+      if constexpr (CG == 2)
+        tc_commit_pair_self(drain_bar);
+      else
+        tc_commit(drain_bar);
       volatile int never = 0;
       mbar_wait(drain_bar, 0, &never, a.err, 0);
     }
@@ -278,16 +357,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int row = q * 32 + lane;
     int it = 0;
     int store_count = 0;                    // TMA-stored chunks of this warp (staging double buffer)
-    for (long long tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+    for (long long lt = tile0; lt < total_tiles; lt += tile_step, ++it) {
+      const long long tile = tile_of(lt);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, a.err, DEVERR_TIMEOUT_EPILOGUE)) break;
       tc_fence_after();
+      if (cl) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the ring is reused for the partial
       const int nt = (int)(tile % a.n_tiles);
       const long long rest = tile / a.n_tiles;
       const int mt = (int)(rest % a.m_tiles);
       const int b = (int)(rest / a.m_tiles);
-      const long long m = (long long)mt * BM + row;
+      const long long trow0 = (long long)mt * (BM * CG) + (long long)prank * BM;   // this CTA's first row
+      const long long m = trow0 + row;
       const bool row_ok = m < a.m_rows;
       TOut* orow = static_cast<TOut*>(a.out) + (long long)b * a.out_batch + (row_ok ? m : 0) * a.ldo;
       const int n0 = nt * BN;
@@ -302,6 +384,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           TMEM_LD32(taddr, rr[h]);
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (cl) {
+          // split-K in a cluster: this split's fp32 partial goes to the (drained) stage
+          // ring as [128 rows][BN/4 float4], the float4 column XOR-swizzled by the row so
+          // that both this row-per-lane write and the column-per-lane reads of the
+          // reduction below are free of bank conflicts
+#pragma unroll
+          for (int h = 0; h < EPI / 32; ++h)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int col4 = (cg + 32 * h) / 4 + k;
+              *reinterpret_cast<float4*>(sA + ((size_t)row * (BN / 4) + (col4 ^ (row & (BN / 4 - 1)))) * 16) =
+                  make_float4(__uint_as_float(rr[h][4 * k]), __uint_as_float(rr[h][4 * k + 1]),
+                              __uint_as_float(rr[h][4 * k + 2]), __uint_as_float(rr[h][4 * k + 3]));
+            }
+          continue;
+        }
         if constexpr (sizeof(TOut) == 4) {
           if (a.tma_store) {
             // stage row `lane` of this warp's 32 x 32 chunk (16-byte chunks XOR-swizzled by
@@ -324,7 +422,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
               __syncwarp();
               if (lane == 0) {
-                tma_store_3d(&tmD, smem_u32(sb), c0, mt * BM + q * 32, b);
+                tma_store_3d(&tmD, smem_u32(sb), c0, (int)trow0 + q * 32, b);
                 bulk_commit();
               }
               ++store_count;
@@ -358,7 +456,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
               __syncwarp();
               if (lane == 0) {
-                tma_store_3d(&tmD, smem_u32(sb), c0, mt * BM + q * 32, b);
+                tma_store_3d(&tmD, smem_u32(sb), c0, (int)trow0 + q * 32, b);
                 bulk_commit();
               }
               ++store_count;
@@ -434,19 +532,85 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       }
       tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
+      if (CG == 2 && prank != 0)
+        mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));   // the pair's accumulator lives on in rank 0's count
+      else
+        mbar_arrive(tempty_bar(acc));
     }
     if (a.tma_store && lane == 0) bulk_wait_all();   // the last stores have landed
     __syncwarp();
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (cl) {
+    // Split-K reduction, shared by the cluster: once every split's partial is in
+    // (the barrier), CTA r sums rows [128 r / ks, 128 (r + 1) / ks) of the tile
+    // over the splits in split order (the order of the separate reduce kernel)
+    // from the CTAs' shared memory, and writes those output rows.
+    cluster_sync_all();
+    if (warp >= 2 && !*abort_flag) {
+      const int ks = a.ksplit;
+      const long long tile = tile_of(blockIdx.x);
+      const int nt = (int)(tile % a.n_tiles);
+      const int mt = (int)((tile / a.n_tiles) % a.m_tiles);
+      const int ew = warp - 2;
+      const int r_lo = (int)((long long)BM * crank / ks), r_hi = (int)((long long)BM * (crank + 1) / ks);
+      const uint32_t pbase = smem_u32(sA);
+      TOut* obase = static_cast<TOut*>(a.out);
+      for (int rr = r_lo + ew; rr < r_hi; rr += 4) {
+        const long long m = (long long)mt * BM + rr;
+        if (m >= a.m_rows) break;
+        for (int c4 = lane; c4 < BN / 4; c4 += 32) {
+          const int col = nt * BN + 4 * c4;
+          if (col >= a.ocols) continue;
+          const uint32_t off = (uint32_t)(((size_t)rr * (BN / 4) + (c4 ^ (rr & (BN / 4 - 1)))) * 16);
+          float4 sum = ld_cluster_f4(mapa_shared(pbase, 0) + off);
+          for (int sp = 1; sp < ks; ++sp) {
+            const float4 pv = ld_cluster_f4(mapa_shared(pbase, (uint32_t)sp) + off);
+            sum.x += pv.x; sum.y += pv.y; sum.z += pv.z; sum.w += pv.w;
+          }
+          TOut* p = obase + m * a.ldo + col;
+          float v[4] = {sum.x, sum.y, sum.z, sum.w};
+          const int nv = a.ocols - col < 4 ? a.ocols - col : 4;
+          if (a.accumulate) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (e < nv)
+                v[e] = Store<TOut>::to_f32(p[e]) + Store<TOut>::to_f32(Store<TOut>::from_f32(v[e]));
+          }
+          if (nv == 4 && (reinterpret_cast<uintptr_t>(p) & (4 * sizeof(TOut) - 1)) == 0) {
+            if constexpr (sizeof(TOut) == 4) {
+              *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+              uint2 u;
+              u.x = pack2<TOut>(v[0], v[1]);
+              u.y = pack2<TOut>(v[2], v[3]);
+              *reinterpret_cast<uint2*>(p) = u;
+            }
+          } else {
+            for (int e = 0; e < nv; ++e) p[e] = Store<TOut>::from_f32(v[e]);
+          }
+        }
+      }
+    }
+  }
+  // In cluster mode no CTA leaves while another may still read its shared
+  // memory: every wait above is bounded, so every thread of the cluster
+  // reaches this barrier.
+  if (cl || CG == 2)
+    cluster_sync_all();
+  else
+    __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"((uint32_t)C::TMEM_COLS)
-                 : "memory");
+    if constexpr (CG == 2)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"((uint32_t)C::TMEM_COLS)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"((uint32_t)C::TMEM_COLS)
+                   : "memory");
   }
 }
 
@@ -483,6 +647,139 @@ cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcAr
   CUtensorMap none;
   memset(&none, 0, sizeof(none));
   return launch_pdl(k, dim3(grid), dim3(THREADS), smem, s, A, B, D ? *D : none, a);
+}
+
+// CTA pairs: clusters of 2 on 256-row tiles, persistent over the tiles (one
+// pair per two SMs).  Sets *launched = false and launches nothing when the
+// device cannot hold such a pair (the caller then runs the 1-CTA kernel).
+template <int BN, int MODE, typename TIn, typename TOut>
+cudaError_t launch_kernel_pair(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int sm_count,
+                               cudaStream_t s, const CUtensorMap* D, bool* launched) {
+  *launched = false;
+  auto k = tc_gemm_kernel<BN, MODE, TIn, TOut, 2>;
+  constexpr int smem = Cfg<BN, 2>::template smem<TOut>();
+  static_assert(smem <= 232448, "shared memory budget");
+  cudaError_t e = set_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  const long long tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
+  if (tiles == 0) return cudaSuccess;
+  const long long pairs = tiles < sm_count / 2 ? tiles : sm_count / 2;
+  if (pairs < 1) return cudaSuccess;
+  static std::mutex mu;
+  static int ok_dev[64];          // 0 unknown, 1 yes, -1 no
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaSuccess;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (ok_dev[dev] == 0) {
+      cfg.numAttrs = 1;
+      int n = 0;
+      const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      if (qe != cudaSuccess) cudaGetLastError();
+      ok_dev[dev] = (qe == cudaSuccess && n >= 1) ? 1 : -1;
+    }
+    if (ok_dev[dev] < 0) return cudaSuccess;
+  }
+  cfg.numAttrs = 2;
+  CUtensorMap none;
+  memset(&none, 0, sizeof(none));
+  e = cudaLaunchKernelEx(&cfg, k, A, B, D ? *D : none, a);
+  if (e == cudaSuccess) *launched = true;
+  return e;
+}
+
+// Run the 1-CTA kernel, or (tile_m == 256) the CTA-pair kernel when the device
+// can hold a pair.  `a.m_tiles` counts rows in units of tile_m; the caller
+// encodes B with a box of BN / (tile_m / 128) rows.
+template <int BN, int MODE, typename TIn, typename TOut>
+cudaError_t launch_tiles(const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& Bpair, const TcArgs& a,
+                         int tile_m, int sm_count, cudaStream_t s, const CUtensorMap* D) {
+  if (tile_m == 256) {
+    bool launched = false;
+    cudaError_t e = launch_kernel_pair<BN, MODE, TIn, TOut>(A, Bpair, a, sm_count, s, D, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
+  TcArgs one = a;
+  one.m_tiles = (int)((a.m_rows + BM - 1) / BM);
+  return launch_kernel<BN, MODE, TIn, TOut>(A, B, one, sm_count, s, D);
+}
+
+// Split-K with the splits of each tile as one thread-block cluster of ks CTAs
+// (grid = tiles x ks, one (tile, split) per CTA).  Sets *launched = false and
+// launches nothing when the device cannot hold such a cluster (the caller then
+// takes the partials-and-reduce route).
+template <int BN, int MODE, typename TIn, typename TOut>
+cudaError_t launch_kernel_cluster(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int ks,
+                                  cudaStream_t s, const CUtensorMap* D, bool* launched) {
+  *launched = false;
+  auto k = tc_gemm_kernel<BN, MODE, TIn, TOut>;
+  constexpr int smem = Cfg<BN>::template smem<TOut>();
+  cudaError_t e = set_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  const long long tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
+  if (tiles == 0 || tiles % ks != 0 || tiles > 0x7fffffffLL) return cudaSuccess;
+  // How many clusters of ks such CTAs can be resident at once?  Asked once per
+  // (kernel, ks, device).  Clusters need ks SMs of one GPC each, so fewer fit
+  // than 148 / ks; unless all of this launch's clusters fit in one wave the
+  // partials-and-reduce route is faster, and the caller takes it.
+  static std::mutex mu;
+  static int cache[64][17];      // [device][ks]: 0 unknown, -1 none, else the resident cluster count
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64 || ks > 16) return cudaSuccess;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev][ks] == 0) {
+      if (ks > 8) cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3((unsigned)tiles);
+      q.blockDim = dim3(THREADS);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = ks;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int n = 0;
+      const cudaError_t qe = cudaOccupancyMaxActiveClusters(&n, k, &q);
+      if (qe != cudaSuccess) cudaGetLastError();      // clear it: the answer is "no"
+      cache[dev][ks] = (qe == cudaSuccess && n >= 1) ? n : -1;
+    }
+    if (cache[dev][ks] < 0 || tiles / ks > cache[dev][ks]) return cudaSuccess;
+  }
+  CUtensorMap none;
+  memset(&none, 0, sizeof(none));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, k, A, B, D ? *D : none, a);
+  if (e == cudaSuccess) *launched = true;
+  return e;
 }
 
 // 3D map over D [batches][rows][cols] (fp32 or 16-bit) for the epilogue's TMA stores: boxes of
@@ -527,7 +824,8 @@ bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const voi
 
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt,
                            int tile_n, int sm_count, int* err_word, bool accumulate, cudaStream_t s, int ksplit,
-                           float* partial) {
+                           float* partial, bool* reduced, int tile_m) {
+  if (reduced) *reduced = false;
   if (!tc_conv_supported(g, dt, in, w)) return cudaErrorNotSupported;
   const long long M = (long long)g.n * g.oh * g.ow;
   if (M == 0) return cudaSuccess;
@@ -566,6 +864,29 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   a.accumulate = accumulate ? 1 : 0;
   a.ksplit = 1;
   a.err = err_word;
+  if (ksplit > 1 && reduced && ksplit <= 16 && ksplit <= taps * a.kb_per_tap) {
+    // split-K inside the kernel: the ksplit CTAs of a tile form a cluster and
+    // rank 0 adds the others' partials (in split order) from their shared memory
+    TcArgs c = a;
+    c.ksplit = ksplit;
+    c.batches = ksplit;
+    c.cluster_reduce = 1;
+    CUtensorMap tD;
+    c.tma_store = !accumulate && encode_store_map(&tD, out, dt, g.o, M, 1) ? 1 : 0;
+    bool launched = false;
+    cudaError_t e;
+    if (dt == CONV_BF16)
+      e = tile_n == 256 ? launch_kernel_cluster<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, c, ksplit, s, &tD, &launched)
+                        : launch_kernel_cluster<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, c, ksplit, s, &tD, &launched);
+    else
+      e = tile_n == 256 ? launch_kernel_cluster<256, 1, __half, __half>(tA, tB, c, ksplit, s, &tD, &launched)
+                        : launch_kernel_cluster<128, 1, __half, __half>(tA, tB, c, ksplit, s, &tD, &launched);
+    if (e != cudaSuccess) return e;
+    if (launched) {
+      *reduced = true;
+      return cudaSuccess;
+    }
+  }
   if (ksplit > 1) {
     // split-K: ksplit partial fp32 results [ksplit][M][O], reduced by launch_splitk_reduce
     if (!partial || ksplit > taps * a.kb_per_tap) return cudaErrorInvalidValue;
@@ -584,6 +905,17 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   }
   CUtensorMap tD;
   a.tma_store = !accumulate && encode_store_map(&tD, out, dt, g.o, M, 1) ? 1 : 0;
+  if (tile_n == 256 && tile_m == 256) {
+    // CTA pairs: each CTA loads 128 weight rows of the 256-column tile
+    CUtensorMap tBp;
+    if (!encode_3d(&tBp, dt, w, g.c, taps, g.o, (uint64_t)g.c * 2, (uint64_t)g.w_row_stride * 2, BK, 1, 128))
+      return cudaErrorInvalidValue;
+    TcArgs p = a;
+    p.m_tiles = (int)((M + 255) / 256);
+    if (dt == CONV_BF16)
+      return launch_tiles<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, tBp, p, 256, sm_count, s, &tD);
+    return launch_tiles<256, 1, __half, __half>(tA, tB, tBp, p, 256, sm_count, s, &tD);
+  }
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD);
@@ -609,7 +941,7 @@ bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const 
 }
 
 cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geom3& g, conv_dtype_t dt, int tile_n,
-                             int sm_count, int* err_word, cudaStream_t s) {
+                             int sm_count, int* err_word, cudaStream_t s, int tile_m) {
   if (!tc_conv3d_supported(g, dt, in, w)) return cudaErrorNotSupported;
   const long long M = (long long)g.n * g.od * g.oh * g.ow;
   if (M == 0) return cudaSuccess;
@@ -649,6 +981,16 @@ cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geo
   a.err = err_word;
   CUtensorMap tD;
   a.tma_store = encode_store_map(&tD, out, dt, g.o, M, 1) ? 1 : 0;
+  if (tile_n == 256 && tile_m == 256) {
+    CUtensorMap tBp;
+    if (!encode_3d(&tBp, dt, w, g.c, taps, g.o, (uint64_t)g.c * 2, (uint64_t)taps * g.c * 2, BK, 1, 128))
+      return cudaErrorInvalidValue;
+    TcArgs p = a;
+    p.m_tiles = (int)((M + 255) / 256);
+    if (dt == CONV_BF16)
+      return launch_tiles<256, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, tBp, p, 256, sm_count, s, &tD);
+    return launch_tiles<256, 2, __half, __half>(tA, tB, tBp, p, 256, sm_count, s, &tD);
+  }
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 2, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD);
@@ -657,7 +999,7 @@ cudaError_t launch_tc_conv3d(const void* in, const void* w, void* out, const Geo
 }
 
 cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int tile_n, int sm_count,
-                                   int* err_word, cudaStream_t s) {
+                                   int* err_word, cudaStream_t s, int tile_m) {
   if (dt == CONV_F32 || !driver_fns()) return cudaErrorNotSupported;
   if (bg.c % 8 != 0 || (reinterpret_cast<uintptr_t>(bg.a) & 15) || (reinterpret_cast<uintptr_t>(bg.b) & 15))
     return cudaErrorNotSupported;
@@ -689,6 +1031,17 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
     if (bg.d_dt != dt) return cudaErrorInvalidValue;
     CUtensorMap tD16;
     a.tma_store = encode_store_map(&tD16, bg.d, dt, bg.o, bg.t, bg.batches) ? 1 : 0;
+    if (tile_n == 256 && tile_m == 256) {
+      CUtensorMap tBp;
+      if (!encode_3d(&tBp, dt, bg.b, bg.c, bg.o, bg.batches, (uint64_t)bg.c * 2, (uint64_t)bg.o * bg.c * 2, BK, 128,
+                     1))
+        return cudaErrorInvalidValue;
+      TcArgs p = a;
+      p.m_tiles = (bg.t + 255) / 256;
+      if (dt == CONV_BF16)
+        return launch_tiles<256, 0, __nv_bfloat16, __nv_bfloat16>(tA, tB, tBp, p, 256, sm_count, s, &tD16);
+      return launch_tiles<256, 0, __half, __half>(tA, tB, tBp, p, 256, sm_count, s, &tD16);
+    }
     if (dt == CONV_BF16)
       return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD16)
                            : launch_kernel<128, 0, __nv_bfloat16, __nv_bfloat16>(tA, tB, a, sm_count, s, &tD16);

@@ -19,6 +19,7 @@
 // on T (batch-tiled Winograd stays bit-identical to untiled).
 #include <cuda_runtime.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace b200conv {
@@ -69,6 +70,11 @@ wino_gemm_f32_kernel(const WgArgs p) {
   const float* __restrict__ B = p.b + bz * p.b_batch;
   float* __restrict__ D = p.d + bz * p.d_batch;
   const int ktiles = (p.c + BK - 1) / BK;
+
+  // Launched with programmatic stream serialization: everything above is
+  // address arithmetic; wait here for the kernel that wrote A (and for the one
+  // that last read D) before the first global access.
+  pdl_wait_then_release();
 
   // Per-thread copy descriptors, fixed across k-tiles (only the k offset moves).
   constexpr int A_PER = (A_CHUNKS + THREADS - 1) / THREADS;
@@ -254,8 +260,7 @@ cudaError_t launch_bn(const WgArgs& p, int batches, cudaStream_t s) {
   }
   const long long mblocks = (p.t + BM - 1) / BM;
   dim3 grid((unsigned)mblocks, (p.o + BN - 1) / BN, batches);
-  wino_gemm_f32_kernel<BN, A_TMAJOR><<<grid, THREADS, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(wino_gemm_f32_kernel<BN, A_TMAJOR>, grid, dim3(THREADS), smem, s, p);
 }
 
 }  // namespace

@@ -67,7 +67,8 @@ struct WinoInArgs {
   int h, w, c, ph, pw, tiles_h, tiles_w;
   long long in_img_stride;
   int n0;                 // first image of this batch tile
-  long long t_count;      // tiles in this batch tile (nb * tiles_h * tiles_w)
+  long long t_base;       // first tile of this call, counted from image n0's first tile
+  long long t_count;      // tiles in this call (V rows 0 .. t_count-1)
   long long t_stride;     // row count of V's planes (the workspace's tile capacity)
 };
 
@@ -75,21 +76,25 @@ struct WinoInArgs {
 // when the host has checked that they fit (fewer address instructions per
 // element), long long otherwise.  Tiles wholly inside the image skip the
 // bounds tests.
+// The body of one input-transform block: block `bid` of a 1D grid, thread
+// (tx, ty) of a bx x by block.
 template <int M, typename Tin, typename Tst, typename Idx>
-__global__ void __launch_bounds__(256)
-wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restrict__ v) {
+__device__ __forceinline__ void wino_input_block(const Tin* __restrict__ in, const WinoInArgs& a,
+                                                 Tst* __restrict__ v, long long bid, int lx, int ly, int bx,
+                                                 int by) {
   constexpr int A = Wino<M>::A;
   // channel group fastest across blocks, so one tile's V rows are written by
   // blocks that run together
-  const int cgroups = (a.c + blockDim.x - 1) / blockDim.x;
-  const int cg = (int)(blockIdx.x % cgroups);
-  const long long tg = blockIdx.x / cgroups;
-  const int c = cg * blockDim.x + threadIdx.x;
-  const long long t = tg * blockDim.y + threadIdx.y;
+  const int cgroups = (a.c + bx - 1) / bx;
+  const int cg = (int)(bid % cgroups);
+  const long long tg = bid / cgroups;
+  const int c = cg * bx + lx;
+  const long long t = tg * by + ly;
   if (c >= a.c || t >= a.t_count) return;
   const int per_img = a.tiles_h * a.tiles_w;
-  const int nl = (int)(t / per_img);
-  const int r = (int)(t - (long long)nl * per_img);
+  const long long tglob = a.t_base + t;
+  const int nl = (int)(tglob / per_img);
+  const int r = (int)(tglob - (long long)nl * per_img);
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
   const int y0 = ty * M - a.ph, x0 = tx * M - a.pw;
   const Tin* base = in + (long long)(a.n0 + nl) * a.in_img_stride + c;
@@ -139,6 +144,13 @@ wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restric
   }
 }
 
+template <int M, typename Tin, typename Tst, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_input_kernel(const Tin* __restrict__ in, const WinoInArgs a, Tst* __restrict__ v) {
+  wino_input_block<M, Tin, Tst, Idx>(in, a, v, blockIdx.x, threadIdx.x, threadIdx.y, blockDim.x, blockDim.y);
+}
+
+
 // ---------------------------------------------------------------------------
 // Output transform: one thread per (tile, output channel).
 // ---------------------------------------------------------------------------
@@ -146,22 +158,27 @@ struct WinoOutArgs {
   int oh, ow, o, tiles_h, tiles_w;
   long long out_img_stride;
   int n0;
+  long long t_base;       // first tile of this call, counted from image n0's first tile
   long long t_count, t_stride;
   int accumulate;
 };
 
 // TM: the element type of M (fp32, or the 16-bit operand type of the
 // tensor-core path).
+// The body of one output-transform block: block (bidx, bidy) of the grid,
+// thread (tx, ty) of a bx x by block.
 template <int M, typename TM, typename Tout, typename Idx>
-__global__ void __launch_bounds__(256)
-wino_output_kernel(const TM* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
+__device__ __forceinline__ void wino_output_block(const TM* __restrict__ mb, const WinoOutArgs& a,
+                                                  Tout* __restrict__ out, long long bidx, int bidy, int lx, int ly,
+                                                  int bx, int by) {
   constexpr int A = Wino<M>::A;
-  const int o = blockIdx.y * blockDim.x + threadIdx.x;
-  const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
+  const int o = bidy * bx + lx;
+  const long long t = bidx * by + ly;
   if (o >= a.o || t >= a.t_count) return;
   const int per_img = a.tiles_h * a.tiles_w;
-  const int nl = (int)(t / per_img);
-  const int r = (int)(t - (long long)nl * per_img);
+  const long long tglob = a.t_base + t;
+  const int nl = (int)(tglob / per_img);
+  const int r = (int)(tglob - (long long)nl * per_img);
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
 
   const Idx plane = (Idx)(a.t_stride * a.o);
@@ -207,6 +224,39 @@ wino_output_kernel(const TM* __restrict__ mb, const WinoOutArgs a, Tout* __restr
   }
 }
 
+template <int M, typename TM, typename Tout, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_output_kernel(const TM* __restrict__ mb, const WinoOutArgs a, Tout* __restrict__ out) {
+  wino_output_block<M, TM, Tout, Idx>(mb, a, out, blockIdx.x, blockIdx.y, threadIdx.x, threadIdx.y, blockDim.x,
+                                      blockDim.y);
+}
+
+// One pass of the chunked fp32 Winograd pipeline: the output transform of
+// chunk i-1 and the input transform of chunk i in one launch (1D grid of
+// 256-thread blocks, the input blocks first).  The output blocks wait for the
+// previous kernel in the stream (the GEMM of chunk i-1) before reading M; the
+// input blocks do not wait: they read only the conv's input and write the V
+// buffer that the GEMM of chunk i-2 read, which had finished before that
+// previous GEMM could start.  They therefore run in the SMs the previous GEMM
+// frees as it drains.  Every block releases the next launch (the GEMM of
+// chunk i), whose own wait covers this whole grid.
+template <int M, typename Tin, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_pass_kernel(const Tin* __restrict__ in, const WinoInArgs ai, float* __restrict__ v, long long in_blocks, int ibx,
+                 const float* __restrict__ mb, const WinoOutArgs ao, Tin* __restrict__ out, unsigned ogx, int obx) {
+  const long long b = blockIdx.x;
+  if (b < in_blocks) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    wino_input_block<M, Tin, float, Idx>(in, ai, v, b, threadIdx.x % ibx, threadIdx.x / ibx, ibx, 256 / ibx);
+  } else {
+    pdl_wait_then_release();
+    const long long ob = b - in_blocks;
+    wino_output_block<M, float, Tin, Idx>(mb, ao, out, ob % ogx, (int)(ob / ogx), threadIdx.x % obx,
+                                          threadIdx.x / obx, obx, 256 / obx);
+  }
+}
+
+
 // ---------------------------------------------------------------------------
 // 16-bit transforms on channel pairs: a thread owns channels (2p, 2p+1) of one
 // tile, so each load and store moves 32 bits (the arithmetic per channel is
@@ -226,8 +276,9 @@ wino_input_pair_kernel(const T* __restrict__ in, const WinoInArgs a, T* __restri
   const long long t = tg * blockDim.y + threadIdx.y;
   if (c2 >= cp || t >= a.t_count) return;
   const int per_img = a.tiles_h * a.tiles_w;
-  const int nl = (int)(t / per_img);
-  const int r = (int)(t - (long long)nl * per_img);
+  const long long tglob = a.t_base + t;
+  const int nl = (int)(tglob / per_img);
+  const int r = (int)(tglob - (long long)nl * per_img);
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
   const int y0 = ty * M - a.ph, x0 = tx * M - a.pw;
   const PT* base = reinterpret_cast<const PT*>(in + (long long)(a.n0 + nl) * a.in_img_stride) + c2;
@@ -301,8 +352,9 @@ wino_output_pair_kernel(const T* __restrict__ mb, const WinoOutArgs a, T* __rest
   const long long t = (long long)blockIdx.x * blockDim.y + threadIdx.y;
   if (o2 >= op || t >= a.t_count) return;
   const int per_img = a.tiles_h * a.tiles_w;
-  const int nl = (int)(t / per_img);
-  const int r = (int)(t - (long long)nl * per_img);
+  const long long tglob = a.t_base + t;
+  const int nl = (int)(tglob / per_img);
+  const int r = (int)(tglob - (long long)nl * per_img);
   const int ty = r / a.tiles_w, tx = r - (r / a.tiles_w) * a.tiles_w;
 
   const Idx plane = (Idx)(a.t_stride * op);
@@ -518,7 +570,7 @@ cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int
   });
 }
 
-cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int m,
+cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, long long t_base, long long t_count, int m,
                               conv_dtype_t in_dt, conv_dtype_t store_dt, void* v, long long t_tile,
                               cudaStream_t s) {
   WinoInArgs a{};
@@ -527,7 +579,8 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   a.tiles_w = (g.ow + m - 1) / m;
   a.in_img_stride = g.in_img_stride;
   a.n0 = n0;
-  a.t_count = (long long)nb * a.tiles_h * a.tiles_w;
+  a.t_base = t_base;
+  a.t_count = t_count;
   a.t_stride = t_tile;
   if (a.t_count == 0) return cudaSuccess;
   int bx = g.c >= 64 ? 64 : 32;
@@ -577,6 +630,56 @@ cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, int nb, int
   });
 }
 
+cudaError_t launch_wino_pass(const void* in, const Geom& g, int m, conv_dtype_t dt, int n0, long long in_t_base,
+                             long long in_t_count, float* v, long long out_t_base, long long out_t_count,
+                             const float* mb, void* out, bool accumulate, bool pdl, cudaStream_t s) {
+  if (in_t_count == 0 && out_t_count == 0) return cudaSuccess;
+  const int tiles_h = (g.oh + m - 1) / m, tiles_w = (g.ow + m - 1) / m;
+  WinoInArgs ai{};
+  ai.h = g.h; ai.w = g.w; ai.c = g.c; ai.ph = g.ph; ai.pw = g.pw;
+  ai.tiles_h = tiles_h; ai.tiles_w = tiles_w;
+  ai.in_img_stride = g.in_img_stride;
+  ai.n0 = n0;
+  ai.t_base = in_t_base;
+  ai.t_count = in_t_count;
+  ai.t_stride = in_t_count;
+  WinoOutArgs ao{};
+  ao.oh = g.oh; ao.ow = g.ow; ao.o = g.o;
+  ao.tiles_h = tiles_h; ao.tiles_w = tiles_w;
+  ao.out_img_stride = g.out_img_stride;
+  ao.n0 = n0;
+  ao.t_base = out_t_base;
+  ao.t_count = out_t_count;
+  ao.t_stride = out_t_count;
+  ao.accumulate = accumulate ? 1 : 0;
+  const int ibx = g.c >= 64 ? 64 : 32, iby = 256 / ibx;
+  const int obx = g.o >= 64 ? 64 : 32, oby = 256 / obx;
+  const long long in_blocks = ((in_t_count + iby - 1) / iby) * ((g.c + ibx - 1) / ibx);
+  const long long ogx = (out_t_count + oby - 1) / oby, ogy = (g.o + obx - 1) / obx;
+  const long long blocks = in_blocks + ogx * ogy;
+  if (blocks > 0x7fffffffLL || ogx > 0xffffffffLL) return cudaErrorInvalidValue;
+  const int a2 = (m + 2) * (m + 2);
+  const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31) &&
+                     (long long)a2 * in_t_count * g.c < (1LL << 31) && g.out_img_stride < (1LL << 31) &&
+                     (long long)a2 * out_t_count * g.o < (1LL << 31);
+  return wino_by_m(m, [&](auto mc) {
+    constexpr int M = decltype(mc)::value;
+    return wino_by_dt(dt, [&](auto ti) {
+      using Tin = decltype(ti);
+      auto run = [&](auto kernel) {
+        const Tin* ip = static_cast<const Tin*>(in);
+        Tin* op = static_cast<Tin*>(out);
+        if (pdl)
+          return launch_pdl(kernel, dim3((unsigned)blocks), dim3(256), 0, s, ip, ai, v, in_blocks, ibx, mb, ao, op,
+                            (unsigned)ogx, obx);
+        kernel<<<(unsigned)blocks, 256, 0, s>>>(ip, ai, v, in_blocks, ibx, mb, ao, op, (unsigned)ogx, obx);
+        return cudaGetLastError();
+      };
+      return idx32 ? run(wino_pass_kernel<M, Tin, int>) : run(wino_pass_kernel<M, Tin, long long>);
+    });
+  });
+}
+
 cudaError_t launch_wino_filter_cmajor(const void* w, long long w_row_stride, int o, int c, int m,
                                       conv_dtype_t in_dt, long long o_pad, float* u, cudaStream_t s) {
   long long n = (long long)o * c;
@@ -620,16 +723,17 @@ cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int 
   });
 }
 
-cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, int nb, int m,
-                               long long t_tile, conv_dtype_t out_dt, void* out, bool accumulate,
-                               cudaStream_t s) {
+cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, long long t_base,
+                               long long t_count, int m, long long t_tile, conv_dtype_t out_dt, void* out,
+                               bool accumulate, cudaStream_t s) {
   WinoOutArgs a{};
   a.oh = g.oh; a.ow = g.ow; a.o = g.o;
   a.tiles_h = (g.oh + m - 1) / m;
   a.tiles_w = (g.ow + m - 1) / m;
   a.out_img_stride = g.out_img_stride;
   a.n0 = n0;
-  a.t_count = (long long)nb * a.tiles_h * a.tiles_w;
+  a.t_base = t_base;
+  a.t_count = t_count;
   a.t_stride = t_tile;
   a.accumulate = accumulate ? 1 : 0;
   if (a.t_count == 0) return cudaSuccess;
