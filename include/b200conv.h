@@ -122,7 +122,13 @@ typedef struct {
  * A non-NULL options struct ignores the environment.  Independently of the
  * options, B200CONV_LOG=1 makes every conv*_forward call print the plan it
  * runs (algorithm, engine, path, tile, Winograd m and batch tile, channel pad,
- * K split, workspace bytes) as one line on stderr.
+ * K split, workspace bytes) as one line on stderr.  Further test hooks, also
+ * read on every call, select between execution routes that give the same
+ * result: B200CONV_TC_PAIR=0 keeps the tensor-core kernels on 128-row tiles
+ * (no CTA pairs); B200CONV_SPLITK_CLUSTER=1 sums split-K partials inside the
+ * conv kernel (thread-block clusters) instead of the reduce kernel;
+ * B200CONV_WINOGRAD_CHUNK_TILES=<tiles> runs the fp32 Winograd path in chunks
+ * of that many tiles (pipelined transform / GEMM passes; 0 or unset: off).
  */
 typedef struct {
     conv_algo_t algo;                     /* CONV_ALGO_AUTO: let the selector choose */
@@ -160,6 +166,9 @@ B200CONV_API conv_status_t conv_device_props(int device, conv_device_props_t *pr
  * The Winograd budget is 3/4 of the device's total memory minus the conv's own
  * tensors (input, output, transformed filter), capped at 8 GiB because the GPU
  * is shared ("Bound winograd conv2d working set by tiling the batch", Fix).
+ * plan->tile_m == 256 means the tensor-core kernel runs CTA pairs: two SMs
+ * per 256 x 256 output tile (cta_group::2), each holding half of the input
+ * and half of the weight tile.
  */
 B200CONV_API conv_status_t conv2d_plan(const conv2d_desc_t *desc, conv_dtype_t dtype, int device,
                           const conv_options_t *opts, conv_plan_t *plan);

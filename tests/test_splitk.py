@@ -1,16 +1,19 @@
 """Split-K on the tensor cores: the K range of a small-M, long-K implicit GEMM
 is split over several CTAs per output tile ("Use the explicit gemm for wide
 convs on neural accelerators", ResNet-50 follow-up: the small late-stage
-layers).  The splits of a tile run as one thread-block cluster: each split
-leaves its fp32 partial in its own shared memory and every CTA of the cluster
-adds, for a slice of the tile's rows, all splits' partials in split order and
-writes those output rows, with no reduce launch.  The older route (fp32 partials in
-the workspace, then a reduce kernel) sums the same values in the same order.
+layers).  Two routes give the same bits:
+
+* the default: every split writes its fp32 partial to the workspace and a
+  reduce kernel sums the splits in split order;
+* the cluster route (B200CONV_SPLITK_CLUSTER=1, a test hook read on every
+  call): the splits of a tile run as one thread-block cluster, each leaving its
+  partial in its own shared memory, and every CTA of the cluster sums a slice
+  of the tile's rows over the splits in split order and writes those rows,
+  with no reduce launch (taken when a launch's clusters all fit at once).
 
 Checked: both routes agree bit for bit, match the oracle, repeat bit for bit,
-launch no reduce kernel when the clusters fit in one wave, and the depth-tap
-accumulate mode (conv3d) works through the cluster epilogue.  B200CONV_SPLITK_CLUSTER=0 (a
-test hook read on every call) selects the older route.
+the cluster route launches no reduce kernel when its clusters fit in one wave,
+and the depth-tap accumulate mode (conv3d) works through the cluster epilogue.
 """
 import os
 
@@ -69,16 +72,16 @@ def test_cluster_split_k_matches_reduce_route_and_oracle(case, dtype):
     p = _plan(shape, dtype)
     assert p["engine"] == "tcgen05" and p["k_split"] > 1, p
     x, w = synth.conv2d_inputs(shape, dtype, "he", 31, device="cuda")
-    B.conv_profile_begin()
-    got = run_conv2d(x, w, shape)
-    again = run_conv2d(x, w, shape)
-    prof = B.profile_end()
+    with env(B200CONV_SPLITK_CLUSTER=1):
+        B.conv_profile_begin()
+        got = run_conv2d(x, w, shape)
+        again = run_conv2d(x, w, shape)
+        prof = B.profile_end()
     if must_cluster:
         assert "splitk_reduce" not in prof, prof      # summed inside the conv kernel
-    with env(B200CONV_SPLITK_CLUSTER=0):
-        B.conv_profile_begin()
-        ref = run_conv2d(x, w, shape)
-        prof2 = B.profile_end()
+    B.conv_profile_begin()
+    ref = run_conv2d(x, w, shape)                     # the default: partials and the reduce kernel
+    prof2 = B.profile_end()
     assert "splitk_reduce" in prof2, prof2
     assert torch.equal(got.view(torch.int16), again.view(torch.int16))
     assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
@@ -95,11 +98,11 @@ def test_cluster_split_k_accumulates_depth_taps(dtype):
     p = B.plan3d(d, dtype, 0, None)
     assert p["taps"] == 3 and p["k_split"] > 1 and p["engine"] == "tcgen05", p
     x, w = synth.conv3d_inputs(s, dtype, "normal", 32, device="cuda")
-    got = B.conv3d(x, w, s.stride, s.pad, s.dilation)
-    torch.cuda.synchronize()
-    with env(B200CONV_SPLITK_CLUSTER=0):
-        ref = B.conv3d(x, w, s.stride, s.pad, s.dilation)
+    with env(B200CONV_SPLITK_CLUSTER=1):
+        got = B.conv3d(x, w, s.stride, s.pad, s.dilation)
         torch.cuda.synchronize()
+    ref = B.conv3d(x, w, s.stride, s.pad, s.dilation)
+    torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
     assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
     want = oracle.conv3d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
