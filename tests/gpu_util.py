@@ -41,15 +41,21 @@ GUARD_BYTES = 4096          # canary band on each side of out and of the workspa
 GUARD_VALUE = 0x5B          # a byte pattern no kernel writes by accident (not 0, not a NaN half)
 
 
+NAN_BYTE = 0xFF             # 0xFFFF... is a NaN in fp32, bf16 and fp16 alike
+
+
 class Guarded:
     """A device buffer of `nbytes` between two canary bands.  The inner
     region starts 4096 bytes into a fresh allocation (so it keeps the
     allocator's 256-byte alignment) and the upper band starts right at its
-    last byte, so any write past either end lands in a band."""
+    last byte, so any write past either end lands in a band.  Around an input
+    the bands hold NaN bytes, so a read past either end turns into a NaN in
+    the output."""
 
-    def __init__(self, nbytes: int, device):
+    def __init__(self, nbytes: int, device, fill: int = GUARD_VALUE):
         self.nbytes = int(nbytes)
-        self.buf = torch.full((GUARD_BYTES + self.nbytes + GUARD_BYTES,), GUARD_VALUE, dtype=torch.uint8,
+        self.fill = fill
+        self.buf = torch.full((GUARD_BYTES + self.nbytes + GUARD_BYTES,), fill, dtype=torch.uint8,
                               device=device)
 
     def inner(self) -> torch.Tensor:
@@ -61,8 +67,8 @@ class Guarded:
     def assert_intact(self, what: str):
         lo = self.buf[:GUARD_BYTES]
         hi = self.buf[GUARD_BYTES + self.nbytes:]
-        bad_lo = int((lo != GUARD_VALUE).sum())
-        bad_hi = int((hi != GUARD_VALUE).sum())
+        bad_lo = int((lo != self.fill).sum())
+        bad_hi = int((hi != self.fill).sum())
         assert bad_lo == 0 and bad_hi == 0, \
             f"{what}: write outside the buffer ({bad_lo} bytes below, {bad_hi} bytes above)"
 
@@ -76,25 +82,40 @@ def guarded_output(shape, dtype, device):
     return g, out
 
 
+def guarded_input(t: torch.Tensor):
+    """A copy of t inside NaN bands (see Guarded)."""
+    g = Guarded(t.numel() * t.element_size(), t.device, fill=NAN_BYTE)
+    x = g.tensor(tuple(t.shape), t.dtype)
+    x.copy_(t)
+    return g, x
+
+
 def guarded_workspace(nbytes: int, device):
     """The plan's workspace, exactly its size, inside canary bands (None if the plan needs none)."""
     return Guarded(nbytes, device) if nbytes else None
 
 
 def run_conv2d(x, w, shape: synth.Conv2dShape, options=None):
-    """Run through the C ABI with a NaN-poisoned output and the exact workspace
-    the plan asks for, both inside canary bands checked after the call."""
+    """Run through the C ABI with the input and weights inside NaN bands (a read
+    past either end of them reaches the output as a NaN), a NaN-poisoned output
+    and the exact workspace the plan asks for inside canary bands; every band is
+    checked after the call (no write outside out and the workspace, none into
+    the inputs)."""
     desc = B.make_desc2d(shape.n, shape.h, shape.w, shape.c, shape.o, shape.kh, shape.kw, shape.stride, shape.pad,
                          shape.dilation)
     dt = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[x.dtype]
     plan = B.plan2d(desc, dt, x.device.index or 0, options)
+    g_x, xg = guarded_input(x)
+    g_w, wg = guarded_input(w)
     g_out, out = guarded_output((shape.n, shape.oh, shape.ow, shape.o), x.dtype, x.device)
     g_ws = guarded_workspace(plan["workspace_bytes"], x.device)
-    out = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation, options=options, out=out,
+    out = B.conv2d(xg, wg, shape.stride, shape.pad, shape.dilation, options=options, out=out,
                    workspace=g_ws.inner() if g_ws else None)
     torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
     g_out.assert_intact(f"{shape.name()} out")
+    g_x.assert_intact(f"{shape.name()} input")
+    g_w.assert_intact(f"{shape.name()} weights")
     if g_ws:
         g_ws.assert_intact(f"{shape.name()} workspace")
     return out

@@ -20,24 +20,29 @@ import torch
 import oracle
 from dense_convolution_nhwc_b200 import binding as B
 from dense_convolution_nhwc_b200 import synth
-from tests.gpu_util import TOL, as_f64, assert_close, guarded_output, guarded_workspace
+from tests.gpu_util import TOL, as_f64, assert_close, guarded_input, guarded_output, guarded_workspace
 
 pytestmark = pytest.mark.gpu
 
 
 def run3d(x, w, s, options=None):
-    """Through the C ABI with a NaN-poisoned output and the plan's exact
-    workspace, both inside canary bands that must stay untouched."""
+    """Through the C ABI with the inputs inside NaN bands (a read past either
+    end reaches the output as a NaN), a NaN-poisoned output and the plan's exact
+    workspace inside canary bands that must stay untouched."""
     desc = B.make_desc3d(s.n, s.d, s.h, s.w, s.c, s.o, s.kd, s.kh, s.kw, s.stride, s.pad, s.dilation)
     dt = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[x.dtype]
     plan = B.plan3d(desc, dt, x.device.index or 0, options)
+    g_x, xg = guarded_input(x)
+    g_w, wg = guarded_input(w)
     g_out, out = guarded_output((s.n, s.od, s.oh, s.ow, s.o), x.dtype, x.device)
     g_ws = guarded_workspace(plan["workspace_bytes"], x.device)
-    out = B.conv3d(x, w, s.stride, s.pad, s.dilation, options=options, out=out,
+    out = B.conv3d(xg, wg, s.stride, s.pad, s.dilation, options=options, out=out,
                    workspace=g_ws.inner() if g_ws else None)
     torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
     g_out.assert_intact(f"{s.name()} out")
+    g_x.assert_intact(f"{s.name()} input")
+    g_w.assert_intact(f"{s.name()} weights")
     if g_ws:
         g_ws.assert_intact(f"{s.name()} workspace")
     return out
