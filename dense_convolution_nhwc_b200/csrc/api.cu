@@ -223,10 +223,15 @@ int tc_tile_n(const Geom& g, const conv_device_props_t& p) {
 long long round4(long long x) { return (x + 3) & ~3LL; }
 
 // CTA pairs (tile_m = 256, two SMs per tile sharing the weight tile) for
-// 256-wide column tiles when there are enough 256-row tiles to give every SM
-// pair one.  B200CONV_TC_PAIR=0 (a test hook, read on every call) keeps 128-row tiles.
-bool tc_pair_tiles(long long rows, long long batches, int o, int tile_n, const conv_device_props_t& p) {
-  if (tile_n != 256) return false;
+// 256-wide column tiles with a K loop of at least 8 steps of 64 when there are
+// enough 256-row tiles to give every SM pair one.  With a shorter K loop the
+// pair's shared accumulator handshake makes every tile wait for the slower of
+// its two epilogues, and the 128-row tiles are faster (measured on the 16-bit
+// Winograd GEMM: pairs slower at C = 128 and 256, faster at C = 512 and 1024).
+// B200CONV_TC_PAIR=0 (a test hook, read on every call) keeps 128-row tiles.
+bool tc_pair_tiles(long long rows, long long batches, int o, int tile_n, long long ksteps,
+                   const conv_device_props_t& p) {
+  if (tile_n != 256 || ksteps < 8) return false;
   if (const char* e = std::getenv("B200CONV_TC_PAIR"))
     if (std::strcmp(e, "0") == 0) return false;
   const long long tiles = batches * ((rows + 255) / 256) * ((o + 255) / 256);
@@ -329,7 +334,8 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
       s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
-      s->tile_m = tc_gemm && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o, s->tile_n, p) ? 256 : 128;
+      s->tile_m = tc_gemm && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o, s->tile_n,
+                                           (g.c + 63) / 64, p) ? 256 : 128;
       s->chunk = (!tc_gemm && kF32VTileMajor && g.c % 4 == 0) ? winograd_chunk_tiles(g, m, p) : 0;
       const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb, s->chunk);
       s->ws = L.u_bytes + L.v_bytes + L.m_bytes;
@@ -395,7 +401,8 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->split_off = s->ws;
       s->ws += align256((size_t)ks * M * g.o * 4);
     }
-    if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack && tc_pair_tiles(M, 1, g.o, s->tile_n, p))
+    if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack &&
+        tc_pair_tiles(M, 1, g.o, s->tile_n, taps * ((c_eff + 63) / 64), p))
       s->tile_m = 256;
   }
   return CONV_OK;
@@ -806,7 +813,8 @@ conv_status_t plan3d_impl(const conv3d_desc_t* d, conv_dtype_t dt, const conv_de
     s->tile_m = 128;
     const long long m_tiles = ((long long)d->n * *od * g2->oh * g2->ow + 127) / 128;
     s->tile_n = d->o <= 128 || m_tiles * ((d->o + 255) / 256) < p.sm_count ? 128 : 256;
-    s->tile_m = tc_pair_tiles((long long)d->n * *od * g2->oh * g2->ow, 1, d->o, s->tile_n, p) ? 256 : 128;
+    s->tile_m = tc_pair_tiles((long long)d->n * *od * g2->oh * g2->ow, 1, d->o, s->tile_n,
+                              (long long)d->kd * d->kh * d->kw * ((d->c + 63) / 64), p) ? 256 : 128;
     s->wino_m = 0;
     s->nb = d->n;
     s->ntiles = 1;

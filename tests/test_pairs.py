@@ -2,9 +2,9 @@
 (tcgen05 cta_group::2), each holding 128 rows of the input tile and half of
 the weight tile, so the weight tile crosses L2 once per pair instead of once
 per SM -- the wide-C_out regime of "Use the explicit gemm for wide convs on
-neural accelerators" (description).  Used for 256-wide column tiles when
-there are enough 256-row tiles; B200CONV_TC_PAIR=0 (a test hook read on every
-call) keeps 128-row tiles.
+neural accelerators" (description).  Used for 256-wide column tiles with a K
+loop of at least 8 steps of 64 when there are enough 256-row tiles;
+B200CONV_TC_PAIR=0 (a test hook read on every call) keeps 128-row tiles.
 
 Checked against the oracle and against the 128-row kernel, on the implicit
 GEMM (aligned, ragged M with a pair whose second half is past the end,
@@ -49,7 +49,7 @@ SHAPES = [
     synth.Conv2dShape(16, 64, 64, 256, 1024, 3, 3, (1, 1), (1, 1), (1, 1)),     # M = 65536, 256 x 4 tiles
     synth.Conv2dShape(5, 45, 47, 128, 2048, 3, 3, (1, 1), (1, 1), (1, 1)),      # ragged M, last pair half empty
     synth.Conv2dShape(4, 128, 128, 128, 512, 5, 5, (2, 2), (4, 4), (2, 2)),     # stride and dilation
-    synth.Conv2dShape(8, 40, 40, 512, 520, 1, 1, (1, 1), (0, 0), (1, 1)),       # 1x1, O past the last full tile
+    synth.Conv2dShape(8, 40, 40, 1024, 520, 1, 1, (1, 1), (0, 0), (1, 1)),      # 1x1, O past the last full tile
 ]
 
 
@@ -75,7 +75,11 @@ def test_pair_tiles_match_oracle_and_single_cta(shape, dtype):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 def test_pair_tiles_winograd_gemm(dtype):
-    s = synth.Conv2dShape(8, 48, 48, 256, 512, 3, 3, (1, 1), (1, 1), (1, 1))
+    """The 16-bit Winograd GEMM with C = 1024 (16 K steps) runs in pairs; with
+    C = 256 (4 K steps) it keeps 128-row tiles."""
+    short = synth.Conv2dShape(8, 48, 48, 256, 512, 3, 3, (1, 1), (1, 1), (1, 1))
+    assert plan(short, dtype, B.make_options("winograd"))["tile_m"] == 128
+    s = synth.Conv2dShape(4, 48, 48, 1024, 512, 3, 3, (1, 1), (1, 1), (1, 1))
     opts = B.make_options("winograd")
     p = plan(s, dtype, opts)
     assert p["algo"] == "winograd" and p["engine"] == "tcgen05" and p["tile_m"] == 256, p
