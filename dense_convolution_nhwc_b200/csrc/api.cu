@@ -181,6 +181,7 @@ struct Sel {
   int tile_m = 128, tile_n = 128;
   int wino_m = 0, nb = 0, ntiles = 0, cpad = 0;
   bool wpack = false;      // KW taps folded into cpad channels (a few-channel input)
+  bool fpack = false;      // all KH*KW taps folded into cpad channels: a 1x1 conv over them
   int ksplit = 1;          // implicit GEMM: K range split over ksplit CTAs, fp32 partials reduced after
   size_t split_off = 0;    // workspace offset of the partials
   conv_dtype_t wino_store = CONV_F32;
@@ -356,7 +357,16 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     s->tile_m = 128;
     s->tile_n = tc_tile_n(g, p);
     s->wpack = false;
-    if (g.c % 8 != 0 && g.kw > 1 && g.kw * g.c <= 64) {
+    s->fpack = false;
+    if (g.c % 8 != 0 && g.kh * g.kw > 1 && g.kh * g.kw * g.c <= 192) {
+      // a few channels and a small window: fold every tap into channels, the
+      // conv becoming a 1x1 conv over at most 3 full K steps (the ResNet stem's
+      // 7x7x3 = 147 -> 152 channels), instead of KH K steps of mostly padding
+      const int cp = (g.kh * g.kw * g.c + 7) / 8 * 8;
+      s->cpad = cp;
+      s->fpack = true;
+      s->ws = align256((size_t)g.n * g.oh * g.ow * cp * esz) + align256((size_t)g.o * cp * esz);
+    } else if (g.c % 8 != 0 && g.kw > 1 && g.kw * g.c <= 64) {
       // a few channels: fold the KW taps into channels (KH x 1 conv over KW*C)
       const int cp = (g.kw * g.c + 7) / 8 * 8;
       s->cpad = cp;
@@ -385,7 +395,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
   const long long M = (long long)g.n * g.oh * g.ow;
   if (s->algo == CONV_ALGO_IMPLICIT_GEMM && M > 0) {
     const int c_eff = s->cpad ? s->cpad : g.c;
-    const long long taps = s->wpack ? g.kh : (long long)g.kh * g.kw;
+    const long long taps = s->fpack ? 1 : (s->wpack ? g.kh : (long long)g.kh * g.kw);
     long long ks = 1;
     if (s->engine == CONV_ENGINE_TCGEN05) {
       const long long ksteps = taps * ((c_eff + 63) / 64);
@@ -401,7 +411,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->split_off = s->ws;
       s->ws += align256((size_t)ks * M * g.o * 4);
     }
-    if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack &&
+    if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack && !s->fpack &&
         tc_pair_tiles(M, 1, g.o, s->tile_n, taps * ((c_eff + 63) / 64), p))
       s->tile_m = 256;
   }
@@ -417,7 +427,7 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->batch_tile = s.nb;
   plan->num_batch_tiles = s.ntiles;
   plan->channel_pad = s.cpad;
-  plan->packed_taps = s.wpack ? 1 : 0;
+  plan->packed_taps = s.fpack ? 2 : (s.wpack ? 1 : 0);
   plan->k_split = s.ksplit;
   plan->taps = taps;
   plan->workspace_bytes = ws;
@@ -445,7 +455,8 @@ void log_plan(const char* op, const char* shape, conv_dtype_t dt, const Sel& s, 
                "b200conv: %s %s %s -> algo=%s engine=%s path=%s tile=%dx%d winograd_m=%d batch_tile=%d "
                "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d workspace=%zu\n",
                op, shape, dtype_name(dt), algo_name(s.algo), s.engine == CONV_ENGINE_TCGEN05 ? "tcgen05" : "simt",
-               path, s.tile_m, s.tile_n, s.wino_m, s.nb, s.ntiles, s.cpad, s.wpack ? 1 : 0, s.ksplit, ws);
+               path, s.tile_m, s.tile_n, s.wino_m, s.nb, s.ntiles, s.cpad, s.fpack ? 2 : (s.wpack ? 1 : 0), s.ksplit,
+               ws);
 }
 
 // ------------------------------- execution -----------------------------------
@@ -552,7 +563,32 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
   const void* cin = in;
   const void* cw = w;
   Geom gg = g;
-  if (s.wpack) {
+  if (s.fpack) {
+    void* pin = base;
+    void* pw = base + align256((size_t)g.n * g.oh * g.ow * s.cpad * esz);
+    cudaError_t e;
+    {
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_fullpack(in, g, pin, s.cpad, dt, d.props.sm_count, st);
+    }
+    if (e == cudaSuccess) {
+      // w[o][kh][kw][c]: rows of KH*KW*C values -> [o][cp]
+      ProfScope ps(K_CHANNEL_PAD, st);
+      e = launch_channel_pad(w, g.o, 1, g.kh * g.kw * g.c, g.w_row_stride, pw, s.cpad, dt, st);
+    }
+    if (e != cudaSuccess) return CONV_ERR_CUDA;
+    cin = pin;
+    cw = pw;
+    gg.h = g.oh;
+    gg.w = g.ow;
+    gg.c = s.cpad;
+    gg.kh = gg.kw = 1;
+    gg.sh = gg.sw = 1;
+    gg.ph = gg.pw = 0;
+    gg.dh = gg.dw = 1;
+    gg.in_img_stride = (long long)g.oh * g.ow * s.cpad;
+    gg.w_row_stride = s.cpad;
+  } else if (s.wpack) {
     void* pin = base;
     void* pw = base + align256((size_t)g.n * g.h * g.ow * s.cpad * esz);
     cudaError_t e;

@@ -210,6 +210,195 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count,
   return cudaErrorInvalidValue;
 }
 
+// Full tap packing for a few-channel input (the ResNet stem): the conv becomes a
+// 1x1 conv over cp = KH*KW*C rounded up to 8 packed channels, packed channel
+// k = (kh*KW + kw)*C + c of output pixel (n, oy, ox) holding
+// src[n][oy*sh - ph + kh*dh][ox*sw - pw + kw*dw][c] (zero outside the image and
+// for k >= KH*KW*C).  One thread writes 8 consecutive packed channels (16 bytes
+// for 16-bit types) of one pixel, so neighbouring threads write neighbouring
+// bytes; (kh, kw, c) are decoded once per thread and then stepped.
+template <typename T, typename Idx>
+__global__ void __launch_bounds__(256)
+fullpack_kernel(const T* __restrict__ src, Idx chunks, int chunks_per_px, int oh, int ow, int h, int w, int c,
+                int kh, int kw, int sh, int sw, int ph, int pw, int dh, int dw, long long in_img_stride,
+                T* __restrict__ dst, int cp) {
+  const int ktot = kh * kw * c;
+  const int kwc = kw * c;
+  const Idx ohw = (Idx)oh * ow;
+  for (Idx i = (Idx)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += (Idx)gridDim.x * blockDim.x) {
+    const Idx px = i / chunks_per_px;
+    const int chunk = (int)(i - px * chunks_per_px);
+    const Idx nimg = px / ohw;
+    const int r = (int)(px - nimg * ohw);
+    const int oy = r / ow, ox = r - (r / ow) * ow;
+    const T* img = src + (long long)nimg * in_img_stride;
+    int k = chunk * 8;
+    int ky = k / kwc;
+    int rem = k - ky * kwc;
+    int kx = rem / c, cc = rem - kx * c;
+    const int y0 = oy * sh - ph, x0 = ox * sw - pw;
+    __align__(16) T v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int y = y0 + ky * dh, x = x0 + kx * dw;
+      const bool ok = k < ktot && y >= 0 && y < h && x >= 0 && x < w;
+      v[e] = ok ? img[((Idx)y * w + x) * c + cc] : Store<T>::from_f32(0.0f);
+      ++k;
+      if (++cc == c) {
+        cc = 0;
+        if (++kx == kw) {
+          kx = 0;
+          ++ky;
+        }
+      }
+    }
+    T* out = dst + (long long)px * cp + chunk * 8;
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(v);
+    } else {
+      *reinterpret_cast<float4*>(out) = *reinterpret_cast<const float4*>(v);
+      *reinterpret_cast<float4*>(out + 4) = *reinterpret_cast<const float4*>(v + 4);
+    }
+  }
+}
+
+// The same packing, staged: one block takes up to P consecutive output pixels of
+// one output row.  It first copies the KH input rows those pixels read (the
+// span of columns they reach, zero outside the image) into shared memory, and a
+// table mapping packed channel k to its offset in that staged span; every packed
+// value of pixel p is then tile[p*sw*C + tab[k]], so no packed value needs an
+// index decode of its own.
+template <typename T>
+__global__ void __launch_bounds__(256, 8)
+fullpack_rows_kernel(const T* __restrict__ src, int oh, int ow, int h, int w, int c, int kh, int kw, int sh,
+                     int sw, int ph, int pw, int dh, int dw, long long in_img_stride, T* __restrict__ dst, int cp,
+                     int P, int xtiles) {
+  extern __shared__ __align__(16) unsigned char fp_smem[];
+  int* tab = reinterpret_cast<int*>(fp_smem);
+  T* tile = reinterpret_cast<T*>(fp_smem + (size_t)cp * sizeof(int));
+  const T zero = Store<T>::from_f32(0.0f);
+  const int bd = blockDim.x;
+  const int b = blockIdx.x;
+  const int xt = b % xtiles;
+  const int rest = b / xtiles;
+  const int oy = rest % oh;
+  const long long nimg = rest / oh;
+  const int ox0 = xt * P;
+  const int np = min(P, ow - ox0);
+  const int L = ((np - 1) * sw + (kw - 1) * dw + 1) * c;   // staged elements per input row
+  const int xs = ox0 * sw - pw;                             // first staged input column
+  const int kwc = kw * c, ktot = kh * kwc;
+  for (int k = threadIdx.x; k < cp; k += bd) {
+    int t = -1;
+    if (k < ktot) {
+      const int ky = k / kwc, r = k - ky * kwc;
+      const int kx = r / c, cc = r - kx * c;
+      t = ky * L + kx * dw * c + cc;
+    }
+    tab[k] = t;
+  }
+  const T* img = src + nimg * in_img_stride;
+  // staged elements e in [lo, hi) of a row lie inside the image columns
+  const int lo = max(0, -xs * c), hi = min(L, (w - xs) * c);
+  for (int ky = 0; ky < kh; ++ky) {
+    const int y = oy * sh - ph + ky * dh;
+    T* trow = tile + ky * L;
+    if (y < 0 || y >= h) {
+      for (int e = threadIdx.x; e < L; e += bd) trow[e] = zero;
+      continue;
+    }
+    const T* row = img + ((long long)y * w + xs) * c;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < L; e += bd) trow[e] = (e >= lo && e < hi) ? row[e] : zero;
+  }
+  __syncthreads();
+  // The block is a whole number R of rows of cp/2 threads: each thread owns one
+  // pair of adjacent packed channels (its two tap offsets held in registers) and
+  // steps through pixels p, p + R, ...; a warp writes contiguous bytes.
+  struct alignas(2 * sizeof(T)) V2 {
+    T x, y;
+  };
+  const int cph = cp / 2;
+  const int R = bd / cph;
+  if (threadIdx.x >= R * cph) return;
+  const int k2 = threadIdx.x % cph;
+  int p = threadIdx.x / cph;
+  const int2 t = reinterpret_cast<const int2*>(tab)[k2];
+  const bool v0 = t.x >= 0, v1 = t.y >= 0;
+  const T* b0 = tile + p * sw * c + (v0 ? t.x : 0);
+  const T* b1 = tile + p * sw * c + (v1 ? t.y : 0);
+  const int pstep = R * sw * c;
+  T* o = dst + (((nimg * oh + oy) * ow + ox0 + p) * (long long)cp + 2 * k2);
+  const long long ostep = (long long)R * cp;
+  for (; p < np; p += R) {
+    V2 v;
+    v.x = v0 ? *b0 : zero;
+    v.y = v1 ? *b1 : zero;
+    *reinterpret_cast<V2*>(o) = v;
+    b0 += pstep;
+    b1 += pstep;
+    o += ostep;
+  }
+}
+
+cudaError_t launch_fullpack(const void* src, const Geom& g, void* dst, int cp, conv_dtype_t dt, int sm_count,
+                            cudaStream_t s) {
+  if (cp % 8 != 0) return cudaErrorInvalidValue;
+  const long long px = (long long)g.n * g.oh * g.ow;
+  const long long chunks = px * (cp / 8);
+  if (chunks == 0) return cudaSuccess;
+  // Staged form: the widest row segment (at most 128 pixels) whose staged input
+  // rows and tap table fit 48 KB of shared memory, narrowed (to no less than 16
+  // pixels) while that leaves fewer than eight blocks per SM.  The block is the
+  // largest whole number of cp/2-thread rows within 256 threads.
+  const int esz = dt == CONV_F32 ? 4 : 2;
+  auto smem_for = [&](long long P) {
+    return (long long)cp * 4 + (long long)g.kh * ((P - 1) * g.sw + (long long)(g.kw - 1) * g.dw + 1) * g.c * esz;
+  };
+  long long P = g.ow < 128 ? g.ow : 128;
+  while (P > 1 && smem_for(P) > 48 * 1024) P /= 2;
+  while (P >= 32 && (long long)g.n * g.oh * ((g.ow + P - 1) / P) < 8LL * sm_count) P = (P + 1) / 2;
+  const long long xtiles = (g.ow + P - 1) / P;
+  const long long row_blocks = (long long)g.n * g.oh * xtiles;
+  if (cp <= 512 && smem_for(P) <= 48 * 1024 && row_blocks < (1LL << 31)) {
+    const size_t smem = (size_t)smem_for(P);
+    auto staged = [&](auto tag) {
+      using T = decltype(tag);
+      fullpack_rows_kernel<T><<<(unsigned)row_blocks, (cp / 2) * (256 / (cp / 2)), smem, s>>>(
+          static_cast<const T*>(src), g.oh, g.ow, g.h, g.w, g.c, g.kh, g.kw, g.sh, g.sw, g.ph, g.pw, g.dh, g.dw,
+          g.in_img_stride, static_cast<T*>(dst), cp, (int)P, (int)xtiles);
+      return cudaGetLastError();
+    };
+    switch (dt) {
+      case CONV_F32: return staged(float{});
+      case CONV_F16: return staged(__half{});
+      case CONV_BF16: return staged(__nv_bfloat16{});
+    }
+    return cudaErrorInvalidValue;
+  }
+  unsigned blocks = (unsigned)((chunks + 255) / 256 < 148 * 32 ? (chunks + 255) / 256 : 148 * 32);
+  // 32-bit index arithmetic when the chunk count and one image fit
+  const bool idx32 = chunks < (1LL << 31) && g.in_img_stride < (1LL << 31);
+  auto go = [&](auto tag) {
+    using T = decltype(tag);
+    if (idx32)
+      fullpack_kernel<T, int><<<blocks, 256, 0, s>>>(static_cast<const T*>(src), (int)chunks, cp / 8, g.oh, g.ow,
+                                                     g.h, g.w, g.c, g.kh, g.kw, g.sh, g.sw, g.ph, g.pw, g.dh, g.dw,
+                                                     g.in_img_stride, static_cast<T*>(dst), cp);
+    else
+      fullpack_kernel<T, long long><<<blocks, 256, 0, s>>>(static_cast<const T*>(src), chunks, cp / 8, g.oh, g.ow,
+                                                           g.h, g.w, g.c, g.kh, g.kw, g.sh, g.sw, g.ph, g.pw, g.dh,
+                                                           g.dw, g.in_img_stride, static_cast<T*>(dst), cp);
+    return cudaGetLastError();
+  };
+  switch (dt) {
+    case CONV_F32: return go(float{});
+    case CONV_F16: return go(__half{});
+    case CONV_BF16: return go(__nv_bfloat16{});
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,
                          long long in_img_stride, void* dst, int cp, conv_dtype_t dt, cudaStream_t s) {
   if (cp % 8 != 0) return cudaErrorInvalidValue;

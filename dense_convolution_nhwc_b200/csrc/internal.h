@@ -149,6 +149,11 @@ cudaError_t launch_fill_zero(void* out, size_t bytes, cudaStream_t s);
 // for channels >= kw*c); dst is dense [n][h][ow][cp].
 cudaError_t launch_wpack(const void* src, long long n, int h, int w, int c, int kw, int sw, int pw, int dw, int ow,
                          long long in_img_stride, void* dst, int cp, conv_dtype_t dt, cudaStream_t s);
+// Full tap packing: dst[n][oy][ox][k] for k < cp (a multiple of 8) holds the input
+// value under tap (kh, kw) and channel c, k = (kh*KW + kw)*C + c (zero outside the
+// image and for k >= KH*KW*C); the conv then runs as a 1x1 conv over cp channels.
+cudaError_t launch_fullpack(const void* src, const Geom& g, void* dst, int cp, conv_dtype_t dt, int sm_count,
+                            cudaStream_t s);
 // Channel pad: dst[a][b][c'] = c' < c ? src[a*src_outer_stride + b*c + c'] : 0 for a < outer,
 // b < inner, c' < cp; dst is dense [outer][inner][cp].  Element strides.
 cudaError_t launch_channel_pad(const void* src, long long outer, long long inner, int c,

@@ -146,7 +146,8 @@ typedef struct {
                                   tile of m output frames) slab */
     int num_batch_tiles;       /* number of batch tiles */
     int channel_pad;           /* padded channel count of the pre-pass, 0 if none */
-    int packed_taps;           /* 1 if the KW taps are folded into channel_pad channels (few-channel inputs) */
+    int packed_taps;           /* few-channel inputs: 1 if the KW taps are folded into channel_pad channels
+                                  (a KH x 1 conv over them), 2 if all KH*KW taps are (a 1 x 1 conv); else 0 */
     int k_split;               /* implicit GEMM: K range split over this many CTAs (fp32 partials), 1 if none */
     int taps;                  /* conv3d: number of depth taps (KD); 1 for conv2d */
     size_t workspace_bytes;    /* bytes the caller must pass to *_forward */

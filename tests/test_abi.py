@@ -112,13 +112,26 @@ def test_tiny_spatial_shape_falls_back_with_one_image_tiles():
     assert st == 0 and p["algo"] == "winograd" and p["num_batch_tiles"] == 1
 
 
+def test_few_channel_tap_packing_choice():
+    """A few-channel input folds every tap into channels when KH*KW*C <= 192
+    (at most three 64-wide K steps), only the KW taps when KW*C <= 64 and the
+    window is larger, else pads the channels to a multiple of 8."""
+    cases = [((1, 32, 32, 3, 64, 7, 7), 2, 152), ((1, 32, 32, 3, 16, 3, 3), 2, 32), ((1, 32, 32, 5, 16, 5, 5), 2, 128),
+             ((1, 32, 32, 6, 16, 7, 7), 1, 48), ((1, 32, 32, 12, 16, 1, 1), 0, 16)]
+    for (n, h, w, c, o, kh, kw), packed, cp in cases:
+        s = synth.Conv2dShape(n, h, w, c, o, kh, kw, (1, 1), (kh // 2, kw // 2), (1, 1))
+        st, p = plan2d(s, "bf16")
+        assert st == 0 and p["engine"] == "tcgen05", s
+        assert p["packed_taps"] == packed and p["channel_pad"] == cp, (s, p)
+
+
 def test_sixteen_bit_takes_tensor_cores():
     for name, shape, _ in synth.resnet50_layers(8):
         for dt in ("f16", "bf16"):
             st, p = plan2d(shape, dt)
             assert st == 0 and p["algo"] == "implicit" and p["engine"] == "tcgen05", name
-            if shape.c == 3:      # the stem: 7 taps x 3 channels folded into 24 channels
-                assert p["channel_pad"] == 24 and p["packed_taps"] == 1 and p["workspace_bytes"] > 0
+            if shape.c == 3:      # the stem: 7 x 7 taps x 3 channels folded into 152 channels, a 1x1 conv
+                assert p["channel_pad"] == 152 and p["packed_taps"] == 2 and p["workspace_bytes"] > 0
             else:
                 assert p["channel_pad"] == 0 and (p["workspace_bytes"] == 0) == (p["k_split"] == 1)
 

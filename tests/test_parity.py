@@ -67,6 +67,33 @@ def test_multi_tile(shape, dtype):
     check_conv2d(shape, dtype)
 
 
+# Few-channel inputs with every tap folded into channels (KH*KW*C <= 192): the
+# conv runs as a 1x1 conv over the packed channels.  Strides, padding,
+# dilation, rectangular windows and C from 1 to 7.
+FULLPACK = [
+    synth.Conv2dShape(2, 30, 31, 3, 64, 7, 7, (2, 2), (3, 3), (1, 1)),
+    synth.Conv2dShape(1, 17, 19, 1, 40, 3, 3, (1, 1), (1, 1), (2, 2)),
+    synth.Conv2dShape(2, 20, 20, 5, 24, 5, 5, (2, 2), (2, 2), (1, 1)),
+    synth.Conv2dShape(1, 9, 33, 2, 8, 3, 5, (1, 2), (1, 2), (2, 1)),
+    synth.Conv2dShape(3, 12, 12, 7, 16, 1, 3, (1, 1), (0, 1), (1, 1)),
+    # packing staged in 128-pixel row segments: 300 output columns end in a ragged 44
+    synth.Conv2dShape(1, 5, 300, 3, 16, 3, 3, (1, 1), (1, 1), (1, 1)),
+    # 32 staged input rows of (127*8 + 128 + 1) values overflow 48 KB: 64-pixel segments
+    synth.Conv2dShape(1, 40, 921, 1, 16, 32, 2, (1, 8), (0, 0), (1, 128)),
+    # 96 rows of 257 values exceed 48 KB even for one pixel: the unstaged packing kernel
+    synth.Conv2dShape(1, 100, 20, 1, 8, 96, 2, (1, 1), (0, 128), (1, 256)),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("shape", FULLPACK, ids=lambda s: s.name())
+def test_full_tap_packing(shape, dtype):
+    d = B.make_desc2d(shape.n, shape.h, shape.w, shape.c, shape.o, shape.kh, shape.kw, shape.stride, shape.pad,
+                      shape.dilation)
+    assert B.plan2d(d, dtype, 0, None)["packed_taps"] == 2
+    check_conv2d(shape, dtype)
+
+
 WINO = [
     synth.Conv2dShape(2, 20, 20, 64, 96, 3, 3, (1, 1), (1, 1), (1, 1)),     # ragged 6x6 tiles
     synth.Conv2dShape(3, 13, 29, 32, 64, 3, 3, (1, 1), (0, 0), (1, 1)),     # no padding
