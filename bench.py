@@ -164,6 +164,11 @@ def kernel_work(conv, plan):
         T = s.n * math.ceil(s.oh / m) * math.ceil(s.ow / m)
         st = 4 if plan["engine"] == "simt" else esz
         add("wino_filter", 0.0, w_b + a2 * s.o * s.c * st)
+        if plan.get("winograd_fused"):
+            # one persistent kernel: the GEMM's FLOPs; bytes = input + output + the V and M
+            # round trips through its per-CTA scratch
+            add("wino_fused", 2.0 * a2 * T * s.c * s.o, in_b + out_b + 2 * a2 * T * (s.c + s.o) * 4)
+            return w
         add("wino_input", 0.0, in_b + a2 * T * s.c * st)
         gk = "wino_gemm_tc" if plan["engine"] == "tcgen05" else "wino_gemm_simt"
         # M is fp32 on the FFMA path and in the 16-bit operand type on the tensor-core path
@@ -181,13 +186,14 @@ def kernel_work(conv, plan):
 def kernel_bound(name):
     if name in ("tc_conv", "tc_conv3d", "wino_gemm_tc", "wino3d_gemm_tc"):
         return "tensor"
-    if name in ("simt_conv", "wino_gemm_simt", "wino3d_gemm_simt"):
+    if name in ("simt_conv", "wino_gemm_simt", "wino3d_gemm_simt", "wino_fused"):
         return "alu"
     return "hbm"
 
 
 KERNEL_SOURCES = {
     "simt_conv": ["simt_conv.cu", "common.cuh"], "wino_gemm_simt": ["wino_gemm_f32.cu"],
+    "wino_fused": ["wino_fused_f32.cu", "wino_tile.cuh", "mbar.cuh", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "tc_conv": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "tc_conv3d": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "wino_input": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],

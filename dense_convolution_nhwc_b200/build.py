@@ -16,8 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libb200conv.so")
 SOURCES = ["api.cu", "simt_conv.cu", "tc_conv.cu", "winograd.cu", "elementwise.cu", "static_scratch.cu", "wino_gemm_f32.cu",
-           "winograd3d.cu", "probe.cu"]
-HEADERS = ["internal.h", "common.cuh", "winograd_gen.cuh", "wino_1d.cuh", "tc_ptx.cuh", os.path.join("..", "..", "include", "b200conv.h")]
+           "winograd3d.cu", "probe.cu", "wino_fused_f32.cu"]
+HEADERS = ["internal.h", "common.cuh", "winograd_gen.cuh", "wino_1d.cuh", "tc_ptx.cuh", "mbar.cuh", "wino_tile.cuh", os.path.join("..", "..", "include", "b200conv.h")]
 
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

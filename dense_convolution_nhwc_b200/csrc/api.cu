@@ -86,11 +86,11 @@ long long out_extent(long long in, int k, int s, int p, int d) {
 
 enum Kind { K_TC_CONV, K_TC_CONV3D, K_SIMT_CONV, K_SPLITK_REDUCE, K_WINO_FILTER, K_WINO_INPUT, K_WINO_GEMM_TC, K_WINO_GEMM_SIMT,
             K_WINO_OUTPUT, K_WINO3D_FILTER, K_WINO3D_INPUT, K_WINO3D_GEMM_TC, K_WINO3D_GEMM_SIMT, K_WINO3D_OUTPUT,
-            K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_WINO_PASS, K_COUNT };
+            K_ACCUMULATE, K_CHANNEL_PAD, K_FILL, K_WINO_PASS, K_WINO_FUSED, K_COUNT };
 const char* const kKindName[K_COUNT] = {"tc_conv", "tc_conv3d", "simt_conv", "splitk_reduce", "wino_filter", "wino_input", "wino_gemm_tc",
                                         "wino_gemm_simt", "wino_output", "wino3d_filter", "wino3d_input", "wino3d_gemm_tc",
                                         "wino3d_gemm_simt", "wino3d_output", "accumulate", "channel_pad", "fill",
-                                        "wino_pass"};
+                                        "wino_pass", "wino_fused"};
 
 struct ProfRecord {
   int kind;
@@ -186,6 +186,8 @@ struct Sel {
   size_t split_off = 0;    // workspace offset of the partials
   conv_dtype_t wino_store = CONV_F32;
   long long chunk = 0;     // Winograd: tiles per transform -> GEMM -> transform pass (0: the whole batch tile)
+  bool fused = false;      // fp32 Winograd as one persistent kernel (transforms overlapped with the GEMM)
+  int fused_grid = 0;      // its CTAs (one per SM)
   size_t ws = 0;
 };
 
@@ -280,6 +282,26 @@ WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m
   return L;
 }
 
+// The persistent fp32 Winograd kernel (transforms overlapped with the FFMA
+// GEMM inside each CTA) against the three-launch path: it needs F(6x6,3x3)
+// with fp32 input and tile-major V.  It is measured slower than the three
+// launches on the 40 x 512 x 512, 192 -> 96 case (19.5 against 18.4 ms), so
+// it runs only when B200CONV_WINOGRAD_FUSED=1 (a test hook, read on every
+// call; =0 or unset keeps the three launches).  kFusedMinBlocksPerSm is the
+// rule it would take by default: enough 128-tile blocks that every SM gets at
+// least eight (its first input transform and last output transform are not
+// overlapped).
+constexpr bool kFusedByDefault = false;
+constexpr long long kFusedMinBlocksPerSm = 8;
+bool winograd_fused_wanted(const Geom& g, conv_dtype_t dt, int m, long long tiles, const conv_device_props_t& p) {
+  if (dt != CONV_F32 || m != 6 || !kF32VTileMajor || !wino_fused_f32_shape_ok(g)) return false;
+  if (const char* e = std::getenv("B200CONV_WINOGRAD_FUSED")) {
+    if (std::strcmp(e, "0") == 0) return false;
+    if (std::strcmp(e, "1") == 0) return true;
+  }
+  return kFusedByDefault && wino_fused_f32_blocks(tiles) >= kFusedMinBlocksPerSm * p.sm_count;
+}
+
 // Tiles per chunk of the fp32 Winograd pass (FFMA GEMM, tile-major V).  0
 // keeps the whole batch tile in one pass.  B200CONV_WINOGRAD_CHUNK_TILES
 // overrides it (a test hook, read on every call).
@@ -324,6 +346,31 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     nb = std::min<long long>(nb, g.n);
     const bool forced_tile = o.winograd_tile_batch > 0;
     if (forced_tile) nb = std::min<long long>(nb, o.winograd_tile_batch);
+    // The persistent fp32 kernel: per-CTA scratch in place of the batch tile's V and M
+    if (!forced_tile && !tc_gemm && winograd_fused_wanted(g, dt, m, (long long)g.n * tiles_per_img, p)) {
+      const long long blocks = wino_fused_f32_blocks((long long)g.n * tiles_per_img);
+      int grid = (int)std::min<long long>(p.sm_count, blocks);
+      // B200CONV_WINOGRAD_FUSED_GRID=<ctas> (a test hook) runs fewer CTAs, each taking more blocks
+      if (const char* e = std::getenv("B200CONV_WINOGRAD_FUSED_GRID"))
+        if (std::atoi(e) > 0) grid = (int)std::min<long long>(std::atoi(e), blocks);
+      const size_t scratch = align256((size_t)grid * wino_fused_f32_cta_bytes(g.c, g.o));
+      if ((long long)scratch <= budget) {
+        s->algo = CONV_ALGO_WINOGRAD;
+        s->engine = CONV_ENGINE_SIMT;
+        s->wino_m = m;
+        s->wino_store = store;
+        s->nb = g.n;
+        s->ntiles = 1;
+        s->tile_n = wino_gemm_f32_tile_n(g.o);
+        s->tile_m = 128;
+        s->chunk = 0;
+        s->fused = true;
+        s->fused_grid = grid;
+        s->ws = u_bytes + scratch;
+        s->cpad = 0;
+        return CONV_OK;
+      }
+    }
     const long long r_min = (long long)p.sm_count * 128;
     bool fallback = nb <= 0 || (!forced_tile && nb < g.n && nb * tiles_per_img < r_min);
     if (fallback && o.algo == CONV_ALGO_WINOGRAD) return CONV_ERR_UNSUPPORTED;
@@ -430,6 +477,7 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->packed_taps = s.fpack ? 2 : (s.wpack ? 1 : 0);
   plan->k_split = s.ksplit;
   plan->taps = taps;
+  plan->winograd_fused = s.fused ? 1 : 0;
   plan->workspace_bytes = ws;
 }
 
@@ -453,10 +501,10 @@ const char* algo_name(conv_algo_t a) {
 void log_plan(const char* op, const char* shape, conv_dtype_t dt, const Sel& s, const char* path, size_t ws) {
   std::fprintf(stderr,
                "b200conv: %s %s %s -> algo=%s engine=%s path=%s tile=%dx%d winograd_m=%d batch_tile=%d "
-               "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d workspace=%zu\n",
+               "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d fused=%d workspace=%zu\n",
                op, shape, dtype_name(dt), algo_name(s.algo), s.engine == CONV_ENGINE_TCGEN05 ? "tcgen05" : "simt",
                path, s.tile_m, s.tile_n, s.wino_m, s.nb, s.ntiles, s.cpad, s.fpack ? 2 : (s.wpack ? 1 : 0), s.ksplit,
-               ws);
+               s.fused ? 1 : 0, ws);
 }
 
 // ------------------------------- execution -----------------------------------
@@ -490,6 +538,14 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
                  : launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
     }
     if (e != cudaSuccess) return CONV_ERR_CUDA;
+    if (s.fused) {
+      // one persistent launch: per-CTA V and M scratch right after U
+      ProfScope ps(K_WINO_FUSED, st);
+      e = launch_wino_fused_f32(static_cast<const float*>(in), g, static_cast<const float*>(u), round4(g.o),
+                                static_cast<float*>(out), reinterpret_cast<float*>(base + L.u_bytes), s.fused_grid,
+                                accumulate, d.err_word, st);
+      return e == cudaSuccess ? CONV_OK : CONV_ERR_CUDA;
+    }
     const bool tmajor = kF32VTileMajor && g.c % 4 == 0;
     if (s.chunk > 0) {
       // Chunked pipeline: per batch tile, chunks of at most s.chunk tiles, so V

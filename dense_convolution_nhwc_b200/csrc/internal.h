@@ -17,6 +17,8 @@ enum DevErr : int {
   DEVERR_TIMEOUT_MMA_FULL = 0x102,   // MMA issuer waited too long for a loaded stage
   DEVERR_TIMEOUT_MMA_TMEM = 0x103,   // MMA issuer waited too long for a drained accumulator
   DEVERR_TIMEOUT_EPILOGUE = 0x104,   // epilogue waited too long for a finished accumulator
+  DEVERR_TIMEOUT_FUSED_GEMM = 0x105,   // persistent fp32 Winograd: a GEMM unit waited too long for V or a free M
+  DEVERR_TIMEOUT_FUSED_XFORM = 0x106,  // persistent fp32 Winograd: the transform warps waited too long for the GEMM
   DEVERR_TIMEOUT_SELFTEST = 0x1ff,   // the watchdog self-test's deliberate wait
 };
 
@@ -123,6 +125,16 @@ cudaError_t launch_wino_input_cmajor(const void* in, const Geom& g, int n0, int 
 cudaError_t launch_wino_gemm_f32(const float* a, const float* b, float* d, int batches, int t, int c, int o,
                                  long long lda, long long ldb, bool a_tmajor, cudaStream_t s);
 int wino_gemm_f32_tile_n(int o);
+
+// The fp32 Winograd F(6x6,3x3) conv as one persistent kernel (input transform,
+// FFMA GEMM and output transform overlapped inside each CTA, blocks of 128
+// tiles).  u: the transformed filter [64][C][ldb] (ldb = O rounded up to 4);
+// scratch: grid x wino_fused_f32_cta_bytes(C, O) bytes, 16-byte aligned.
+bool wino_fused_f32_shape_ok(const Geom& g);
+size_t wino_fused_f32_cta_bytes(int c, int o);
+long long wino_fused_f32_blocks(long long tiles);
+cudaError_t launch_wino_fused_f32(const float* in, const Geom& g, const float* u, long long ldb, float* out,
+                                  float* scratch, int grid, bool accumulate, int* err_word, cudaStream_t s);
 // M [a2][t_tile][O] in m_dt (fp32, or the 16-bit operand type of the tensor-core path).
 cudaError_t launch_wino_output(const void* mbuf, conv_dtype_t m_dt, const Geom& g, int n0, long long t_base,
                                long long t_count, int m, long long t_tile, conv_dtype_t out_dt, void* out,

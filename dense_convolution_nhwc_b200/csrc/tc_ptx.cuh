@@ -1,11 +1,8 @@
 // tc_ptx.cuh -- the sm_100a building blocks shared by the tcgen05 kernels:
-// bounded mbarrier waits, TMA loads and stores, tcgen05 MMA / commit / TMEM
-// loads, the UMMA descriptors, and the host-side tensor-map encoders (reached
-// through the runtime's driver entry points, so no -lcuda).
-//
-// Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that runs
-// out records a code in the device error word and raises a CTA-wide abort
-// flag, so a fault in a pipeline can never hang the GPU.
+// TMA loads and stores, tcgen05 MMA / commit / TMEM loads, the UMMA
+// descriptors, cluster helpers, and the host-side tensor-map encoders (reached
+// through the runtime's driver entry points, so no -lcuda).  The bounded
+// mbarrier waits they use are in mbar.cuh.
 #pragma once
 
 #include <cuda.h>
@@ -17,61 +14,10 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mbar.cuh"
 
 namespace b200conv {
 namespace {
-
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-
-// ------------------------------- PTX wrappers -------------------------------
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: true when the phase completed; false after limit_ns of
-// %globaltimer or when another role raised the abort flag.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int* err, int code, unsigned long long limit_ns = kWaitLimitNs) {
-  if (mbar_try(bar, parity)) return true;
-  const unsigned long long t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort_flag) return false;
-      if (gtimer() - t0 > limit_ns) {
-        *abort_flag = 1;
-        if (code) atomicCAS(err, 0, code);
-        return false;
-      }
-    }
-  }
-}
 
 // ----------------------- thread-block cluster helpers ------------------------
 // Used by the split-K mode whose K splits of one output tile form a cluster

@@ -128,7 +128,10 @@ typedef struct {
  * (no CTA pairs); B200CONV_SPLITK_CLUSTER=1 sums split-K partials inside the
  * conv kernel (thread-block clusters) instead of the reduce kernel;
  * B200CONV_WINOGRAD_CHUNK_TILES=<tiles> runs the fp32 Winograd path in chunks
- * of that many tiles (pipelined transform / GEMM passes; 0 or unset: off).
+ * of that many tiles (pipelined transform / GEMM passes; 0 or unset: off);
+ * B200CONV_WINOGRAD_FUSED=1 runs the fp32 Winograd F(6x6,3x3) path as one
+ * persistent kernel whenever the shape allows (=0 or unset: three launches);
+ * B200CONV_WINOGRAD_FUSED_GRID=<ctas> runs that kernel on fewer CTAs.
  */
 typedef struct {
     conv_algo_t algo;                     /* CONV_ALGO_AUTO: let the selector choose */
@@ -150,6 +153,9 @@ typedef struct {
                                   (a KH x 1 conv over them), 2 if all KH*KW taps are (a 1 x 1 conv); else 0 */
     int k_split;               /* implicit GEMM: K range split over this many CTAs (fp32 partials), 1 if none */
     int taps;                  /* conv3d: number of depth taps (KD); 1 for conv2d */
+    int winograd_fused;        /* 1 if the fp32 Winograd F(6x6,3x3) runs as one persistent kernel (input
+                                  transform, FFMA GEMM and output transform overlapped inside each CTA,
+                                  per-CTA scratch in the workspace); else 0 */
     size_t workspace_bytes;    /* bytes the caller must pass to *_forward */
 } conv_plan_t;
 

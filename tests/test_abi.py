@@ -64,17 +64,51 @@ def plan2d(shape: synth.Conv2dShape, dtype="f32", **opt):
     return st, p.as_dict()
 
 
-def test_winograd_shape_plan():
-    """40 x 512 x 512, 192 -> 96, fp32: F(6x6,3x3), per-image scratch
-    64 * 86^2 * (192 + 96) * 4 bytes = 545 MB, so an 8 GiB budget gives
+def test_winograd_shape_plan(monkeypatch):
+    """40 x 512 x 512, 192 -> 96, fp32, in three launches: F(6x6,3x3), per-image
+    scratch 64 * 86^2 * (192 + 96) * 4 bytes = 545 MB, so an 8 GiB budget gives
     batch tiles of 15 images (15, 15, 10)."""
+    monkeypatch.setenv("B200CONV_WINOGRAD_FUSED", "0")
     st, p = plan2d(synth.WINOGRAD_F32)
     assert st == 0
     assert p["algo"] == "winograd" and p["winograd_m"] == 6 and p["engine"] == "simt"
+    assert p["winograd_fused"] == 0
     assert p["batch_tile"] == 15 and p["num_batch_tiles"] == 3
     per_img = 64 * 86 * 86 * (192 + 96) * 4
     assert p["workspace_bytes"] >= 15 * per_img
     assert p["workspace_bytes"] < 15 * per_img + 64 * 192 * 96 * 4 + 4096
+
+
+def test_winograd_fused_plan(monkeypatch):
+    """The same shape on the persistent kernel (B200CONV_WINOGRAD_FUSED=1):
+    untiled, one CTA per SM, each holding two V and two M buffers of a 128-tile
+    block: 148 * 2 * 64 * 128 * (192 + 96) * 4 bytes after U (64 * 192 * 96 * 4)."""
+    assert plan2d(synth.WINOGRAD_F32)[1]["winograd_fused"] == 0      # off by default
+    monkeypatch.setenv("B200CONV_WINOGRAD_FUSED", "1")
+    st, p = plan2d(synth.WINOGRAD_F32)
+    assert st == 0
+    assert p["algo"] == "winograd" and p["winograd_m"] == 6 and p["engine"] == "simt"
+    assert p["winograd_fused"] == 1 and p["batch_tile"] == 40 and p["num_batch_tiles"] == 1
+    u = 64 * 192 * 96 * 4
+    scratch = 148 * 2 * 64 * 128 * (192 + 96) * 4
+    assert p["workspace_bytes"] == -(-u // 256) * 256 + -(-scratch // 256) * 256
+
+
+def test_winograd_fused_rules(monkeypatch):
+    """Not for 16-bit inputs, a forced batch tile, or a budget below the per-CTA
+    scratch; the test hook turns it on and off."""
+    big = synth.WINOGRAD_F32
+    small = synth.Conv2dShape(2, 40, 40, 64, 64, 3, 3, (1, 1), (1, 1), (1, 1))
+    monkeypatch.setenv("B200CONV_WINOGRAD_FUSED", "1")
+    assert plan2d(big, "f16")[1]["winograd_fused"] == 0
+    assert plan2d(big, winograd_tile_batch=8)[1]["winograd_fused"] == 0
+    st, p = plan2d(big, winograd_budget_bytes=2 * 2 ** 30)                    # 2.79 GB of scratch does not fit
+    assert st == 0 and p["winograd_fused"] == 0 and p["batch_tile"] == 3
+    st, p = plan2d(small, algo="winograd")
+    assert st == 0 and p["winograd_fused"] == 1
+    assert p["workspace_bytes"] == -(-64 * 64 * 64 * 4 // 256) * 256 + 2 * 64 * 128 * (64 + 64) * 4
+    monkeypatch.setenv("B200CONV_WINOGRAD_FUSED", "0")
+    assert plan2d(big)[1]["winograd_fused"] == 0
 
 
 def test_small_shape_takes_implicit_gemm():

@@ -37,9 +37,26 @@ def plan3d(s, dt, algo="auto"):
 
 
 def test_default_workload_winograd_fp32():
-    """40 x 512 x 512, 192 -> 96: F(6x6,3x3), T = 40 * 86 * 86 tiles, alpha^2 = 64."""
+    """40 x 512 x 512, 192 -> 96: F(6x6,3x3), T = 40 * 86 * 86 tiles, alpha^2 = 64,
+    on the persistent kernel: the GEMM's FLOPs; input, output and the V / M
+    round trips through its scratch."""
     s = synth.WINOGRAD_F32
-    w = bench.kernel_work(bench.Conv(s, "f32", "uniform"), plan2d(s, "f32"))
+    p = plan2d(s, "f32")
+    p["winograd_fused"] = 1
+    w = bench.kernel_work(bench.Conv(s, "f32", "uniform"), p)
+    T = 40 * 86 * 86
+    assert set(w) == {"wino_filter", "wino_fused"}
+    assert w["wino_fused"][0] == 2.0 * 64 * T * 192 * 96
+    assert w["wino_fused"][1] == (40 * 512 * 512 * (192 + 96) + 2 * 64 * T * (192 + 96)) * 4
+    assert bench.kernel_bound("wino_fused") == "alu"
+
+
+def test_default_workload_winograd_fp32_three_launches():
+    """The same shape in three launches (the default plan)."""
+    s = synth.WINOGRAD_F32
+    p = plan2d(s, "f32")
+    assert p["winograd_fused"] == 0
+    w = bench.kernel_work(bench.Conv(s, "f32", "uniform"), p)
     T = 40 * 86 * 86
     assert w["wino_gemm_simt"][0] == 2.0 * 64 * T * 192 * 96
     assert w["wino_gemm_simt"][1] == 64 * T * (192 + 96) * 4            # V read + M write
