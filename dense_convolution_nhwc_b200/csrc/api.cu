@@ -284,8 +284,9 @@ WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m
 
 // The persistent fp32 Winograd kernel (transforms overlapped with the FFMA
 // GEMM inside each CTA) against the three-launch path: it needs F(6x6,3x3)
-// with fp32 input and tile-major V.  It is measured slower than the three
-// launches on the 40 x 512 x 512, 192 -> 96 case (19.5 against 18.4 ms), so
+// with fp32 input and tile-major V.  On the 40 x 512 x 512, 192 -> 96 case it
+// measured 18.2 against 18.4 ms for the three launches (one run each on one
+// B200), a gain inside run-to-run spread for 2.8 GB of per-CTA scratch, so
 // it runs only when B200CONV_WINOGRAD_FUSED=1 (a test hook, read on every
 // call; =0 or unset keeps the three launches).  kFusedMinBlocksPerSm is the
 // rule it would take by default: enough 128-tile blocks that every SM gets at

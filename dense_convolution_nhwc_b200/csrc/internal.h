@@ -19,6 +19,7 @@ enum DevErr : int {
   DEVERR_TIMEOUT_EPILOGUE = 0x104,   // epilogue waited too long for a finished accumulator
   DEVERR_TIMEOUT_FUSED_GEMM = 0x105,   // persistent fp32 Winograd: a GEMM unit waited too long for V or a free M
   DEVERR_TIMEOUT_FUSED_XFORM = 0x106,  // persistent fp32 Winograd: the transform warps waited too long for the GEMM
+  DEVERR_FUSED_SMEM_ALIGN = 0x107,     // persistent fp32 Winograd: input boxes not 128-byte aligned (read without TMA)
   DEVERR_TIMEOUT_SELFTEST = 0x1ff,   // the watchdog self-test's deliberate wait
 };
 

@@ -64,6 +64,25 @@ __device__ __forceinline__ bool mbar_wait_inl(uint32_t bar, uint32_t parity, vol
     }
   }
 }
+// Bounded wait that sleeps between polls (32 ns doubling to 2 us), for roles
+// that may wait a long time beside warps that need the issue slots.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                                int code, unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  unsigned ns = 32;
+  for (;;) {
+    __nanosleep(ns);
+    if (mbar_try(bar, parity)) return true;
+    if (ns < 2048) ns *= 2;
+    if (*abort_flag) return false;
+    if (gtimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      if (code) atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+}
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err, int code,
                                        unsigned long long limit_ns = kWaitLimitNs) {
   return mbar_wait_inl(bar, parity, abort_flag, err, code, limit_ns);

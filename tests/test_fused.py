@@ -135,3 +135,21 @@ def test_fused_headline_shape():
     torch.cuda.synchronize()
     assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
     assert torch.equal(_bits(got), _bits(ref))
+
+
+def test_fused_unaligned_input_reads_without_tma():
+    """An input 4 bytes off a 16-byte boundary cannot be a TMA source: the
+    transform warpgroup then reads it with per-thread loads, same bits."""
+    s = synth.Conv2dShape(2, 64, 64, 64, 96, 3, 3, (1, 1), (1, 1), (1, 1))
+    x0, w = synth.conv2d_inputs(s, "f32", "normal", 35, device="cuda")
+    buf = torch.empty(x0.numel() + 1, dtype=torch.float32, device="cuda")
+    x = buf[1:].view(x0.shape)
+    x.copy_(x0)
+    assert x.data_ptr() % 16 != 0
+    with env(B200CONV_WINOGRAD_FUSED=0):
+        ref = B.conv2d(x0, w, s.stride, s.pad, s.dilation)
+    with env(B200CONV_WINOGRAD_FUSED=1, B200CONV_WINOGRAD_FUSED_GRID=3):
+        got = B.conv2d(x, w, s.stride, s.pad, s.dilation)
+    torch.cuda.synchronize()
+    assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    assert torch.equal(_bits(got), _bits(ref))
