@@ -860,8 +860,20 @@ bool select_wino3d(const conv3d_desc_t* d, const Geom3& g, conv_dtype_t dt, cons
   nu = std::min<long long>(nu, L1.units);
   const bool forced_tile = o.winograd_tile_batch > 0;
   if (forced_tile) nu = std::min<long long>(nu, o.winograd_tile_batch);
-  const long long r_min = (long long)p.sm_count * 128;
-  if (nu <= 0 || (!forced_tile && nu < L1.units && nu * L1.tiles_hw < r_min)) return false;
+  // A batch tile of nu units runs its alpha^3 point GEMMs in one batched launch
+  // of nu * tiles_hw rows each, so the tile needs only a few full 128-row GEMM
+  // tiles per point to fill the GPU (the 2D rule's full wave of rows per point
+  // undercounts the launch by alpha^3).  Measured on 1 x 41 x 120 x 208,
+  // 512 -> 512, fp32 under the 8 GiB cap: 6-unit tiles (9,360 rows) 35.2 ms
+  // against 55.5 ms for its depth taps.
+  const long long rows_min = 4 * 128;
+  if (nu <= 0 || (!forced_tile && nu < L1.units && nu * L1.tiles_hw < rows_min)) return false;
+  // the same number of tiles, evened out (5 + 5 units measured 34.7 ms against
+  // 35.2 for 6 + 4 on that case)
+  if (!forced_tile && nu < L1.units) {
+    const long long nt = (L1.units + nu - 1) / nu;
+    nu = (L1.units + nt - 1) / nt;
+  }
   s->algo = CONV_ALGO_WINOGRAD;
   s->engine = tc_gemm ? CONV_ENGINE_TCGEN05 : CONV_ENGINE_SIMT;
   s->wino_m = m;

@@ -423,7 +423,15 @@ wino_fused_f32_kernel(const __grid_constant__ CUtensorMap tmIn, const FusedArgs 
             issue_more();
             cur = nx;
           }
-          if (abort_flag) break;
+          if (abort_flag) {
+            // leave no box in flight into this CTA's shared memory (bounded waits)
+            if (xt == 0) {
+              volatile int never = 0;
+              for (uint32_t k = kin; k < kissue; ++k)
+                mbar_wait_sleep(infull((int)(k % NIBUF)), (k / NIBUF) & 1u, &never, p.err, 0, 100000000ull);
+            }
+            break;
+          }
         } else {
           const int cgroups = (C + ibx - 1) / ibx;
           const long long nb = ((ai.t_count + iby - 1) / iby) * cgroups;

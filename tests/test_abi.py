@@ -338,8 +338,9 @@ def test_conv3d_winograd_plan():
 
 def test_conv3d_winograd_budget_tiles_units():
     """The budget bounds V + M per unit (one image's depth tile of m frames); a
-    forced tile is capped by it; tiles under one wave of 128-row GEMM tiles, or
-    a budget under one unit, fall back to the depth taps."""
+    forced tile is capped by it; tiles of fewer than four 128-row GEMM tiles per
+    point (all alpha^3 points run in one batched launch), or a budget under one
+    unit, fall back to the depth taps."""
     s = synth.Conv3dShape(1, 42, 64, 64, 64, 256, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))   # OD = 40: 10 units
     per_unit = 216 * (16 * 16) * (64 * 4 + 256 * 4)
     st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit + 5, winograd_tile_batch=10)
@@ -347,16 +348,19 @@ def test_conv3d_winograd_budget_tiles_units():
     assert p["workspace_bytes"] == wino3d_ws(s, 4, 4, True, 3)
     st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit, winograd_tile_batch=2)
     assert st == 0 and p["batch_tile"] == 2 and p["num_batch_tiles"] == 5
-    st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit)      # 768 rows per tile < one wave
-    assert st == 0 and p["taps"] == 3
+    st, p = plan3d(s, "f32", winograd_budget_bytes=3 * per_unit)      # 3 * 256 = 768 rows per point >= 512
+    # 10 units in tiles of at most 3: four tiles, evened out to 3, 3, 3, 1
+    assert st == 0 and p["algo"] == "winograd" and p["taps"] == 1 and p["batch_tile"] == 3
+    st, p = plan3d(s, "f32", winograd_budget_bytes=6 * per_unit)      # two tiles: 5 + 5, not 6 + 4
+    assert st == 0 and p["batch_tile"] == 5 and p["num_batch_tiles"] == 2
+    st, p = plan3d(s, "f32", winograd_budget_bytes=per_unit)          # 256 rows per point < 512
+    assert st == 0 and p["taps"] == 3 and p["winograd_m"] != 4        # depth taps (each a 2D Winograd)
     st, p = plan3d(s, "f32", winograd_budget_bytes=per_unit - 1, winograd_tile_batch=1)
     assert st == 0 and p["taps"] == 3
     big = synth.Conv3dShape(1, 42, 256, 256, 64, 256, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
     per_unit = 216 * (64 * 64) * (64 * 4 + 256 * 4)
-    st, p = plan3d(big, "f32", winograd_budget_bytes=5 * per_unit)    # 5 * 4096 rows >= 148 * 128
-    assert st == 0 and p["algo"] == "winograd" and p["batch_tile"] == 5 and p["num_batch_tiles"] == 2
-    st, p = plan3d(big, "f32", winograd_budget_bytes=4 * per_unit)    # 4 * 4096 rows < 148 * 128
-    assert st == 0 and p["taps"] == 3 and p["winograd_m"] != 4        # depth taps (each a 2D Winograd)
+    st, p = plan3d(big, "f32", winograd_budget_bytes=4 * per_unit)    # 4 * 4096 rows per point; tiles of 4, 4, 2 units
+    assert st == 0 and p["algo"] == "winograd" and p["batch_tile"] == 4 and p["num_batch_tiles"] == 3
 
 
 def test_split_k_for_small_m_long_k():

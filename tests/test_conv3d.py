@@ -255,6 +255,6 @@ def test_winograd3d_unit_tiling_is_bit_identical(dtype):
 
 @pytest.mark.parametrize("s", synth.CONV3D_TAPS, ids=lambda s: s.name())
 def test_workload_shapes_f32_sampled(s):
-    """The conv3d workload in fp32: the 3D Winograd where its budget allows a
-    wave of GEMM rows, depth taps (each a 2D Winograd) otherwise."""
+    """The conv3d workload in fp32: the native 3D Winograd on all three shapes
+    (the largest in batch tiles of depth units under the 8 GiB workspace cap)."""
     check3d(s, "f32", sample=4096)
