@@ -118,8 +118,8 @@ def test_small_shape_takes_implicit_gemm():
 
 
 @pytest.mark.parametrize("budget,expect", [
-    (2 * 2 ** 30, ("winograd", 3)),        # 3 images/tile = 22188 GEMM rows >= 148 * 128
-    (2 ** 30, ("implicit", None)),         # 1 image/tile = 7396 rows: too few, falls back
+    (2 * 2 ** 30, ("winograd", 3)),        # 3 images/tile
+    (2 ** 30, ("winograd", 1)),            # 1 image/tile = 7396 GEMM rows per point: still Winograd (fp32)
     (2 ** 20, ("implicit", None)),         # not even one image fits
 ])
 def test_budget_injection(budget, expect):
