@@ -464,6 +464,10 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->ksplit = (int)ks;
       s->split_off = s->ws;
       s->ws += align256((size_t)ks * M * g.o * 4);
+      // arrival counters of the serial in-kernel reduction: one per (128-row tile,
+      // column tile, epilogue warp)
+      if (s->engine == CONV_ENGINE_TCGEN05)
+        s->ws += align256((size_t)((M + 127) / 128) * ((g.o + s->tile_n - 1) / s->tile_n) * 4 * sizeof(int));
     }
     if (s->engine == CONV_ENGINE_TCGEN05 && s->ksplit == 1 && !s->wpack && !s->fpack &&
         tc_pair_tiles(M, 1, g.o, s->tile_n, taps * ((c_eff + 63) / 64), p))
@@ -704,9 +708,20 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
     // barrier plus distributed-shared-memory sums.
     const char* sc = std::getenv("B200CONV_SPLITK_CLUSTER");
     const bool cluster_ok = sc && std::strcmp(sc, "1") == 0;
+    // The serial in-kernel reduction (B200CONV_SPLITK_SERIAL=1, a test hook read
+    // on every call): the last-arriving split of each tile sums the partials;
+    // its counters are cleared before the launch.
+    const char* ss = std::getenv("B200CONV_SPLITK_SERIAL");
+    int* counters = nullptr;
+    if (s.ksplit > 1 && ss && std::strcmp(ss, "1") == 0) {
+      const long long Mr = (long long)g.n * g.oh * g.ow;
+      const size_t n_cnt = (size_t)((Mr + 127) / 128) * ((g.o + s.tile_n - 1) / s.tile_n) * 4;
+      counters = reinterpret_cast<int*>(base + s.split_off + align256((size_t)s.ksplit * Mr * g.o * 4));
+      if (cudaMemsetAsync(counters, 0, n_cnt * sizeof(int), st) != cudaSuccess) return CONV_ERR_CUDA;
+    }
     ProfScope ps(K_TC_CONV, st);
     if (launch_tc_conv(cin, cw, out, gg, dt, s.tile_n, d.props.sm_count, d.err_word, accumulate, st, s.ksplit,
-                       partial, cluster_ok ? &reduced : nullptr, s.tile_m) != cudaSuccess)
+                       partial, (cluster_ok || counters) ? &reduced : nullptr, s.tile_m, counters) != cudaSuccess)
       return CONV_ERR_CUDA;
     done = true;
   }

@@ -75,14 +75,17 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, size_t count,
 bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const void* w);
 // accumulate: out = round(out + round(result)), the unfused depth-tap add's arithmetic.
 // ksplit > 1: the K range is split over ksplit CTAs per tile.  With `reduced`
-// given, the splits of a tile run as one thread-block cluster that sums the
-// partials in split order inside the kernel and sets *reduced; otherwise (or
-// when the device cannot hold the cluster) fp32 partials [ksplit][M][O] go to
-// `partial` and the caller runs launch_splitk_reduce (same sums, same order).
+// and `tile_cnt` given (M/128 x O/tile_n x 4 zeroed counters), each split writes
+// fp32 partials [ksplit][M][O] to `partial` and the last split of each (tile,
+// epilogue warp) sums them in split order and writes the output (*reduced set).
+// With `reduced` alone, the splits of a tile run as one thread-block cluster
+// that sums the partials from shared memory (*reduced set unless the device
+// cannot hold the cluster).  Otherwise the caller runs launch_splitk_reduce on
+// `partial` (the same sums in the same order on every route).
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g,
                            conv_dtype_t dt, int tile_n, int sm_count, int* err_word,
                            bool accumulate, cudaStream_t s, int ksplit = 1, float* partial = nullptr,
-                           bool* reduced = nullptr, int tile_m = 128);
+                           bool* reduced = nullptr, int tile_m = 128, int* tile_cnt = nullptr);
 // Native 3D implicit GEMM on tcgen05: K = KD*KH*KW*C in one main loop, the A
 // tiles gathered by a 5D TMA im2col map (corners limited to [-16, 15]).
 bool tc_conv3d_supported(const Geom3& g, conv_dtype_t dt, const void* in, const void* w);

@@ -83,6 +83,11 @@ struct TcArgs {
   int tma_store;               // write 32-row x 128-byte chunks with TMA stores through tmD
   int cluster_reduce;          // split-K whose ksplit CTAs of a tile form a cluster: rank 0 sums the
                                // others' fp32 partials from their shared memory and writes out
+  int serial_reduce;           // split-K whose last-arriving split of a tile sums the fp32 partials
+  float* partial;              // serial_reduce: [ksplit][m_rows][ocols] fp32 partials
+  long long part_batch;        // serial_reduce: elements between splits' partials
+  int* tile_cnt;               // serial_reduce: m_tiles * n_tiles * 4 arrival counters (one per tile and
+                               // epilogue warp), zero on entry
   int* err;
 };
 
@@ -119,6 +124,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
   static_assert(BM * BN * 4 <= C::STAGES * C::STAGE_BYTES, "split partial fits the stage ring");
   const bool cl = CG == 1 && MODE == 1 && a.cluster_reduce;
+  const bool sr = CG == 1 && MODE == 1 && a.serial_reduce && !a.cluster_reduce;
   const uint32_t crank = cl ? cluster_rank() : 0u;
   // CTA pair: rank 0 issues the MMAs; both load and drain their own halves.
   const uint32_t prank = CG == 2 ? cluster_rank() : 0u;
@@ -400,6 +406,30 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
           continue;
         }
+        if (sr) {
+          // serial split-K: this split's fp32 partial rows (the output comes later)
+          if (row_ok) {
+            float* prow = a.partial + (long long)b * a.part_batch + m * a.ocols;
+            const bool vec4 = (a.ocols & 3) == 0;
+#pragma unroll
+            for (int h = 0; h < EPI / 32; ++h) {
+              const int c0 = n0 + cg + 32 * h;
+              if (c0 >= a.ocols) continue;
+              if (vec4 && c0 + 32 <= a.ocols) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                  reinterpret_cast<float4*>(prow + c0)[v] =
+                      make_float4(__uint_as_float(rr[h][4 * v]), __uint_as_float(rr[h][4 * v + 1]),
+                                  __uint_as_float(rr[h][4 * v + 2]), __uint_as_float(rr[h][4 * v + 3]));
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (c0 + j < a.ocols) prow[c0 + j] = __uint_as_float(rr[h][j]);
+              }
+            }
+          }
+          continue;
+        }
         if constexpr (sizeof(TOut) == 4) {
           if (a.tma_store) {
             // stage row `lane` of this warp's 32 x 32 chunk (16-byte chunks XOR-swizzled by
@@ -536,6 +566,90 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));   // the pair's accumulator lives on in rank 0's count
       else
         mbar_arrive(tempty_bar(acc));
+      if (sr) {
+        // Serial split-K, per epilogue warp (its 32 rows): publish this split's
+        // partial rows, count the arrivals at (tile, warp); the split that arrives
+        // last sums all partials in split order (the order of the reduce kernel)
+        // and writes those output rows.  No warp or split waits for another.
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          int* cnt = a.tile_cnt + (((long long)mt * a.n_tiles + nt) * 4 + q);
+          last = atomicAdd(cnt, 1) == a.ksplit - 1;
+          if (last) *cnt = 0;              // ready for the next call on this workspace
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          // warp q sums its 32 rows, 8 at a time, lane = 4 columns: the 8 rows'
+          // loads of one split are in flight together
+          TOut* obase = static_cast<TOut*>(a.out);
+          const bool vec4 = (a.ocols & 3) == 0;
+          for (int c4 = lane; c4 < BN / 4; c4 += 32) {
+            const int col = n0 + 4 * c4;
+            if (col >= a.ocols) continue;
+            const int nv = a.ocols - col < 4 ? a.ocols - col : 4;
+            for (int i0 = 0; i0 < 32; i0 += 8) {
+              float4 acc[8];
+              bool rok[8];
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                const long long mr = trow0 + q * 32 + i0 + r;
+                rok[r] = mr < a.m_rows;
+                acc[r] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (rok[r] && vec4) acc[r] = __ldcg(reinterpret_cast<const float4*>(a.partial + mr * a.ocols + col));
+              }
+              if (vec4) {
+#pragma unroll 2
+                for (int sp = 1; sp < a.ksplit; ++sp) {
+                  float4 t[8];
+#pragma unroll
+                  for (int r = 0; r < 8; ++r) {
+                    const long long mr = trow0 + q * 32 + i0 + r;
+                    t[r] = rok[r] ? __ldcg(reinterpret_cast<const float4*>(a.partial + sp * a.part_batch +
+                                                                            mr * a.ocols + col))
+                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                  }
+#pragma unroll
+                  for (int r = 0; r < 8; ++r) {
+                    acc[r].x += t[r].x; acc[r].y += t[r].y; acc[r].z += t[r].z; acc[r].w += t[r].w;
+                  }
+                }
+              } else {
+                // O not a multiple of 4: element by element, in split order from 0
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                  if (!rok[r]) continue;
+                  const long long mr = trow0 + q * 32 + i0 + r;
+                  float e4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                  for (int e = 0; e < nv; ++e) {
+                    float sum = 0.0f;
+                    for (int sp = 0; sp < a.ksplit; ++sp) sum += __ldcg(a.partial + sp * a.part_batch + mr * a.ocols + col + e);
+                    e4[e] = sum;
+                  }
+                  acc[r] = make_float4(e4[0], e4[1], e4[2], e4[3]);
+                }
+              }
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                if (!rok[r]) continue;
+                const long long mr = trow0 + q * 32 + i0 + r;
+                TOut* po = obase + mr * a.ldo + col;
+                const float v[4] = {acc[r].x, acc[r].y, acc[r].z, acc[r].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  if (e < nv) {
+                    float rv = v[e];
+                    if (a.accumulate) rv = Store<TOut>::to_f32(po[e]) + Store<TOut>::to_f32(Store<TOut>::from_f32(v[e]));
+                    po[e] = Store<TOut>::from_f32(rv);
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
     }
     if (a.tma_store && lane == 0) bulk_wait_all();   // the last stores have landed
     __syncwarp();
@@ -824,7 +938,7 @@ bool tc_conv_supported(const Geom& g, conv_dtype_t dt, const void* in, const voi
 
 cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom& g, conv_dtype_t dt,
                            int tile_n, int sm_count, int* err_word, bool accumulate, cudaStream_t s, int ksplit,
-                           float* partial, bool* reduced, int tile_m) {
+                           float* partial, bool* reduced, int tile_m, int* tile_cnt) {
   if (reduced) *reduced = false;
   if (!tc_conv_supported(g, dt, in, w)) return cudaErrorNotSupported;
   const long long M = (long long)g.n * g.oh * g.ow;
@@ -864,7 +978,28 @@ cudaError_t launch_tc_conv(const void* in, const void* w, void* out, const Geom&
   a.accumulate = accumulate ? 1 : 0;
   a.ksplit = 1;
   a.err = err_word;
-  if (ksplit > 1 && reduced && ksplit <= 16 && ksplit <= taps * a.kb_per_tap) {
+  if (ksplit > 1 && reduced && tile_cnt && partial && ksplit <= taps * a.kb_per_tap) {
+    // split-K inside the kernel, serially: the last split of each (tile, epilogue
+    // warp) sums the fp32 partials in split order and writes the output
+    TcArgs c = a;
+    c.ksplit = ksplit;
+    c.batches = ksplit;
+    c.serial_reduce = 1;
+    c.partial = partial;
+    c.part_batch = M * g.o;
+    c.tile_cnt = tile_cnt;
+    c.tma_store = 0;
+    cudaError_t e;
+    if (dt == CONV_BF16)
+      e = tile_n == 256 ? launch_kernel<256, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, c, sm_count, s)
+                        : launch_kernel<128, 1, __nv_bfloat16, __nv_bfloat16>(tA, tB, c, sm_count, s);
+    else
+      e = tile_n == 256 ? launch_kernel<256, 1, __half, __half>(tA, tB, c, sm_count, s)
+                        : launch_kernel<128, 1, __half, __half>(tA, tB, c, sm_count, s);
+    if (e == cudaSuccess) *reduced = true;
+    return e;
+  }
+  if (ksplit > 1 && reduced && !tile_cnt && ksplit <= 16 && ksplit <= taps * a.kb_per_tap) {
     // split-K inside the kernel: the ksplit CTAs of a tile form a cluster and
     // rank 0 adds the others' partials (in split order) from their shared memory
     TcArgs c = a;

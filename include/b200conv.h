@@ -127,6 +127,7 @@ typedef struct {
  * result: B200CONV_TC_PAIR=0 keeps the tensor-core kernels on 128-row tiles
  * (no CTA pairs); B200CONV_SPLITK_CLUSTER=1 sums split-K partials inside the
  * conv kernel (thread-block clusters) instead of the reduce kernel;
+ * B200CONV_SPLITK_SERIAL=1 has the last-arriving split of each tile sum them;
  * B200CONV_WINOGRAD_CHUNK_TILES=<tiles> runs the fp32 Winograd path in chunks
  * of that many tiles (pipelined transform / GEMM passes; 0 or unset: off);
  * B200CONV_WINOGRAD_FUSED=1 runs the fp32 Winograd F(6x6,3x3) path as one

@@ -9,7 +9,10 @@ layers).  Two routes give the same bits:
   call): the splits of a tile run as one thread-block cluster, each leaving its
   partial in its own shared memory, and every CTA of the cluster sums a slice
   of the tile's rows over the splits in split order and writes those rows,
-  with no reduce launch (taken when a launch's clusters all fit at once).
+  with no reduce launch (taken when a launch's clusters all fit at once);
+* the serial route (B200CONV_SPLITK_SERIAL=1): every split writes its partial
+  and counts its arrival per (tile, epilogue warp); the split that arrives last
+  sums the partials in split order and writes the output, no reduce launch.
 
 Checked: both routes agree bit for bit, match the oracle, repeat bit for bit,
 the cluster route launches no reduce kernel when its clusters fit in one wave,
@@ -107,3 +110,40 @@ def test_cluster_split_k_accumulates_depth_taps(dtype):
     assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
     want = oracle.conv3d(x.cpu(), w.cpu(), dtype, s.stride, s.pad, s.dilation)
     assert_close(as_f64(got), want, dtype, s.name())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("case", SHAPES, ids=lambda c: c[0].name())
+def test_serial_split_k_matches_reduce_route_and_oracle(case, dtype):
+    """The last-arriving split reduces: no reduce launch, the same bits as the
+    reduce kernel, repeatable (the counters reset themselves), and the oracle."""
+    shape, _ = case
+    p = _plan(shape, dtype)
+    assert p["engine"] == "tcgen05" and p["k_split"] > 1, p
+    x, w = synth.conv2d_inputs(shape, dtype, "he", 33, device="cuda")
+    with env(B200CONV_SPLITK_SERIAL=1):
+        B.conv_profile_begin()
+        got = run_conv2d(x, w, shape)
+        again = run_conv2d(x, w, shape)
+        prof = B.profile_end()
+    assert "splitk_reduce" not in prof, prof
+    ref = run_conv2d(x, w, shape)
+    assert torch.equal(got.view(torch.int16), again.view(torch.int16))
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    want = oracle.conv2d(x.cpu(), w.cpu(), dtype, shape.stride, shape.pad, shape.dilation)
+    assert_close(as_f64(got), want, dtype, shape.name())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_serial_split_k_accumulates_depth_taps(dtype):
+    """conv3d depth taps whose 2D convs are split-K on the serial route: the
+    last split adds into out; equal to the reduce route bit for bit."""
+    s = synth.Conv3dShape(1, 5, 7, 7, 512, 512, 3, 3, 3, (1, 1, 1), (0, 1, 1), (1, 1, 1))
+    x, w = synth.conv3d_inputs(s, dtype, "normal", 34, device="cuda")
+    with env(B200CONV_SPLITK_SERIAL=1):
+        got = B.conv3d(x, w, s.stride, s.pad, s.dilation)
+        torch.cuda.synchronize()
+    ref = B.conv3d(x, w, s.stride, s.pad, s.dilation)
+    torch.cuda.synchronize()
+    assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
