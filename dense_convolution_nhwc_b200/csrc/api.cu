@@ -187,6 +187,7 @@ struct Sel {
   conv_dtype_t wino_store = CONV_F32;
   long long chunk = 0;     // Winograd: tiles per transform -> GEMM -> transform pass (0: the whole batch tile)
   bool fused = false;      // fp32 Winograd as one persistent kernel (transforms overlapped with the GEMM)
+  bool split_bf16 = false; // fp32 Winograd whose GEMM runs on tcgen05 over split-bf16 operands
   int fused_grid = 0;      // its CTAs (one per SM)
   size_t ws = 0;
 };
@@ -263,10 +264,21 @@ struct WinoLayout {
 
 // chunk > 0: the batch tile's tiles pass through V and M in chunks of at most
 // `chunk` tiles, so V and M hold one chunk.
-WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb, long long chunk = 0) {
+// split: the split-bf16 fp32 GEMM's operands, U [a2][O][6C] and V [a2][T][3C]
+// in bf16, M [a2][T][O] fp32.
+WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb, long long chunk = 0,
+                           bool split = false) {
   WinoLayout L;
   const long long a2 = (long long)(m + 2) * (m + 2);
   L.tiles_per_img = (long long)((g.oh + m - 1) / m) * ((g.ow + m - 1) / m);
+  if (split) {
+    const long long t = nb * L.tiles_per_img;
+    L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * 6 + (size_t)g.o * 4);
+    L.u_bytes = align256((size_t)(a2 * g.o * g.c) * 12);
+    L.v_bytes = align256((size_t)(a2 * t * g.c) * 6);
+    L.m_bytes = align256((size_t)(a2 * t * g.o) * 4);
+    return L;
+  }
   const int esz = dtype_size(store);
   L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * esz + (size_t)g.o * (cmajor ? 4 : esz));
   const long long t = chunk > 0 ? std::min(nb * L.tiles_per_img, chunk) : nb * L.tiles_per_img;
@@ -312,6 +324,20 @@ long long winograd_chunk_tiles(const Geom& g, int m, const conv_device_props_t& 
   return 0;
 }
 
+// The fp32 Winograd GEMM on the tensor cores over split-bf16 operands: each fp32
+// value is the exact sum of three bf16 parts, and the six products a_i b_j with
+// i + j <= 2 are accumulated in fp32 (TMEM) in one K = 6C reduction, which
+// keeps fp32 accuracy (the dropped products are below 2^-24 of the result).
+// It needs F(6x6,3x3), a tcgen05 device, C a multiple of 64 and O of 4.
+// B200CONV_WINOGRAD_SPLIT_BF16=1 turns it on (a test hook read on every call).
+bool winograd_split_wanted(const Geom& g, conv_dtype_t dt, int m, const conv_device_props_t& p) {
+  if (dt != CONV_F32 || m != 6 || p.cc_major != 10 || g.c % 64 != 0 || g.o % 4 != 0) return false;
+  if (const char* f = std::getenv("B200CONV_WINOGRAD_FUSED"))
+    if (std::strcmp(f, "1") == 0) return false;
+  const char* e = std::getenv("B200CONV_WINOGRAD_SPLIT_BF16");
+  return e && std::strcmp(e, "1") == 0;
+}
+
 conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t& p,
                        const conv_options_t& o, Sel* s) {
   const int esz = dtype_size(dt);
@@ -330,9 +356,10 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     const int m = winograd_m_for(dt);
     // 16-bit operands go to the tensor cores when their rows meet the
     // 16-byte rule, else the transforms store fp32 for the FFMA engine.
-    const bool tc_gemm = dt != CONV_F32 && p.cc_major == 10 && g.c % 8 == 0;
-    const conv_dtype_t store = (dt == CONV_F32 || !tc_gemm) ? CONV_F32 : dt;
-    const WinoLayout L1 = winograd_layout(g, store, !tc_gemm, m, 1);
+    const bool split = winograd_split_wanted(g, dt, m, p);
+    const bool tc_gemm = split || (dt != CONV_F32 && p.cc_major == 10 && g.c % 8 == 0);
+    const conv_dtype_t store = split ? CONV_BF16 : ((dt == CONV_F32 || !tc_gemm) ? CONV_F32 : dt);
+    const WinoLayout L1 = winograd_layout(g, store, !tc_gemm, m, 1, 0, split);
     const size_t u_bytes = L1.u_bytes, per_img = L1.per_img;
     const long long tiles_per_img = L1.tiles_per_img;
     long long budget;
@@ -378,7 +405,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
     // 40 x 512 x 512, 192 -> 96, 1-image tiles took 19.5 ms against 18.6
     // untiled and 76.9 ms for the implicit GEMM.  The tensor-core path keeps a
     // full wave of rows per point before it prefers Winograd over its implicit GEMM.
-    const long long r_min = tc_gemm ? (long long)p.sm_count * 128 : 4 * 128;
+    const long long r_min = (tc_gemm && !split) ? (long long)p.sm_count * 128 : 4 * 128;
     bool fallback = nb <= 0 || (!forced_tile && nb < g.n && nb * tiles_per_img < r_min);
     if (fallback && o.algo == CONV_ALGO_WINOGRAD) return CONV_ERR_UNSUPPORTED;
     if (!fallback) {
@@ -389,10 +416,11 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
       s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
-      s->tile_m = tc_gemm && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o, s->tile_n,
-                                           (g.c + 63) / 64, p) ? 256 : 128;
+      s->tile_m = tc_gemm && !split && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o,
+                                                     s->tile_n, (g.c + 63) / 64, p) ? 256 : 128;
       s->chunk = (!tc_gemm && kF32VTileMajor && g.c % 4 == 0) ? winograd_chunk_tiles(g, m, p) : 0;
-      const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb, s->chunk);
+      s->split_bf16 = split;
+      const WinoLayout L = winograd_layout(g, store, !tc_gemm, m, nb, s->chunk, split);
       s->ws = L.u_bytes + L.v_bytes + L.m_bytes;
       s->cpad = 0;
       return CONV_OK;
@@ -536,17 +564,18 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
   if (s.algo == CONV_ALGO_WINOGRAD) {
     const int m = s.wino_m, a2 = (m + 2) * (m + 2);
     const bool cmajor = s.engine == CONV_ENGINE_SIMT;
-    const WinoLayout L = winograd_layout(g, s.wino_store, cmajor, m, s.nb, s.chunk);
+    const WinoLayout L = winograd_layout(g, s.wino_store, cmajor, m, s.nb, s.chunk, s.split_bf16);
     uint8_t* base = static_cast<uint8_t*>(ws);
     void* u = base;
     void* v = base + L.u_bytes;
     void* mb = base + L.u_bytes + L.v_bytes;
-    const conv_dtype_t m_dt = cmajor ? CONV_F32 : s.wino_store;
+    const conv_dtype_t m_dt = (cmajor || s.split_bf16) ? CONV_F32 : s.wino_store;
     cudaError_t e;
     {
       ProfScope ps(K_WINO_FILTER, st);
-      e = cmajor ? launch_wino_filter_cmajor(w, g.w_row_stride, g.o, g.c, m, dt, round4(g.o), static_cast<float*>(u), st)
-                 : launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
+      e = s.split_bf16 ? launch_wino_filter_split(static_cast<const float*>(w), g.w_row_stride, g.o, g.c, u, st)
+          : cmajor ? launch_wino_filter_cmajor(w, g.w_row_stride, g.o, g.c, m, dt, round4(g.o), static_cast<float*>(u), st)
+                   : launch_wino_filter(w, g.w_row_stride, g.o, g.c, m, dt, s.wino_store, u, st);
     }
     if (e != cudaSuccess) return CONV_ERR_CUDA;
     if (s.fused) {
@@ -598,7 +627,9 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
         const long long tb = 0, t = t_all;
         {
           ProfScope ps(K_WINO_INPUT, st);
-          if (cmajor && !tmajor)
+          if (s.split_bf16)
+            e = launch_wino_input_split(static_cast<const float*>(in), g, n0, t, v, t, st);
+          else if (cmajor && !tmajor)
             e = launch_wino_input_cmajor(in, g, n0, nbi, m, dt, static_cast<float*>(v), round4(t), st);
           else
             e = launch_wino_input(in, g, n0, tb, t, m, dt, s.wino_store, v, t, st);
@@ -610,6 +641,7 @@ conv_status_t run2d(const void* in, const void* w, void* out, const Geom& g, con
                                    a2, (int)t, g.c, g.o, tmajor ? g.c : round4(t), round4(g.o), tmajor, st);
         } else {
           BatchedGemm bg{a2, (int)t, g.c, g.o, v, u, mb, m_dt};
+          bg.split_bf16 = s.split_bf16;
           ProfScope ps(K_WINO_GEMM_TC, st);
           e = launch_tc_batched_gemm(bg, s.wino_store, s.tile_n, d.props.sm_count, d.err_word, st, s.tile_m);
         }

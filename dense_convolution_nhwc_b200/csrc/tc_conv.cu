@@ -83,6 +83,9 @@ struct TcArgs {
   int tma_store;               // write 32-row x 128-byte chunks with TMA stores through tmD
   int cluster_reduce;          // split-K whose ksplit CTAs of a tile form a cluster: rank 0 sums the
                                // others' fp32 partials from their shared memory and writes out
+  int split_cb;                // batched GEMM on split-bf16 operands: A's K holds three parts of C
+                               // (split_cb 64-wide blocks each), B's K six (b0 b1 b0 b2 b1 b0); K-block
+                               // kb reads A's part (0,0,1,0,1,2)[kb / split_cb]; 0: plain K
   int serial_reduce;           // split-K whose last-arriving split of a tile sums the fp32 partials
   float* partial;              // serial_reduce: [ksplit][m_rows][ocols] fp32 partials
   long long part_batch;        // serial_reduce: elements between splits' partials
@@ -181,6 +184,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const long long total_tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
   const int ksteps = a.taps * a.kb_per_tap;
 
+  // A's K coordinate of K-block kb (MODE 0): the split-bf16 GEMM reads part
+  // (0,0,1,0,1,2)[kb / split_cb] of A for the six B segments
+  auto a_kcoord = [&](int kb) {
+    if (MODE != 0 || a.split_cb == 0) return kb * BK;
+    const int term = kb / a.split_cb, sub = kb - term * a.split_cb;
+    const int part = (0x210100 >> (4 * term)) & 0xF;
+    return (part * a.split_cb + sub) * BK;
+  };
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
@@ -245,7 +256,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                       (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
               tma_load_3d_pair(dB, &tmB, fb0, kb * BK, tap, ncol);
             } else {
-              tma_load_3d_pair(dA, &tmA, fb0, kb * BK, (int)row0, b);
+              tma_load_3d_pair(dA, &tmA, fb0, a_kcoord(kb), (int)row0, b);
               tma_load_3d_pair(dB, &tmB, fb0, kb * BK, ncol, b);
             }
             ++issued;
@@ -270,7 +281,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
             tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
           } else {
-            tma_load_3d(dA, &tmA, fb, kb * BK, (int)row0, b);
+            tma_load_3d(dA, &tmA, fb, a_kcoord(kb), (int)row0, b);
             tma_load_3d(dB, &tmB, fb, kb * BK, nt * BN, b);
           }
           ++issued;
@@ -1138,19 +1149,21 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   if (dt == CONV_F32 || !driver_fns()) return cudaErrorNotSupported;
   if (bg.c % 8 != 0 || (reinterpret_cast<uintptr_t>(bg.a) & 15) || (reinterpret_cast<uintptr_t>(bg.b) & 15))
     return cudaErrorNotSupported;
+  if (bg.split_bf16 && (dt != CONV_BF16 || bg.c % BK != 0 || bg.d_dt != CONV_F32)) return cudaErrorNotSupported;
   if (bg.t == 0 || bg.batches == 0) return cudaSuccess;
+  // K extents of A and B (the split-bf16 GEMM: 3C parts of A against 6C of B)
+  const long long ka = bg.split_bf16 ? 3LL * bg.c : bg.c, kb_ = bg.split_bf16 ? 6LL * bg.c : bg.c;
   CUtensorMap tA, tB;
-  if (!encode_3d(&tA, dt, bg.a, bg.c, bg.t, bg.batches, (uint64_t)bg.c * 2, (uint64_t)bg.t * bg.c * 2, BK,
-                 BM, 1))
+  if (!encode_3d(&tA, dt, bg.a, ka, bg.t, bg.batches, (uint64_t)ka * 2, (uint64_t)bg.t * ka * 2, BK, BM, 1))
     return cudaErrorInvalidValue;
-  if (!encode_3d(&tB, dt, bg.b, bg.c, bg.o, bg.batches, (uint64_t)bg.c * 2, (uint64_t)bg.o * bg.c * 2, BK,
-                 tile_n, 1))
+  if (!encode_3d(&tB, dt, bg.b, kb_, bg.o, bg.batches, (uint64_t)kb_ * 2, (uint64_t)bg.o * kb_ * 2, BK, tile_n, 1))
     return cudaErrorInvalidValue;
   TcArgs a{};
   a.m_tiles = (bg.t + BM - 1) / BM;
   a.n_tiles = (bg.o + tile_n - 1) / tile_n;
   a.batches = bg.batches;
-  a.kb_per_tap = (bg.c + BK - 1) / BK;
+  a.kb_per_tap = (int)((kb_ + BK - 1) / BK);
+  a.split_cb = bg.split_bf16 ? bg.c / BK : 0;
   a.taps = 1;
   a.kw = 1; a.dh = 1; a.dw = 1;
   a.oh = 1; a.ow = bg.t; a.sh = 1; a.sw = 1; a.ph = 0; a.pw = 0;

@@ -34,7 +34,19 @@ struct WinoInArgs {
 // bounds tests.
 // The body of one input-transform block: block `bid` of a 1D grid, thread
 // (tx, ty) of a bx x by block.
-template <int M, typename Tin, typename Tst, typename Idx>
+// An fp32 value as three bf16 parts whose sum is the value (each part the
+// round-to-nearest bf16 of what the parts before it leave; the residuals are
+// exact in fp32): the operand split of the split-bf16 fp32 GEMM.
+__device__ __forceinline__ void split_bf16x3(float x, __nv_bfloat16& p0, __nv_bfloat16& p1, __nv_bfloat16& p2) {
+  p0 = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(p0);
+  p1 = __float2bfloat16_rn(r1);
+  p2 = __float2bfloat16_rn(r1 - __bfloat162float(p1));
+}
+
+// SPLIT = 1: Tst is bf16 and every V row holds the three bf16 parts of the fp32
+// values side by side ([t][3C]: part 0 at c, part 1 at C + c, part 2 at 2C + c).
+template <int M, typename Tin, typename Tst, typename Idx, int SPLIT = 0>
 __device__ __forceinline__ void wino_input_block(const Tin* __restrict__ in, const WinoInArgs& a,
                                                  Tst* __restrict__ v, long long bid, int lx, int ly, int bx,
                                                  int by) {
@@ -89,14 +101,26 @@ __device__ __forceinline__ void wino_input_block(const Tin* __restrict__ in, con
 #pragma unroll
     for (int i = 0; i < A; ++i) tt[i][j] = res[i];
   }
-  const Idx plane = (Idx)(a.t_stride * a.c);
-  Tst* vp = v + t * a.c + c;
+  const Idx rowc = SPLIT ? (Idx)3 * a.c : (Idx)a.c;
+  const Idx plane = (Idx)(a.t_stride * rowc);
+  Tst* vp = v + t * rowc + c;
 #pragma unroll
   for (int i = 0; i < A; ++i) {
     float res[A];
     Wino<M>::bt(tt[i], res);
 #pragma unroll
-    for (int j = 0; j < A; ++j) vp[(Idx)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
+    for (int j = 0; j < A; ++j) {
+      if constexpr (SPLIT) {
+        __nv_bfloat16 p0, p1, p2;
+        split_bf16x3(res[j], p0, p1, p2);
+        Tst* q = vp + (Idx)(i * A + j) * plane;
+        q[0] = p0;
+        q[a.c] = p1;
+        q[2 * a.c] = p2;
+      } else {
+        vp[(Idx)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
+      }
+    }
   }
 }
 

@@ -60,6 +60,59 @@ __global__ void wino_filter_kernel(const Tin* __restrict__ w, long long w_row_st
   }
 }
 
+// Filter transform for the split-bf16 fp32 GEMM: U''[xi][o][6C] bf16, the six
+// C-wide segments holding the parts (b0, b1, b0, b2, b1, b0) of the fp32 value,
+// against V's parts (a0, a0, a1, a0, a1, a2): the products a_i b_j with
+// i + j <= 2 in one K = 6C reduction.
+template <int M, typename Tin>
+__global__ void wino_filter_split_kernel(const Tin* __restrict__ w, long long w_row_stride, int O, int C,
+                                         __nv_bfloat16* __restrict__ u) {
+  constexpr int A = Wino<M>::A;
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)O * C) return;
+  int o = (int)(idx / C), c = (int)(idx - (long long)o * C);
+  const Tin* wp = w + (long long)o * w_row_stride + c;
+  float g[3][3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) g[i][j] = Store<Tin>::to_f32(wp[(long long)(i * 3 + j) * C]);
+  float t[A][3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    float col[3] = {g[0][j], g[1][j], g[2][j]}, r[A];
+    Wino<M>::g(col, r);
+#pragma unroll
+    for (int i = 0; i < A; ++i) t[i][j] = r[i];
+  }
+  const long long plane = (long long)O * 6 * C;
+  __nv_bfloat16* up = u + (long long)o * 6 * C + c;
+#pragma unroll
+  for (int i = 0; i < A; ++i) {
+    float r[A];
+    Wino<M>::g(t[i], r);
+#pragma unroll
+    for (int j = 0; j < A; ++j) {
+      __nv_bfloat16 b[3];
+      split_bf16x3(r[j], b[0], b[1], b[2]);
+      __nv_bfloat16* q = up + (long long)(i * A + j) * plane;
+      q[0] = b[0];
+      q[C] = b[1];
+      q[2 * C] = b[0];
+      q[3 * C] = b[2];
+      q[4 * C] = b[1];
+      q[5 * C] = b[0];
+    }
+  }
+}
+
+template <int M, typename Idx>
+__global__ void __launch_bounds__(256)
+wino_input_split_kernel(const float* __restrict__ in, const WinoInArgs a, __nv_bfloat16* __restrict__ v) {
+  wino_input_block<M, float, __nv_bfloat16, Idx, 1>(in, a, v, blockIdx.x, threadIdx.x, threadIdx.y, blockDim.x,
+                                                    blockDim.y);
+}
+
 // Input transform: one thread per (tile, channel); threadIdx.x runs over
 // channels so loads and stores are coalesced.
 template <int M, typename Tin, typename Tst, typename Idx>
@@ -413,6 +466,40 @@ cudaError_t launch_wino_filter(const void* w, long long w_row_stride, int o, int
       });
     });
   });
+}
+
+cudaError_t launch_wino_filter_split(const float* w, long long w_row_stride, int o, int c, void* u,
+                                     cudaStream_t s) {
+  long long n = (long long)o * c;
+  if (n == 0) return cudaSuccess;
+  wino_filter_split_kernel<6, float><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      w, w_row_stride, o, c, static_cast<__nv_bfloat16*>(u));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wino_input_split(const float* in, const Geom& g, int n0, long long t_count, void* v,
+                                    long long t_tile, cudaStream_t s) {
+  constexpr int m = 6;
+  WinoInArgs a{};
+  a.h = g.h; a.w = g.w; a.c = g.c; a.ph = g.ph; a.pw = g.pw;
+  a.tiles_h = (g.oh + m - 1) / m;
+  a.tiles_w = (g.ow + m - 1) / m;
+  a.in_img_stride = g.in_img_stride;
+  a.n0 = n0;
+  a.t_base = 0;
+  a.t_count = t_count;
+  a.t_stride = t_tile;
+  if (a.t_count == 0) return cudaSuccess;
+  const int bx = g.c >= 64 ? 64 : 32;
+  dim3 block(bx, 256 / bx);
+  const long long blocks = ((a.t_count + block.y - 1) / block.y) * ((g.c + bx - 1) / bx);
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31) && 64LL * t_tile * 3 * g.c < (1LL << 31);
+  if (idx32)
+    wino_input_split_kernel<m, int><<<(unsigned)blocks, block, 0, s>>>(in, a, static_cast<__nv_bfloat16*>(v));
+  else
+    wino_input_split_kernel<m, long long><<<(unsigned)blocks, block, 0, s>>>(in, a, static_cast<__nv_bfloat16*>(v));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_wino_input(const void* in, const Geom& g, int n0, long long t_base, long long t_count, int m,
