@@ -169,10 +169,16 @@ def kernel_work(conv, plan):
             # round trips through its per-CTA scratch
             add("wino_fused", 2.0 * a2 * T * s.c * s.o, in_b + out_b + 2 * a2 * T * (s.c + s.o) * 4)
             return w
-        add("wino_input", 0.0, in_b + a2 * T * s.c * st)
+        # the split-bf16 route writes V as three bf16 parts (6 bytes per value)
+        add("wino_input", 0.0, in_b + a2 * T * s.c * (6 if plan.get("winograd_split_bf16") else st))
         gk = "wino_gemm_tc" if plan["engine"] == "tcgen05" else "wino_gemm_simt"
-        # M is fp32 on the FFMA path and in the 16-bit operand type on the tensor-core path
-        add(gk, 2.0 * a2 * T * s.c * s.o, a2 * T * (s.c * st + s.o * st))
+        if plan.get("winograd_split_bf16"):
+            # six bf16 products per fp32 product on the tensor cores: 3C bf16 parts of V read,
+            # fp32 M written
+            add("wino_gemm_tc", 6 * 2.0 * a2 * T * s.c * s.o, a2 * T * (3 * s.c * 2 + s.o * 4))
+        else:
+            # M is fp32 on the FFMA path and in the 16-bit operand type on the tensor-core path
+            add(gk, 2.0 * a2 * T * s.c * s.o, a2 * T * (s.c * st + s.o * st))
         add("wino_output", 0.0, a2 * T * s.o * st + out_b)
     else:
         k = "tc_conv" if plan["engine"] == "tcgen05" else "simt_conv"
@@ -437,6 +443,9 @@ PER_CONFIG = [
     ("config4_wide3_f16_winograd", "wide3_f16", "winograd", False),
     ("config5_conv3d_bf16", "conv3d_bf16", "auto", False),
     ("config5_conv3d_f32", "conv3d_f32", "auto", False),
+    # config 2 with the fp32 Winograd GEMM on the tensor cores over split-bf16 operands
+    # (fp32-accurate emulation, not the default; the headline line keeps FFMA arithmetic)
+    ("config2_f32_gemm_split_bf16", "winograd_f32", "auto", False, {"B200CONV_WINOGRAD_SPLIT_BF16": "1"}),
 ]
 
 
@@ -614,7 +623,20 @@ def kernels_and_roofline(bench, prof, steps, peaks, fp32_pk, wl_name=None):
     return kernels, roof
 
 
-def per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, fp32_pk, min_steps):
+def per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, fp32_pk, min_steps, env=None):
+    old_env = {k: os.environ.get(k) for k in (env or {})}
+    os.environ.update(env or {})
+    try:
+        return _per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, fp32_pk, min_steps, env)
+    finally:
+        for k, v in old_env.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+def _per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, fp32_pk, min_steps, env):
     import torch
     bench = Bench(wl_name, algo, dev, stream)
     for _ in range(3):
@@ -625,6 +647,12 @@ def per_config_entry(key, wl_name, algo, use_graph, dev, stream, world, peaks, f
     steps = int(min(2000, max(min_steps, math.ceil(400.0 / max(one, 1e-3)))))
     entry = {"workload": bench.desc, "algo": algo, "dtype": bench.dtype, "convs": len(bench.items),
              "flops_per_step": bench.total_flops}
+    if env:
+        entry["env"] = dict(env)
+    if any(plan.get("winograd_split_bf16") for *_, plan, _ in bench.items):
+        entry["arithmetic"] = ("fp32 transforms; the Winograd GEMM on the tensor cores over split-bf16 operands "
+                               "(each fp32 value the exact sum of three bf16 parts, six bf16 products per fp32 "
+                               "product accumulated in fp32): fp32-accurate emulation, not FFMA arithmetic")
     barrier(world)
     with ClockSampler(dev.index or 0) as clk:
         ms_eager = statistics.median(bench.timed(steps))
@@ -841,12 +869,12 @@ def main():
     if not args.no_per_config:
         only = {k for k in args.per_config_only.split(",") if k}
         per_config = {}
-        for key, wl, algo, use_graph in PER_CONFIG:
+        for key, wl, algo, use_graph, *rest in PER_CONFIG:
             if only and key not in only:
                 continue
             try:
                 per_config[key] = per_config_entry(key, wl, algo, use_graph, dev, stream, world, peaks, fp32_pk,
-                                                   min_steps=10)
+                                                   min_steps=10, env=rest[0] if rest else None)
             except Exception as exc:      # report, never hide, a failed entry
                 per_config[key] = {"error": f"{type(exc).__name__}: {exc}"}
         assert B.conv_check(sptr) == 0

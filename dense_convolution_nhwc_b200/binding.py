@@ -65,6 +65,7 @@ class ConvPlan(ctypes.Structure):
                 ("tile_n", ctypes.c_int), ("winograd_m", ctypes.c_int), ("batch_tile", ctypes.c_int),
                 ("num_batch_tiles", ctypes.c_int), ("channel_pad", ctypes.c_int), ("packed_taps", ctypes.c_int),
                 ("k_split", ctypes.c_int), ("taps", ctypes.c_int), ("winograd_fused", ctypes.c_int),
+                ("winograd_split_bf16", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t)]
 
     def as_dict(self) -> dict:
@@ -73,7 +74,7 @@ class ConvPlan(ctypes.Structure):
                 "tile_m": self.tile_m, "tile_n": self.tile_n, "winograd_m": self.winograd_m,
                 "batch_tile": self.batch_tile, "num_batch_tiles": self.num_batch_tiles,
                 "channel_pad": self.channel_pad, "packed_taps": self.packed_taps, "k_split": self.k_split, "taps": self.taps,
-                "winograd_fused": self.winograd_fused,
+                "winograd_fused": self.winograd_fused, "winograd_split_bf16": self.winograd_split_bf16,
                 "workspace_bytes": int(self.workspace_bytes)}
 
 

@@ -415,7 +415,8 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->wino_store = store;
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
-      s->tile_n = tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
+      s->tile_n = split ? (g.o <= 96 ? 96 : (g.o <= 128 ? 128 : 256))
+                  : tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
       s->tile_m = tc_gemm && !split && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o,
                                                      s->tile_n, (g.c + 63) / 64, p) ? 256 : 128;
       s->chunk = (!tc_gemm && kF32VTileMajor && g.c % 4 == 0) ? winograd_chunk_tiles(g, m, p) : 0;
@@ -517,6 +518,7 @@ void fill_plan(const Sel& s, conv_plan_t* plan, int taps, size_t ws) {
   plan->k_split = s.ksplit;
   plan->taps = taps;
   plan->winograd_fused = s.fused ? 1 : 0;
+  plan->winograd_split_bf16 = s.split_bf16 ? 1 : 0;
   plan->workspace_bytes = ws;
 }
 
@@ -540,10 +542,10 @@ const char* algo_name(conv_algo_t a) {
 void log_plan(const char* op, const char* shape, conv_dtype_t dt, const Sel& s, const char* path, size_t ws) {
   std::fprintf(stderr,
                "b200conv: %s %s %s -> algo=%s engine=%s path=%s tile=%dx%d winograd_m=%d batch_tile=%d "
-               "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d fused=%d workspace=%zu\n",
+               "batch_tiles=%d channel_pad=%d packed_taps=%d k_split=%d fused=%d split_bf16=%d workspace=%zu\n",
                op, shape, dtype_name(dt), algo_name(s.algo), s.engine == CONV_ENGINE_TCGEN05 ? "tcgen05" : "simt",
                path, s.tile_m, s.tile_n, s.wino_m, s.nb, s.ntiles, s.cpad, s.fpack ? 2 : (s.wpack ? 1 : 0), s.ksplit,
-               s.fused ? 1 : 0, ws);
+               s.fused ? 1 : 0, s.split_bf16 ? 1 : 0, ws);
 }
 
 // ------------------------------- execution -----------------------------------

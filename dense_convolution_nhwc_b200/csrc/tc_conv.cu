@@ -56,7 +56,10 @@ template <int BN, int CG = 1> struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = (BN / CG) * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;           // two fp32 accumulators
+  // two fp32 accumulators, ACC_COLS apart; the allocation is a power of two
+  // columns (BN = 96: 256 columns, the accumulators at 0 and 128)
+  static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
+  static constexpr int ACC_COLS = TMEM_COLS / 2;
   static constexpr int BAR_BYTES = 256;
   // The epilogue stages each warp's output chunk for a TMA store: 32 rows of
   // 128 bytes (32 fp32 or 64 16-bit columns), 4 warps x 2 buffers, 128-byte swizzled
@@ -322,7 +325,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_COLS);
         int nks = ksteps;
         if (MODE != 0 && a.ksplit > 1) {
           const int b = (int)(tile / a.n_tiles / a.m_tiles);
@@ -397,7 +400,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         uint32_t rr[EPI / 32][32];
 #pragma unroll
         for (int h = 0; h < EPI / 32; ++h) {
-          const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cg + 32 * h);
+          const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS + cg + 32 * h);
           TMEM_LD32(taddr, rr[h]);
         }
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -1198,6 +1201,8 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   }
   CUtensorMap tD;
   a.tma_store = encode_store_map(&tD, bg.d, CONV_F32, bg.o, bg.t, bg.batches) ? 1 : 0;
+  if (dt == CONV_BF16 && tile_n == 96)
+    return launch_kernel<96, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);

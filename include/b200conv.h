@@ -132,7 +132,9 @@ typedef struct {
  * of that many tiles (pipelined transform / GEMM passes; 0 or unset: off);
  * B200CONV_WINOGRAD_FUSED=1 runs the fp32 Winograd F(6x6,3x3) path as one
  * persistent kernel whenever the shape allows (=0 or unset: three launches);
- * B200CONV_WINOGRAD_FUSED_GRID=<ctas> runs that kernel on fewer CTAs.
+ * B200CONV_WINOGRAD_FUSED_GRID=<ctas> runs that kernel on fewer CTAs;
+ * B200CONV_WINOGRAD_SPLIT_BF16=1 runs the fp32 Winograd GEMM on the tensor
+ * cores over split-bf16 operands (fp32 accuracy; C a multiple of 64, O of 4).
  */
 typedef struct {
     conv_algo_t algo;                     /* CONV_ALGO_AUTO: let the selector choose */
@@ -157,6 +159,9 @@ typedef struct {
     int winograd_fused;        /* 1 if the fp32 Winograd F(6x6,3x3) runs as one persistent kernel (input
                                   transform, FFMA GEMM and output transform overlapped inside each CTA,
                                   per-CTA scratch in the workspace); else 0 */
+    int winograd_split_bf16;   /* 1 if the fp32 Winograd GEMM runs on the tensor cores over split-bf16
+                                  operands (each fp32 value the exact sum of three bf16 parts, the six
+                                  products a_i b_j with i + j <= 2 accumulated in fp32); else 0 */
     size_t workspace_bytes;    /* bytes the caller must pass to *_forward */
 } conv_plan_t;
 

@@ -111,10 +111,10 @@ def test_per_config_block_covers_every_config():
     config-2 headline, every dtype the configs name, and every workload it
     names resolves (no device needed)."""
     keys = [k for k, *_ in bench.PER_CONFIG]
-    for cfg in ("config1_", "config3_", "config4_", "config5_"):
+    for cfg in ("config1_", "config2_", "config3_", "config4_", "config5_"):
         assert any(k.startswith(cfg) for k in keys), cfg
     seen = set()
-    for key, wl, algo, _ in bench.PER_CONFIG:
+    for key, wl, algo, _, *env in bench.PER_CONFIG:
         desc, convs, dt = bench.workload(wl)
         assert convs and algo in ("auto", "implicit", "winograd", "direct")
         seen.add((key.split("_")[0], dt))
@@ -124,3 +124,17 @@ def test_per_config_block_covers_every_config():
     _, convs, _ = bench.workload("wide_bf16")
     assert all(c.shape.o >= 512 and c.shape.n * c.shape.oh * c.shape.ow >= 16384 for c in convs)
     assert all(c.shape.stride == (1, 1) and c.shape.dilation == (1, 1) for c in convs)
+
+
+def test_split_bf16_work_counts_the_bf16_products():
+    """The split-bf16 GEMM route's roofline counts the tensor cores' six bf16
+    products per fp32 product; the conv's own FLOPs (the metric) do not change."""
+    s = synth.WINOGRAD_F32
+    p = plan2d(s, "f32")
+    p["engine"] = "tcgen05"
+    p["winograd_split_bf16"] = 1
+    w = bench.kernel_work(bench.Conv(s, "f32", "uniform"), p)
+    T = 40 * 86 * 86
+    assert w["wino_gemm_tc"][0] == 6 * 2.0 * 64 * T * 192 * 96
+    assert w["wino_gemm_tc"][1] == 64 * T * (3 * 192 * 2 + 96 * 4)
+    assert bench.kernel_bound("wino_gemm_tc") == "tensor"
