@@ -264,7 +264,7 @@ struct WinoLayout {
 
 // chunk > 0: the batch tile's tiles pass through V and M in chunks of at most
 // `chunk` tiles, so V and M hold one chunk.
-// split: the split-bf16 fp32 GEMM's operands, U [a2][O][6C] and V [a2][T][3C]
+// split: the split-bf16 fp32 GEMM's operands, U [a2][O][3C] and V [a2][T][3C]
 // in bf16, M [a2][T][O] fp32.
 WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m, long long nb, long long chunk = 0,
                            bool split = false) {
@@ -274,7 +274,7 @@ WinoLayout winograd_layout(const Geom& g, conv_dtype_t store, bool cmajor, int m
   if (split) {
     const long long t = nb * L.tiles_per_img;
     L.per_img = (size_t)(a2 * L.tiles_per_img) * ((size_t)g.c * 6 + (size_t)g.o * 4);
-    L.u_bytes = align256((size_t)(a2 * g.o * g.c) * 12);
+    L.u_bytes = align256((size_t)(a2 * g.o * g.c) * 6);
     L.v_bytes = align256((size_t)(a2 * t * g.c) * 6);
     L.m_bytes = align256((size_t)(a2 * t * g.o) * 4);
     return L;
@@ -326,8 +326,8 @@ long long winograd_chunk_tiles(const Geom& g, int m, const conv_device_props_t& 
 
 // The fp32 Winograd GEMM on the tensor cores over split-bf16 operands: each fp32
 // value is the exact sum of three bf16 parts, and the six products a_i b_j with
-// i + j <= 2 are accumulated in fp32 (TMEM) in one K = 6C reduction, which
-// keeps fp32 accuracy (the dropped products are below 2^-24 of the result).
+// i + j <= 2 are accumulated in fp32 (TMEM), which keeps fp32 accuracy (the
+// dropped products are below 2^-24 of the result).
 // It needs F(6x6,3x3), a tcgen05 device, C a multiple of 64 and O of 4.
 // B200CONV_WINOGRAD_SPLIT_BF16=1 turns it on (a test hook read on every call).
 bool winograd_split_wanted(const Geom& g, conv_dtype_t dt, int m, const conv_device_props_t& p) {
@@ -415,7 +415,7 @@ conv_status_t select2d(const Geom& g, conv_dtype_t dt, const conv_device_props_t
       s->wino_store = store;
       s->nb = (int)nb;
       s->ntiles = (int)((g.n + nb - 1) / nb);
-      s->tile_n = split ? (g.o <= 96 ? 96 : (g.o <= 128 ? 128 : 256))
+      s->tile_n = split ? (g.o <= 96 ? 96 : 128)
                   : tc_gemm ? (g.o <= 128 ? 128 : 256) : wino_gemm_f32_tile_n(g.o);
       s->tile_m = tc_gemm && !split && tc_pair_tiles(nb * tiles_per_img, (long long)(m + 2) * (m + 2), g.o,
                                                      s->tile_n, (g.c + 63) / 64, p) ? 256 : 128;

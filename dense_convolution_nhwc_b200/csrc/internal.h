@@ -54,8 +54,8 @@ struct BatchedGemm {
   const void* b;        // [batches][O][C]
   void* d;              // [batches][T][O] in d_dt
   conv_dtype_t d_dt;
-  // split-bf16 fp32 GEMM: a is [batches][T][3C] (the three bf16 parts of each
-  // value), b is [batches][O][6C] (parts b0 b1 b0 b2 b1 b0), d is fp32; K = 6C
+  // split-bf16 fp32 GEMM: a is [batches][T][3C] and b is [batches][O][3C] (the
+  // three bf16 parts of each value side by side), d is fp32
   bool split_bf16 = false;
 };
 
@@ -133,7 +133,7 @@ cudaError_t launch_wino_gemm_f32(const float* a, const float* b, float* d, int b
                                  long long lda, long long ldb, bool a_tmajor, cudaStream_t s);
 int wino_gemm_f32_tile_n(int o);
 
-// Split-bf16 fp32 Winograd F(6x6,3x3): the filter transform as U''[64][O][6C]
+// Split-bf16 fp32 Winograd F(6x6,3x3): the filter transform as U'[64][O][3C]
 // bf16 and the input transform as V'[64][t_tile][3C] bf16 (fp32 input).
 cudaError_t launch_wino_filter_split(const float* w, long long w_row_stride, int o, int c, void* u,
                                      cudaStream_t s);

@@ -51,10 +51,14 @@ constexpr int THREADS = 192;
 
 // CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a CTA pair computes a
 // 256 x BN tile, each CTA holding 128 rows of A and BN/2 rows of B per stage.
-template <int BN, int CG = 1> struct Cfg {
-  static constexpr int STAGES = CG == 2 ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = (BN / CG) * BK * 2;
+// PARTS = 3: the split-bf16 batched GEMM, whose stage holds the three bf16
+// parts of one 64-wide K block of A and of B.
+template <int BN, int CG = 1, int PARTS = 1> struct Cfg {
+  static constexpr int STAGES = PARTS == 3 ? 2 : (CG == 2 ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
+  static constexpr int A_PART = BM * BK * 2;
+  static constexpr int B_PART = (BN / CG) * BK * 2;
+  static constexpr int A_BYTES = PARTS * A_PART;
+  static constexpr int B_BYTES = PARTS * B_PART;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // two fp32 accumulators, ACC_COLS apart; the allocation is a power of two
   // columns (BN = 96: 256 columns, the accumulators at 0 and 128)
@@ -86,9 +90,8 @@ struct TcArgs {
   int tma_store;               // write 32-row x 128-byte chunks with TMA stores through tmD
   int cluster_reduce;          // split-K whose ksplit CTAs of a tile form a cluster: rank 0 sums the
                                // others' fp32 partials from their shared memory and writes out
-  int split_cb;                // batched GEMM on split-bf16 operands: A's K holds three parts of C
-                               // (split_cb 64-wide blocks each), B's K six (b0 b1 b0 b2 b1 b0); K-block
-                               // kb reads A's part (0,0,1,0,1,2)[kb / split_cb]; 0: plain K
+  int split_cb;                // MODE 3 (split-bf16 batched GEMM): 64-wide K blocks per part; A and B
+                               // rows hold three parts of C side by side
   int serial_reduce;           // split-K whose last-arriving split of a tile sums the fp32 partials
   float* partial;              // serial_reduce: [ksplit][m_rows][ocols] fp32 partials
   long long part_batch;        // serial_reduce: elements between splits' partials
@@ -99,13 +102,16 @@ struct TcArgs {
 
 // --------------------------------- kernel -----------------------------------
 
-// MODE 0: batched GEMM (tiled A); 1: conv2d (4D im2col A); 2: conv3d (5D im2col A).
+// MODE 0: batched GEMM (tiled A); 1: conv2d (4D im2col A); 2: conv3d (5D im2col A);
+// 3: batched GEMM over split-bf16 operands (each stage the three parts of a K
+// block of A and of B; the six products a_i b_j with i + j <= 2 per stage).
 // CG = 2: CTA pairs (clusters of 2) on 256-row tiles, a.m_tiles counting 256-row tiles.
 template <int BN, int MODE, typename TIn, typename TOut, int CG = 1>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const TcArgs a) {
-  using C = Cfg<BN, CG>;
+  using C = Cfg<BN, CG, MODE == 3 ? 3 : 1>;
+  static_assert(MODE != 3 || CG == 1, "split-bf16 GEMM on single CTAs");
   constexpr int STORE_BYTES = C::STORE_BYTES;
   constexpr uint32_t IDESC = make_idesc<BN, BM * CG>(std::is_same<TIn, __nv_bfloat16>::value ? 1u : 0u);
   static_assert(CG == 1 || CG == 2, "CTA group");
@@ -187,14 +193,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const long long total_tiles = (long long)a.batches * a.m_tiles * a.n_tiles;
   const int ksteps = a.taps * a.kb_per_tap;
 
-  // A's K coordinate of K-block kb (MODE 0): the split-bf16 GEMM reads part
-  // (0,0,1,0,1,2)[kb / split_cb] of A for the six B segments
-  auto a_kcoord = [&](int kb) {
-    if (MODE != 0 || a.split_cb == 0) return kb * BK;
-    const int term = kb / a.split_cb, sub = kb - term * a.split_cb;
-    const int part = (0x210100 >> (4 * term)) & 0xF;
-    return (part * a.split_cb + sub) * BK;
-  };
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0) {
@@ -211,7 +209,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // this CTA's 128 rows of the tile (the second half of a pair's 256)
         const long long row0 = (long long)mt * (BM * CG) + (long long)prank * BM;
         int img = 0, wx = 0, hy = 0, dz = 0;
-        if (MODE != 0) {
+        if (MODE == 1 || MODE == 2) {
           // first output pixel of the tile -> its window's corner in the input
           const long long m0 = row0;
           const long long ohw = (long long)a.oh * a.ow;
@@ -228,7 +226,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           img = (int)fr;
         }
         int ks_lo = 0, ks_hi = ksteps;
-        if (MODE != 0 && a.ksplit > 1) {
+        if ((MODE == 1 || MODE == 2) && a.ksplit > 1) {
           ks_lo = (int)((long long)ksteps * b / a.ksplit);
           ks_hi = (int)((long long)ksteps * (b + 1) / a.ksplit);
         }
@@ -259,7 +257,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                       (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
               tma_load_3d_pair(dB, &tmB, fb0, kb * BK, tap, ncol);
             } else {
-              tma_load_3d_pair(dA, &tmA, fb0, a_kcoord(kb), (int)row0, b);
+              tma_load_3d_pair(dA, &tmA, fb0, kb * BK, (int)row0, b);
               tma_load_3d_pair(dB, &tmB, fb0, kb * BK, ncol, b);
             }
             ++issued;
@@ -283,8 +281,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tma_load_im2col_5d(dA, &tmA, fb, kb * BK, wx, hy, dz, img, (uint16_t)(kx * a.dw),
                                (uint16_t)(ky * a.dh), (uint16_t)(kz * a.dd));
             tma_load_3d(dB, &tmB, fb, kb * BK, tap, nt * BN);
+          } else if (MODE == 3) {
+            // the three parts of K block kb of A and of B, one barrier for all six
+#pragma unroll
+            for (int pt = 0; pt < 3; ++pt) {
+              tma_load_3d(dA + pt * C::A_PART, &tmA, fb, (pt * a.split_cb + kb) * BK, (int)row0, b);
+              tma_load_3d(dB + pt * C::B_PART, &tmB, fb, (pt * a.split_cb + kb) * BK, nt * BN, b);
+            }
           } else {
-            tma_load_3d(dA, &tmA, fb, a_kcoord(kb), (int)row0, b);
+            tma_load_3d(dA, &tmA, fb, kb * BK, (int)row0, b);
             tma_load_3d(dB, &tmB, fb, kb * BK, nt * BN, b);
           }
           ++issued;
@@ -327,7 +332,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::ACC_COLS);
         int nks = ksteps;
-        if (MODE != 0 && a.ksplit > 1) {
+        if ((MODE == 1 || MODE == 2) && a.ksplit > 1) {
           const int b = (int)(tile / a.n_tiles / a.m_tiles);
           nks = (int)((long long)ksteps * (b + 1) / a.ksplit) - (int)((long long)ksteps * b / a.ksplit);
         }
@@ -344,6 +349,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int k = 0; k < BK / 16; ++k)
               tc_mma_pair(d_tmem, sdesc(aa + 32u * k), sdesc(bb + 32u * k), IDESC, (ks | k) != 0 ? 1u : 0u);
             tc_commit_pair_both(empty_bar(stage));      // frees the stage in both CTAs
+          } else if constexpr (MODE == 3) {
+            // products a_i b_j, i + j <= 2: A parts (0,0,1,0,1,2) against B parts (0,1,0,2,1,0)
+#pragma unroll
+            for (int term = 0; term < 6; ++term) {
+              const uint32_t ai = (0x210100u >> (4 * term)) & 0xFu, bj = (0x012010u >> (4 * term)) & 0xFu;
+#pragma unroll
+              for (int k = 0; k < BK / 16; ++k)
+                tc_mma(d_tmem, sdesc(aa + ai * C::A_PART + 32u * k), sdesc(bb + bj * C::B_PART + 32u * k), IDESC,
+                       (ks | term | k) != 0 ? 1u : 0u);
+            }
+            tc_commit(empty_bar(stage));
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
@@ -765,7 +781,7 @@ template <int BN, int MODE, typename TIn, typename TOut>
 cudaError_t launch_kernel(const CUtensorMap& A, const CUtensorMap& B, const TcArgs& a, int sm_count,
                           cudaStream_t s, const CUtensorMap* D = nullptr) {
   auto k = tc_gemm_kernel<BN, MODE, TIn, TOut>;
-  constexpr int smem = Cfg<BN>::template smem<TOut>();
+  constexpr int smem = Cfg<BN, 1, MODE == 3 ? 3 : 1>::template smem<TOut>();
   static_assert(smem <= 232448, "shared memory budget");
   cudaError_t e = set_smem(k, smem);
   if (e != cudaSuccess) return e;
@@ -1154,8 +1170,8 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
     return cudaErrorNotSupported;
   if (bg.split_bf16 && (dt != CONV_BF16 || bg.c % BK != 0 || bg.d_dt != CONV_F32)) return cudaErrorNotSupported;
   if (bg.t == 0 || bg.batches == 0) return cudaSuccess;
-  // K extents of A and B (the split-bf16 GEMM: 3C parts of A against 6C of B)
-  const long long ka = bg.split_bf16 ? 3LL * bg.c : bg.c, kb_ = bg.split_bf16 ? 6LL * bg.c : bg.c;
+  // K extents of A and B (the split-bf16 GEMM: rows of three C-wide parts)
+  const long long ka = bg.split_bf16 ? 3LL * bg.c : bg.c, kb_ = ka;
   CUtensorMap tA, tB;
   if (!encode_3d(&tA, dt, bg.a, ka, bg.t, bg.batches, (uint64_t)ka * 2, (uint64_t)bg.t * ka * 2, BK, BM, 1))
     return cudaErrorInvalidValue;
@@ -1165,7 +1181,7 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   a.m_tiles = (bg.t + BM - 1) / BM;
   a.n_tiles = (bg.o + tile_n - 1) / tile_n;
   a.batches = bg.batches;
-  a.kb_per_tap = (int)((kb_ + BK - 1) / BK);
+  a.kb_per_tap = bg.split_bf16 ? bg.c / BK : (int)((kb_ + BK - 1) / BK);
   a.split_cb = bg.split_bf16 ? bg.c / BK : 0;
   a.taps = 1;
   a.kw = 1; a.dh = 1; a.dw = 1;
@@ -1201,8 +1217,11 @@ cudaError_t launch_tc_batched_gemm(const BatchedGemm& bg, conv_dtype_t dt, int t
   }
   CUtensorMap tD;
   a.tma_store = encode_store_map(&tD, bg.d, CONV_F32, bg.o, bg.t, bg.batches) ? 1 : 0;
-  if (dt == CONV_BF16 && tile_n == 96)
-    return launch_kernel<96, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
+  if (bg.split_bf16) {
+    if (tile_n != 96 && tile_n != 128) return cudaErrorInvalidValue;
+    return tile_n == 96 ? launch_kernel<96, 3, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
+                        : launch_kernel<128, 3, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);
+  }
   if (dt == CONV_BF16)
     return tile_n == 256 ? launch_kernel<256, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD)
                          : launch_kernel<128, 0, __nv_bfloat16, float>(tA, tB, a, sm_count, s, &tD);

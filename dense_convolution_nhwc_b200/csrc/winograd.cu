@@ -60,10 +60,8 @@ __global__ void wino_filter_kernel(const Tin* __restrict__ w, long long w_row_st
   }
 }
 
-// Filter transform for the split-bf16 fp32 GEMM: U''[xi][o][6C] bf16, the six
-// C-wide segments holding the parts (b0, b1, b0, b2, b1, b0) of the fp32 value,
-// against V's parts (a0, a0, a1, a0, a1, a2): the products a_i b_j with
-// i + j <= 2 in one K = 6C reduction.
+// Filter transform for the split-bf16 fp32 GEMM: U'[xi][o][3C] bf16, the three
+// C-wide segments holding the parts (b0, b1, b2) of the fp32 value.
 template <int M, typename Tin>
 __global__ void wino_filter_split_kernel(const Tin* __restrict__ w, long long w_row_stride, int O, int C,
                                          __nv_bfloat16* __restrict__ u) {
@@ -85,8 +83,8 @@ __global__ void wino_filter_split_kernel(const Tin* __restrict__ w, long long w_
 #pragma unroll
     for (int i = 0; i < A; ++i) t[i][j] = r[i];
   }
-  const long long plane = (long long)O * 6 * C;
-  __nv_bfloat16* up = u + (long long)o * 6 * C + c;
+  const long long plane = (long long)O * 3 * C;
+  __nv_bfloat16* up = u + (long long)o * 3 * C + c;
 #pragma unroll
   for (int i = 0; i < A; ++i) {
     float r[A];
@@ -98,10 +96,7 @@ __global__ void wino_filter_split_kernel(const Tin* __restrict__ w, long long w_
       __nv_bfloat16* q = up + (long long)(i * A + j) * plane;
       q[0] = b[0];
       q[C] = b[1];
-      q[2 * C] = b[0];
-      q[3 * C] = b[2];
-      q[4 * C] = b[1];
-      q[5 * C] = b[0];
+      q[2 * C] = b[2];
     }
   }
 }
