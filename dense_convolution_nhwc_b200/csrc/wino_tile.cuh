@@ -9,6 +9,8 @@
 
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "wino_1d.cuh"
 
@@ -101,8 +103,12 @@ __device__ __forceinline__ void wino_input_block(const Tin* __restrict__ in, con
 #pragma unroll
     for (int i = 0; i < A; ++i) tt[i][j] = res[i];
   }
-  const Idx rowc = SPLIT ? (Idx)3 * a.c : (Idx)a.c;
-  const Idx plane = (Idx)(a.t_stride * rowc);
+  // V offsets: Idx, except in the split form, whose three-part rows make the
+  // plane set 3x larger; there they are 64-bit so that Idx (int for every
+  // image below 2^31 elements) bounds only the input offsets
+  using VIdx = typename std::conditional<SPLIT != 0, long long, Idx>::type;
+  const VIdx rowc = SPLIT ? (VIdx)3 * a.c : (VIdx)a.c;
+  const VIdx plane = (VIdx)(a.t_stride * rowc);
   Tst* vp = v + t * rowc + c;
 #pragma unroll
   for (int i = 0; i < A; ++i) {
@@ -113,12 +119,12 @@ __device__ __forceinline__ void wino_input_block(const Tin* __restrict__ in, con
       if constexpr (SPLIT) {
         __nv_bfloat16 p0, p1, p2;
         split_bf16x3(res[j], p0, p1, p2);
-        Tst* q = vp + (Idx)(i * A + j) * plane;
+        Tst* q = vp + (VIdx)(i * A + j) * plane;
         q[0] = p0;
         q[a.c] = p1;
         q[2 * a.c] = p2;
       } else {
-        vp[(Idx)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
+        vp[(VIdx)(i * A + j) * plane] = Store<Tst>::from_f32(res[j]);
       }
     }
   }

@@ -489,7 +489,9 @@ cudaError_t launch_wino_input_split(const float* in, const Geom& g, int n0, long
   dim3 block(bx, 256 / bx);
   const long long blocks = ((a.t_count + block.y - 1) / block.y) * ((g.c + bx - 1) / bx);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31) && 64LL * t_tile * 3 * g.c < (1LL << 31);
+  // int input offsets whenever one image (with a row of slack for the
+  // padding) stays below 2^31 elements; the V offsets are 64-bit in this form
+  const bool idx32 = g.in_img_stride + 4LL * g.w * g.c < (1LL << 31);
   if (idx32)
     wino_input_split_kernel<m, int><<<(unsigned)blocks, block, 0, s>>>(in, a, static_cast<__nv_bfloat16*>(v));
   else
