@@ -202,8 +202,8 @@ KERNEL_SOURCES = {
     "wino_fused": ["wino_fused_f32.cu", "wino_tile.cuh", "mbar.cuh", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "tc_conv": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"], "wino_gemm_tc": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "tc_conv3d": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
-    "wino_input": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
-    "wino_output": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino_input": ["winograd.cu", "wino_tile.cuh", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
+    "wino_output": ["winograd.cu", "wino_tile.cuh", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino_filter": ["winograd.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
     "wino3d_gemm_simt": ["wino_gemm_f32.cu"], "wino3d_gemm_tc": ["tc_conv.cu", "tc_ptx.cuh", "common.cuh"],
     "wino3d_input": ["winograd3d.cu", "wino_1d.cuh", "winograd_gen.cuh", "common.cuh"],
