@@ -111,6 +111,57 @@ def test_winograd_fused_rules(monkeypatch):
     assert plan2d(big)[1]["winograd_fused"] == 0
 
 
+def test_winograd_split_bf16_plan(monkeypatch):
+    """The fp32 Winograd GEMM over split-bf16 operands (B200CONV_WINOGRAD_SPLIT_BF16=1,
+    off by default): the tcgen05 engine on 96-column tiles for O = 96, and a workspace
+    of U [64][O][3C] and V [64][T][3C] in bf16 plus M [64][T][O] in fp32.  The batch
+    tile comes from the same 8 GiB budget: 64 * 7396 * (192 * 6 + 96 * 4) bytes per
+    image gives 11 images (11, 11, 11, 7)."""
+    monkeypatch.delenv("B200CONV_WINOGRAD_FUSED", raising=False)
+    assert plan2d(synth.WINOGRAD_F32)[1]["winograd_split_bf16"] == 0
+    monkeypatch.setenv("B200CONV_WINOGRAD_SPLIT_BF16", "1")
+    st, p = plan2d(synth.WINOGRAD_F32)
+    assert st == 0
+    assert p["algo"] == "winograd" and p["engine"] == "tcgen05" and p["winograd_m"] == 6
+    assert p["winograd_split_bf16"] == 1 and p["winograd_fused"] == 0
+    assert p["tile_n"] == 96 and p["tile_m"] == 128
+    tiles = 86 * 86
+    nb = (8 * 2 ** 30) // (64 * tiles * (192 * 6 + 96 * 4))
+    assert nb == 11 and p["batch_tile"] == nb and p["num_batch_tiles"] == 4
+    t = nb * tiles
+
+    def al(x):
+        return -(-x // 256) * 256
+
+    assert p["workspace_bytes"] == al(64 * 96 * 192 * 6) + al(64 * t * 192 * 6) + al(64 * t * 96 * 4)
+    # O > 96: 128-column tiles
+    wide = synth.Conv2dShape(2, 64, 64, 64, 128, 3, 3, (1, 1), (1, 1), (1, 1))
+    st, p = plan2d(wide, algo="winograd")
+    assert st == 0 and p["winograd_split_bf16"] == 1 and p["tile_n"] == 128
+
+
+def test_winograd_split_bf16_rules(monkeypatch):
+    """Only fp32 inputs with C % 64 == 0 and O % 4 == 0 on a compute-capability-10
+    device take it, and the persistent fp32 kernel's hook takes precedence."""
+    monkeypatch.delenv("B200CONV_WINOGRAD_FUSED", raising=False)
+    monkeypatch.setenv("B200CONV_WINOGRAD_SPLIT_BF16", "1")
+    big = synth.WINOGRAD_F32
+    assert plan2d(big, "f16")[1]["winograd_split_bf16"] == 0
+    assert plan2d(big, "bf16")[1]["winograd_split_bf16"] == 0
+    for c, o in ((96, 96), (64, 98)):
+        s = synth.Conv2dShape(2, 40, 40, c, o, 3, 3, (1, 1), (1, 1), (1, 1))
+        st, p = plan2d(s, algo="winograd")
+        assert st == 0 and p["algo"] == "winograd" and p["winograd_split_bf16"] == 0 and p["engine"] == "simt"
+    desc = B.make_desc2d(big.n, big.h, big.w, big.c, big.o, big.kh, big.kw, big.stride, big.pad, big.dilation)
+    p = B.ConvPlan()
+    hopper = B.DeviceProps(132, 9, 0, 80 * 2 ** 30)
+    assert B.conv2d_plan_for_props(desc, B.DTYPE["f32"], hopper, B.make_options(), p) == 0
+    assert p.as_dict()["winograd_split_bf16"] == 0
+    monkeypatch.setenv("B200CONV_WINOGRAD_FUSED", "1")
+    st, p = plan2d(big)
+    assert st == 0 and p["winograd_split_bf16"] == 0 and p["winograd_fused"] == 1
+
+
 def test_small_shape_takes_implicit_gemm():
     st, p = plan2d(synth.SMALL_F32)       # C + O = 64 < 256
     assert st == 0 and p["algo"] == "implicit" and p["engine"] == "simt"
