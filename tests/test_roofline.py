@@ -1,4 +1,4 @@
-"""The bench's roofline arithmetic without a GPU.
+"""The bench's roofline arithmetic and clock record without a GPU.
 
 For the dominant kernel of a step the bench reports the kernel's algorithmic
 work per launch (its FLOPs or bytes, from the plan the library will run) over
@@ -120,3 +120,27 @@ def test_conv_flops_are_the_direct_count():
     s = synth.WINOGRAD_F32
     cv = bench.Conv(s, "f32", "uniform")
     assert cv.flops == 2 * 40 * 512 * 512 * 96 * 192 * 9
+
+
+def test_clock_record_from_samples(tmp_path):
+    """The clock record of a timed region: the median SM clock under load, the
+    maximum, every throttle reason seen active in any sample, the peak power;
+    rows that are not full samples are skipped."""
+    p = tmp_path / "clocks.csv"
+    p.write_text(
+        "0, 1965, 1965, 640.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+        "0, 1590, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+        "0, 1800, 1965, 800.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+        "0, [N/A]\n")
+    cs = bench.ClockSampler(0)
+    cs.path = str(p)
+    rec = cs.summary()
+    assert rec["sm_mhz"] == 1800.0 and rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["sw_power_cap"] and rec["samples"] == 3 and rec["power_w_max"] == 990.0
+    assert not p.exists()                       # the sample file is removed once read
+    q = tmp_path / "hot.csv"
+    q.write_text("0, 1400, 1965, 700, 0x48, Active, Active, Not Active, Not Active\n")
+    cs.path = str(q)
+    assert cs.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    cs.path = str(tmp_path / "missing.csv")
+    assert cs.summary()["reasons"] == ["nvidia-smi unavailable"]
