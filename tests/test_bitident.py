@@ -12,9 +12,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from dense_convolution_nhwc_b200 import binding as B
 from dense_convolution_nhwc_b200 import synth
-from tests.gpu_util import check_conv2d
+from tests.gpu_util import as_f64, assert_close, check_conv2d
 
 pytestmark = pytest.mark.gpu
 
@@ -92,3 +93,37 @@ def test_large_workload_forced_tiles_bitwise():
     del implicit, ref, x, w
     torch.cuda.empty_cache()
     check_conv2d(s, "f32", dist="uniform")
+
+
+@pytest.mark.parametrize("dtype,shape,budget,small_tile", [
+    # F(6x6,3x3): 64 x 295,840 x 192 = 3.6e9 V elements in one 40-image tile (a 24 GiB budget)
+    ("f32", synth.WINOGRAD_F32, 24 * 2 ** 30, 7),
+    # F(2x2,3x3) on the tensor cores: 16 x 131,072 x 1024 = 2.1e9 V elements in one tile
+    ("bf16", synth.Conv2dShape(32, 128, 128, 1024, 256, 3, 3, (1, 1), (1, 1), (1, 1)), -1, 8),
+], ids=["f32", "bf16"])
+def test_plane_set_past_2_31_takes_64bit_offsets_bitwise(dtype, shape, budget, small_tile):
+    """A batch tile whose V plane set (alpha^2 x T x C elements) reaches 2^31 runs
+    its input transform with 64-bit offsets; the output equals the 32-bit-offset
+    run of smaller tiles bit for bit and matches the oracle on sampled pixels."""
+    m = 6 if dtype == "f32" else 2
+    tiles = -(-shape.oh // m) * -(-shape.ow // m)
+    a2 = (m + 2) ** 2
+    desc = B.make_desc2d(shape.n, shape.h, shape.w, shape.c, shape.o, shape.kh, shape.kw, shape.stride,
+                         shape.pad, shape.dilation)
+    big_opts = B.make_options("winograd", budget, shape.n)
+    plan = B.plan2d(desc, dtype, 0, big_opts)
+    assert plan["algo"] == "winograd" and plan["winograd_m"] == m
+    assert plan["batch_tile"] == shape.n and plan["num_batch_tiles"] == 1
+    assert a2 * shape.n * tiles * shape.c >= 2 ** 31 > a2 * small_tile * tiles * shape.c
+    x, w = synth.conv2d_inputs(shape, dtype, "uniform" if dtype == "f32" else "normal", 5, device="cuda")
+    big = B.conv2d(x, w, shape.stride, shape.pad, shape.dilation, options=big_opts)
+    small = run(x, w, shape, algo="winograd", winograd_tile_batch=small_tile)
+    torch.cuda.synchronize()
+    assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
+    iv = torch.int32 if dtype == "f32" else torch.int16
+    assert torch.equal(big.view(iv), small.view(iv))
+    del small
+    pix = synth.sample_pixels(shape.n, shape.oh, shape.ow, 4096, 11)
+    want = oracle.conv2d(x.cpu(), w.cpu(), dtype, shape.stride, shape.pad, shape.dilation, pixels=pix.numpy())
+    p = pix.long()
+    assert_close(as_f64(big[p[:, 0], p[:, 1], p[:, 2]]), want, dtype, shape.name())
