@@ -225,3 +225,25 @@ def test_bad_out_tensor_is_refused_before_any_launch():
             B.conv2d(x, w, 1, 1, 1, options=opts, out=out, workspace=ws)
     torch.cuda.synchronize()
     assert torch.isnan(out).all() and torch.isnan(o3.float()).all() and torch.isnan(o1).all()
+
+
+def test_plan_log_line(capfd, monkeypatch):
+    """B200CONV_LOG=1 (read on every call) prints one stderr line per forward call
+    with the shape, the dtype and the plan that runs; unset or 0 prints nothing."""
+    s = synth.Conv2dShape(2, 20, 20, 64, 96, 3, 3, (1, 1), (1, 1), (1, 1))
+    x, w = synth.conv2d_inputs(s, "bf16", "normal", 0, device="cuda")
+    capfd.readouterr()
+    monkeypatch.setenv("B200CONV_LOG", "1")
+    B.conv2d(x, w, 1, 1, 1)
+    B.conv2d(x.float(), w.float(), 1, 1, 1, options=B.make_options("winograd"))
+    torch.cuda.synchronize()
+    lines = [ln for ln in capfd.readouterr().err.splitlines() if ln.startswith("b200conv: ")]
+    assert len(lines) == 2, lines
+    assert "conv2d n2 20x20 64->96 k3x3 s1,1 p1,1 d1,1 bf16" in lines[0]
+    assert "algo=implicit engine=tcgen05" in lines[0] and "workspace=" in lines[0]
+    assert " f32 " in lines[1] and "algo=winograd engine=simt" in lines[1] and "winograd_m=6" in lines[1]
+    monkeypatch.setenv("B200CONV_LOG", "0")
+    B.conv2d(x, w, 1, 1, 1)
+    torch.cuda.synchronize()
+    assert "b200conv: " not in capfd.readouterr().err
+    assert B.conv_check(torch.cuda.current_stream().cuda_stream) == 0
